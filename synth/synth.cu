@@ -1,0 +1,120 @@
+// Device side of the seeded synthetic-input generator (test and bench
+// infrastructure, not part of the attention library).  The definition is the
+// one in synth/__init__.py: SplitMix64 output function (Steele, Lea, Flood,
+// OOPSLA 2014) over a counter stream, twelve 16-bit uniforms summed and
+// centred (Irwin-Hall), times 2^-16 * sigma (sigma a power of two, so exact),
+// rounded to bf16 with round-to-nearest-even.  The host regenerates any slice
+// bit for bit.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace {
+
+__host__ __device__ __forceinline__ uint64_t mix64(uint64_t z) {
+  z ^= z >> 30;
+  z *= 0xBF58476D1CE4E5B9ull;
+  z ^= z >> 27;
+  z *= 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  return z;
+}
+
+constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
+constexpr uint64_t kSalt = 0x5851F42D4C957F2Dull;
+constexpr int kMean12 = 393210;
+constexpr uint64_t kPosStride = 1ull << 20;
+
+__device__ __forceinline__ uint16_t gen_bf16(uint64_t key, uint64_t index, float scale) {
+  int acc = 0;
+#pragma unroll
+  for (int r = 0; r < 3; ++r) {
+    uint64_t w = mix64(key + (index * 3ull + (uint64_t)r + 1ull) * kGamma);
+#pragma unroll
+    for (int f = 0; f < 4; ++f) acc += (int)((w >> (16 * f)) & 0xFFFFull);
+  }
+  float x = (float)(acc - kMean12) * scale;   // exact: |acc - mean| < 2^20, scale a power of two
+  __nv_bfloat16 b = __float2bfloat16_rn(x);
+  return *reinterpret_cast<uint16_t*>(&b);
+}
+
+// out[b, t, h, d] = value at logical index ((b*H + h) * 2^20 + pos0 + t) * D + d
+__global__ void fill_tokens_kernel(uint16_t* __restrict__ out, int B, int T, int H, int D,
+                                   long long pos0, uint64_t key, float scale) {
+  long long n = (long long)B * T * H * D;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    long long d = e % D;
+    long long r = e / D;
+    long long h = r % H;
+    r /= H;
+    long long t = r % T;
+    long long b = r / T;
+    uint64_t idx = (((uint64_t)b * H + h) * kPosStride + (uint64_t)(pos0 + t)) * D + d;
+    out[e] = gen_bf16(key, idx, scale);
+  }
+}
+
+// cache[b, h, row, d]: linear (row = position, rows >= n_pos zero) or ring of
+// cap rows (row s = largest p < n_pos with p % cap == s, zero if none).
+__global__ void fill_cache_kernel(uint16_t* __restrict__ out, int B, int H, int cap, int D,
+                                  long long n_pos, int ring, uint64_t key, float scale) {
+  long long n = (long long)B * H * cap * D;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    long long d = e % D;
+    long long r = e / D;
+    long long row = r % cap;
+    r /= cap;
+    long long h = r % H;
+    long long b = r / H;
+    long long p;
+    if (ring) {
+      p = (n_pos > 0) ? (n_pos - 1) - (((n_pos - 1) - row) % cap + cap) % cap : -1;
+    } else {
+      p = (row < n_pos) ? row : -1;
+    }
+    uint16_t v = 0;
+    if (p >= 0) {
+      uint64_t idx = (((uint64_t)b * H + h) * kPosStride + (uint64_t)p) * D + d;
+      v = gen_bf16(key, idx, scale);
+    }
+    out[e] = v;
+  }
+}
+
+float sigma_scale(float sigma) { return sigma * (1.0f / 65536.0f); }
+
+uint64_t stream_key(uint64_t seed, uint64_t tid) { return mix64((seed << 32) ^ tid ^ kSalt); }
+
+int grid_for(long long n) {
+  long long g = (n + 255) / 256;
+  if (g > 148LL * 64) g = 148LL * 64;
+  if (g < 1) g = 1;
+  return (int)g;
+}
+
+}  // namespace
+
+extern "C" {
+
+int spark_synth_fill_tokens(void* out, int B, int T, int H, int D, long long pos0,
+                            unsigned long long seed, unsigned long long tid, float sigma, void* stream) {
+  if (!out || B <= 0 || T <= 0 || H <= 0 || D <= 0 || pos0 < 0 || pos0 + T > (long long)kPosStride) return -1;
+  long long n = (long long)B * T * H * D;
+  fill_tokens_kernel<<<grid_for(n), 256, 0, (cudaStream_t)stream>>>(
+      (uint16_t*)out, B, T, H, D, pos0, stream_key(seed, tid), sigma_scale(sigma));
+  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+int spark_synth_fill_cache(void* out, int B, int H, int cap, int D, long long n_pos, int ring,
+                           unsigned long long seed, unsigned long long tid, float sigma, void* stream) {
+  if (!out || B <= 0 || H <= 0 || cap <= 0 || D <= 0 || n_pos < 0 || n_pos > (long long)kPosStride) return -1;
+  if (!ring && n_pos > cap) return -1;
+  long long n = (long long)B * H * cap * D;
+  fill_cache_kernel<<<grid_for(n), 256, 0, (cudaStream_t)stream>>>(
+      (uint16_t*)out, B, H, cap, D, n_pos, ring, stream_key(seed, tid), sigma_scale(sigma));
+  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+}  // extern "C"
