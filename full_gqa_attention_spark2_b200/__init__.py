@@ -1,0 +1,197 @@
+"""Python binding of libspark_attn.so: the Spark2_5 hybrid GQA attention core on B200.
+
+Argument marshalling only.  Every step of the computation runs in the CUDA
+kernels of libspark_attn.so (C ABI in include/spark_attn.h); there is no CPU
+or PyTorch fallback, and a missing library raises at import of the first call.
+PyTorch supplies device memory and streams.  The function names are the C
+entry points'; tensors replace (pointer, size) pairs.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+SPARK_SLIDING = 0
+SPARK_FULL = 1
+SPARK_ROPE_FUSED = 1
+N_LAYERS = 36
+N_Q_HEADS = 16
+N_KV_HEADS = 4
+HEAD_DIM = 256
+WINDOW = 512
+MAX_POSITION = 1 << 20
+
+_STATUS = {0: "OK", -1: "INVALID_ARG", -2: "UNSUPPORTED", -3: "CUDA", -4: "TIMEOUT", -5: "DEVICE_ARG"}
+
+
+class SparkError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"spark status {status} ({_STATUS.get(status, '?')}): {message}")
+        self.status = status
+
+
+class SparkLayerCfg(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("window", ctypes.c_int), ("rot_dim", ctypes.c_int),
+                ("n_q", ctypes.c_int), ("n_kv", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("theta", ctypes.c_double), ("scale", ctypes.c_float)]
+
+
+_LIB = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+
+def lib_path() -> str:
+    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspark_attn.so")
+
+
+def _lib():
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = lib_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing; build it with __graft_entry__.build()")
+    lib = ctypes.CDLL(path)
+    cfgp = ctypes.POINTER(SparkLayerCfg)
+    sig = {
+        "spark_layer_cfg_for_layer": (_I, [_I, cfgp]),
+        "spark_layer_cfg_for_kind": (_I, [_I, cfgp]),
+        "spark_kv_cache_bytes": (ctypes.c_longlong, [cfgp, _I, ctypes.c_longlong]),
+        "spark_stack_kv_bytes": (ctypes.c_longlong, [_I, ctypes.c_longlong]),
+        "spark_rope_apply": (_I, [_P, _I, _I, _I, _P, cfgp, _P]),
+        "spark_kv_append": (_I, [_P, _P, _I, _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
+        "spark_attn_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
+        "spark_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
+        "spark_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, cfgp, _P, ctypes.c_size_t, ctypes.c_uint, _P]),
+        "spark_check": (_I, [_P]),
+        "spark_last_error": (ctypes.c_char_p, []),
+        "spark_version": (_I, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _LIB = lib
+    return lib
+
+
+def exported_symbols():
+    """Names of the C entry points this binding expects the library to export."""
+    return ["spark_layer_cfg_for_layer", "spark_layer_cfg_for_kind", "spark_kv_cache_bytes",
+            "spark_stack_kv_bytes", "spark_rope_apply", "spark_kv_append", "spark_attn_prefill",
+            "spark_decode_workspace_bytes", "spark_attn_decode", "spark_check", "spark_last_error",
+            "spark_version"]
+
+
+def _raise(rc: int):
+    if rc != 0:
+        raise SparkError(rc, spark_last_error())
+
+
+def spark_last_error() -> str:
+    return _lib().spark_last_error().decode(errors="replace")
+
+
+def spark_version() -> int:
+    return _lib().spark_version()
+
+
+def spark_layer_cfg_for_layer(layer: int) -> SparkLayerCfg:
+    c = SparkLayerCfg()
+    _raise(_lib().spark_layer_cfg_for_layer(layer, ctypes.byref(c)))
+    return c
+
+
+def spark_layer_cfg_for_kind(kind: int) -> SparkLayerCfg:
+    c = SparkLayerCfg()
+    _raise(_lib().spark_layer_cfg_for_kind(kind, ctypes.byref(c)))
+    return c
+
+
+def spark_kv_cache_bytes(cfg: SparkLayerCfg, B: int, cap: int) -> int:
+    return int(_lib().spark_kv_cache_bytes(ctypes.byref(cfg), B, cap))
+
+
+def spark_stack_kv_bytes(B: int, ctx: int) -> int:
+    return int(_lib().spark_stack_kv_bytes(B, ctx))
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=torch.bfloat16, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def spark_rope_apply(x: torch.Tensor, pos0: torch.Tensor, cfg: SparkLayerCfg, stream=None) -> None:
+    """Rotate x [B, T, H, 256] bf16 in place; token t of sequence b is at pos0[b] + t."""
+    px = _dev(x, "x", ndim=4)
+    pp = _dev(pos0, "pos0", torch.int32, 1)
+    B, T, H, D = x.shape
+    _raise(_lib().spark_rope_apply(px, B, T, H, pp, ctypes.byref(cfg), _stream(stream)))
+
+
+def spark_kv_append(k_cache, v_cache, k, v, pos0, cfg: SparkLayerCfg, flags: int = 0, stream=None) -> None:
+    """Append k, v [B, T, 4, 256] at positions pos0[b] + t into caches [B, 4, cap, 256]."""
+    pkc, pvc = _dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4)
+    pk, pv = _dev(k, "k", ndim=4), _dev(v, "v", ndim=4)
+    pp = _dev(pos0, "pos0", torch.int32, 1)
+    B, T = k.shape[0], k.shape[1]
+    cap = k_cache.shape[2]
+    _raise(_lib().spark_kv_append(pkc, pvc, cap, pk, pv, B, T, pp, ctypes.byref(cfg), flags, _stream(stream)))
+
+
+def spark_attn_prefill(out, q, k, v, gate, k_cache, v_cache, pos0, cfg: SparkLayerCfg, flags: int = 0,
+                       stream=None) -> None:
+    """Gated GQA attention of a chunk of T queries per sequence (see include/spark_attn.h)."""
+    po = _dev(out, "out", ndim=4)
+    pq, pk, pv = _dev(q, "q", ndim=4), _dev(k, "k", ndim=4), _dev(v, "v", ndim=4)
+    pg = _dev(gate, "gate", ndim=3)
+    pp = _dev(pos0, "pos0", torch.int32, 1)
+    if k_cache is None:
+        pkc = pvc = None
+        cap = 0
+    else:
+        pkc, pvc = _dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4)
+        cap = k_cache.shape[2]
+    B, T = q.shape[0], q.shape[1]
+    _raise(_lib().spark_attn_prefill(po, pq, pk, pv, pg, pkc, pvc, cap, B, T, pp, ctypes.byref(cfg), flags,
+                                     _stream(stream)))
+
+
+def spark_decode_workspace_bytes(B: int, cap: int, cfg: SparkLayerCfg) -> int:
+    return int(_lib().spark_decode_workspace_bytes(B, cap, ctypes.byref(cfg)))
+
+
+def spark_attn_decode(out, q, gate, k_cache, v_cache, pos, cfg: SparkLayerCfg, workspace: torch.Tensor,
+                      flags: int = 0, stream=None) -> None:
+    """Attention of one new token per sequence at pos[b] (its k/v already appended)."""
+    po, pq = _dev(out, "out", ndim=3), _dev(q, "q", ndim=3)
+    pg = _dev(gate, "gate", ndim=2)
+    pkc, pvc = _dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4)
+    pp = _dev(pos, "pos", torch.int32, 1)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    B = q.shape[0]
+    cap = k_cache.shape[2]
+    _raise(_lib().spark_attn_decode(po, pq, pg, pkc, pvc, cap, B, pp, ctypes.byref(cfg), workspace.data_ptr(),
+                                    ws_bytes, flags, _stream(stream)))
+
+
+def spark_check(stream=None) -> None:
+    """Synchronise the stream and raise SparkError if a kernel flagged a device-side error."""
+    _raise(_lib().spark_check(_stream(stream)))

@@ -1,0 +1,321 @@
+// Split-KV decode ("flash decoding") for one new token per sequence.
+//
+// Work unit: (sequence b, KV head g, split s).  The four query heads 4g..4g+3
+// that share KV head g ("Spark-X2.6-4B-Base" page §配套效率设计: 16 query heads
+// share 4 KV heads) are packed into one pass over that head's keys, so every
+// K/V byte is read from HBM once per step.  The pass is HBM-bound: per key it
+// reads 1 KB (K and V, 256 dims, bf16) and does 4 KFLOP.
+//
+// Data path per block: one producer warp streams 64-key K and V tiles with
+// TMA (128-byte swizzled, 3 stages of 64 KB) into shared memory; four
+// consumer warps each take 16 keys of a tile and do
+//     S  = Q K^T        mma.m16n8k16, A = the 4 query rows (padded to 16),
+//                       B = K straight from the swizzled tile (ldmatrix)
+//     online softmax    fp32, exp2 domain
+//     O^T += V^T P^T    A = V^T via ldmatrix.trans, B = P from S's registers
+// then the four warps merge in shared memory and the block writes an
+// unnormalised partial (m, l, o[256]) per query head.  A second kernel merges
+// the splits with a log-sum-exp and applies the sigmoid gate.
+#pragma once
+#include <cuda.h>
+#include "ptx.cuh"
+#include "rope_append.cuh"
+
+namespace spark {
+
+constexpr int kDecNK = 64;                                   // keys per tile
+constexpr int kDecStages = 3;
+constexpr int kDecConsumerWarps = 4;
+constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;    // + 1 producer warp
+constexpr int kDecTileBytes = kDecNK * kHeadDim * 2;         // 32 KB (K or V)
+constexpr int kDecBoxBytes = kDecNK * 128;                   // one 64-dim box: 8 KB
+constexpr int kDecStageBytes = 2 * kDecTileBytes;
+constexpr int kDecMergeBytes = kDecConsumerWarps * 4 * kHeadDim * 4;   // 16 KB
+constexpr int kDecSmemBytes = 1024 /*align slack*/ + kDecStages * kDecStageBytes +
+                              kDecMergeBytes + 1024 /*q, barriers, m/l*/;
+
+struct DecodeParams {
+  const __nv_bfloat16* q;     // [B][16][256]
+  const int* pos;             // [B]
+  float* o_part;              // [B][16][splits][256]
+  float* ml_part;             // [B][16][splits][2]
+  int B, cap, sliding, n_splits, tiles_per_split;
+  int rope, rot;
+  double log2_theta;
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ uint32_t swz_addr(uint32_t tile, int key, int dim) {
+  // byte address of (key, dim) in a tile of four [64 keys x 128 B] boxes, 128 B swizzle
+  return tile + (uint32_t)(dim >> 6) * kDecBoxBytes + (uint32_t)key * 128u +
+         ((uint32_t)(((dim & 63) >> 3) ^ (key & 7)) << 4);
+}
+
+__global__ void __launch_bounds__(kDecThreads, 1)
+    decode_partial_kernel(const __grid_constant__ CUtensorMap kmap,
+                          const __grid_constant__ CUtensorMap vmap, const DecodeParams P) {
+  extern __shared__ uint8_t dsmem[];
+  const uint32_t raw = smem_u32(dsmem);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = dsmem + (base - raw);
+  // layout: [stages x (K tile | V tile)] | merge area (also q staging) | barriers, abort, m, l
+  float* mrg_o = reinterpret_cast<float*>(gbase + kDecStages * kDecStageBytes);
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(mrg_o);        // [4][256], before the loop
+  uint8_t* misc = gbase + kDecStages * kDecStageBytes + kDecMergeBytes;
+  const uint32_t bar_full = smem_u32(misc);
+  const uint32_t bar_empty = bar_full + 8 * kDecStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 16 * kDecStages);
+  float* sm_m = reinterpret_cast<float*>(misc + 16 * kDecStages + 16);
+  float* sm_l = sm_m + 16;
+
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int p = P.pos[b];
+  const bool bad = p < 0 || p >= kMaxPos || (!P.sliding && p >= P.cap);
+  const int n_keys = bad ? 0 : (P.sliding ? min(p + 1, kWindow) : p + 1);
+  const int key_begin = split * P.tiles_per_split * kDecNK;
+  const int key_end = min(n_keys, key_begin + P.tiles_per_split * kDecNK);
+  const int n_tiles = key_end > key_begin ? (key_end - key_begin + kDecNK - 1) / kDecNK : 0;
+  if (bad && threadIdx.x == 0 && split == 0 && g == 0) raise_error(kErrPosition, 0x300u | (unsigned)b);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, kDecConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kDecConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      const int plane = b * kNkv + g;
+      int issued = 0;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % kDecStages;
+        if (i >= kDecStages &&
+            !mbar_wait(bar_empty + 8 * s, ((i / kDecStages) - 1) & 1, abort_flag, P.timeout_ns, 0x10u))
+          break;
+        const uint32_t full = bar_full + 8 * s;
+        mbar_arrive_expect_tx(full, kDecStageBytes);
+        const uint32_t kt = base + s * kDecStageBytes;
+        const int row0 = key_begin + i * kDecNK;
+#pragma unroll
+        for (int d = 0; d < 4; ++d) {
+          tma_load_3d(kt + d * kDecBoxBytes, &kmap, full, d * 64, row0, plane);
+          tma_load_3d(kt + kDecTileBytes + d * kDecBoxBytes, &vmap, full, d * 64, row0, plane);
+        }
+        issued = i + 1;
+      }
+      // Never leave with copies in flight: wait for the last issued tiles to land.
+      for (int i = max(0, issued - kDecStages); i < issued; ++i) {
+        volatile int no_abort = 0;
+        if (!mbar_wait(bar_full + 8 * (i % kDecStages), (i / kDecStages) & 1, &no_abort, 200000000ull, 0x11u))
+          break;
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int tid = threadIdx.x;                 // 0..127
+  const int gq = lane >> 2, cq = lane & 3;     // mma fragment row group / column pair
+  {
+    // Stage the four query rows of this KV group: rotate (optional), scale by
+    // 1/16 (exact in binary), round to bf16.
+    const __nv_bfloat16* qrow = P.q + ((long long)b * kNq + g * 4) * kHeadDim;
+    const int half = P.rot >> 1;
+    for (int e = tid; e < 4 * kHeadDim; e += 128) {
+      const int d = e & (kHeadDim - 1);
+      float x = __bfloat162float(qrow[e]);
+      if (P.rope && d < P.rot && !bad) {
+        const int i = d < half ? d : d - half;
+        const float xp = __bfloat162float(qrow[e + (d < half ? half : -half)]);
+        float c, s;
+        rope_angle(p, exp2(-(2.0 * i / P.rot) * P.log2_theta), c, s);
+        // bf16 rounding of the rotated value, as the stand-alone RoPE kernel does
+        x = __bfloat162float(__float2bfloat16_rn(d < half ? x * c - xp * s : x * c + xp * s));
+      }
+      qs[e] = __float2bfloat16_rn(x * 0.0625f);
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  }
+  uint32_t qa[16][2];
+#pragma unroll
+  for (int ks = 0; ks < 16; ++ks) {
+    if (gq < 4) {
+      qa[ks][0] = *reinterpret_cast<const uint32_t*>(qs + gq * kHeadDim + 16 * ks + 2 * cq);
+      qa[ks][1] = *reinterpret_cast<const uint32_t*>(qs + gq * kHeadDim + 16 * ks + 2 * cq + 8);
+    } else {
+      qa[ks][0] = 0u;
+      qa[ks][1] = 0u;
+    }
+  }
+
+  float o[16][4];
+#pragma unroll
+  for (int t = 0; t < 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+  float m_run = -INFINITY, l_part = 0.f;
+  const float kLog2e = 1.4426950408889634f;
+
+  // ldmatrix lane addressing: matrix mi = lane / 8, row r = lane % 8
+  const int mi = lane >> 3, r8 = lane & 7;
+  const int key_l = warp * 16 + (mi >> 1) * 8 + r8;     // key row this lane addresses
+  const int dim_off = (mi & 1) * 8;
+
+  for (int i = 0; i < n_tiles; ++i) {
+    const int s = i % kDecStages;
+    if (!mbar_wait(bar_full + 8 * s, (i / kDecStages) & 1, abort_flag, P.timeout_ns, 0x12u)) break;
+    const uint32_t kt = base + s * kDecStageBytes;
+    const uint32_t vt = kt + kDecTileBytes;
+
+    // S = Q K^T for this warp's 16 keys, two accumulation chains per n-tile
+    float sa[2][2][4];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) sa[a][c][0] = sa[a][c][1] = sa[a][c][2] = sa[a][c][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 16; ++ks) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(swz_addr(kt, key_l, 16 * ks + dim_off), b0, b1, b2, b3);
+      mma_bf16_16816(sa[0][ks & 1], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
+      mma_bf16_16816(sa[1][ks & 1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
+    }
+    // scores of row gq at keys (8*nt + 2*cq + j)
+    const int kbase = key_begin + i * kDecNK + warp * 16;
+    float tv[2][2];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int kidx = kbase + nt * 8 + 2 * cq + j;
+        const float sv = (sa[nt][0][j] + sa[nt][1][j]) * kLog2e;
+        tv[nt][j] = kidx < key_end ? sv : -INFINITY;
+        mx = fmaxf(mx, tv[nt][j]);
+      }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float m_use = m_new == -INFINITY ? 0.f : m_new;
+    const float alpha = fast_exp2(m_run - m_use);
+    float pv[2][2], psum = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        pv[nt][j] = fast_exp2(tv[nt][j] - m_use);
+        psum += pv[nt][j];
+      }
+    l_part = l_part * alpha + psum;
+    m_run = m_new;
+    const float a_lo = __shfl_sync(0xffffffffu, alpha, (8 * cq) & 31);
+    const float a_hi = __shfl_sync(0xffffffffu, alpha, (8 * cq + 4) & 31);
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      o[t][0] *= a_lo;
+      o[t][1] *= a_hi;
+      o[t][2] *= a_lo;
+      o[t][3] *= a_hi;
+    }
+    const uint32_t pb0 = pack_bf16(pv[0][0], pv[0][1]);
+    const uint32_t pb1 = pack_bf16(pv[1][0], pv[1][1]);
+
+    // O^T += V^T P^T
+#pragma unroll
+    for (int mt = 0; mt < 16; ++mt) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_t(swz_addr(vt, key_l, 16 * mt + dim_off), a0, a1, a2, a3);
+      mma_bf16_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+  }
+
+  // ----------------------------------------------------- merge the 4 warps
+  asm volatile("bar.sync 1, 128;" ::: "memory");    // q staging area is free again
+  float l_row = l_part;
+  l_row += __shfl_xor_sync(0xffffffffu, l_row, 1);
+  l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
+  if (cq == 0 && gq < 4) {
+    sm_m[warp * 4 + gq] = m_run;
+    sm_l[warp * 4 + gq] = l_row;
+  }
+  if (cq < 2) {
+    float* w = mrg_o + warp * 4 * kHeadDim;
+#pragma unroll
+    for (int mt = 0; mt < 16; ++mt) {
+      const int d0 = 16 * mt + gq;
+      w[(2 * cq) * kHeadDim + d0] = o[mt][0];
+      w[(2 * cq + 1) * kHeadDim + d0] = o[mt][1];
+      w[(2 * cq) * kHeadDim + d0 + 8] = o[mt][2];
+      w[(2 * cq + 1) * kHeadDim + d0 + 8] = o[mt][3];
+    }
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  {
+    const int hh = tid >> 5;                      // query head within the group
+    float mw[kDecConsumerWarps], ms = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDecConsumerWarps; ++w) {
+      mw[w] = sm_m[w * 4 + hh];
+      ms = fmaxf(ms, mw[w]);
+    }
+    float ew[kDecConsumerWarps], ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecConsumerWarps; ++w) {
+      ew[w] = (ms == -INFINITY) ? 0.f : fast_exp2(mw[w] - ms);
+      ls += ew[w] * sm_l[w * 4 + hh];
+    }
+    const long long row = ((long long)b * kNq + g * 4 + hh) * P.n_splits + split;
+    float* dst = P.o_part + row * kHeadDim;
+    for (int d = (tid & 31); d < kHeadDim; d += 32) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecConsumerWarps; ++w) acc += ew[w] * mrg_o[(w * 4 + hh) * kHeadDim + d];
+      dst[d] = acc;
+    }
+    if ((tid & 31) == 0) {
+      P.ml_part[row * 2 + 0] = ms;
+      P.ml_part[row * 2 + 1] = ls;
+    }
+  }
+}
+
+// out[b][h][:] = gate-scaled log-sum-exp merge of the splits' partials.
+__global__ void __launch_bounds__(64) decode_combine_kernel(__nv_bfloat16* __restrict__ out,
+                                                            const __nv_bfloat16* __restrict__ gate,
+                                                            const float* __restrict__ o_part,
+                                                            const float* __restrict__ ml_part,
+                                                            int n_splits) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const long long row0 = ((long long)b * kNq + h) * n_splits;
+  float ms = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) ms = fmaxf(ms, ml_part[(row0 + s) * 2]);
+  float ls = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < n_splits; ++s) {
+    const float m = ml_part[(row0 + s) * 2];
+    const float e = (m == -INFINITY) ? 0.f : fast_exp2(m - ms);
+    ls += e * ml_part[(row0 + s) * 2 + 1];
+    const float4 v = reinterpret_cast<const float4*>(o_part + (row0 + s) * kHeadDim)[threadIdx.x];
+    acc.x += e * v.x;
+    acc.y += e * v.y;
+    acc.z += e * v.z;
+    acc.w += e * v.w;
+  }
+  const float gl = __bfloat162float(gate[(long long)b * kNq + h]);
+  const float scale = (ls > 0.f) ? (1.f / ls) * (1.f / (1.f + expf(-gl))) : 0.f;
+  uint2 packed;
+  packed.x = pack_bf16(acc.x * scale, acc.y * scale);
+  packed.y = pack_bf16(acc.z * scale, acc.w * scale);
+  reinterpret_cast<uint2*>(out + ((long long)b * kNq + h) * kHeadDim)[threadIdx.x] = packed;
+}
+
+}  // namespace spark

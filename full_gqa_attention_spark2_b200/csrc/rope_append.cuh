@@ -1,0 +1,120 @@
+// RoPE and KV-cache append kernels (memory-bound, bf16 in / bf16 out).
+//
+// RoPE ("Spark-X2.6-4B config.json" page §1M 上下文如何做到 and "Spark-X2.6-4B-Base"
+// page §全局注意力 5M 基频 RoPE): for i < rot/2 the pair (x_i, x_{i+rot/2}) turns
+// by a = pos * theta^(-2i/rot); sliding layers rot = 256, theta = 1e4; full
+// layers rot = 64, theta = 5e6 (dims 64..255 untouched).
+//
+// Angle accuracy: at pos ~ 2^20 the product pos * f_i in fp32 would carry an
+// error of ~0.06 rad.  The product and its reduction into [-pi, pi] are done
+// in fp64, then sincosf runs on the reduced fp32 angle (error ~1e-7 rad).
+#pragma once
+#include "ptx.cuh"
+
+namespace spark {
+
+constexpr int kHeadDim = 256;
+constexpr int kNq = 16;
+constexpr int kNkv = 4;
+constexpr int kWindow = 512;
+constexpr int kMaxPos = 1 << 20;
+
+// cos/sin of pos * f for an integer position, via an fp64 reduction mod 2*pi.
+__device__ __forceinline__ void rope_angle(int pos, double f, float& c, float& s) {
+  const double kTwoPi = 6.283185307179586476925286766559;
+  const double kInvTwoPi = 0.15915494309189533576888376337251;
+  double a = (double)pos * f;
+  double k = rint(a * kInvTwoPi);
+  double r = fma(-k, kTwoPi, a);
+  sincosf((float)r, &s, &c);
+}
+
+// x [B][T][H][256], in place.  One thread per (token, two consecutive pairs).
+__global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x, int B, int T,
+                                                   int H, const int* __restrict__ pos0,
+                                                   double log2_theta, int rot) {
+  __shared__ double freq[128];
+  const int half = rot >> 1;
+  for (int i = threadIdx.x; i < half; i += blockDim.x)
+    freq[i] = exp2(-(2.0 * i / rot) * log2_theta);
+  __syncthreads();
+
+  const int per_tok = half >> 1;                  // threads per token
+  const int tok_per_block = blockDim.x / per_tok;
+  const int j = threadIdx.x % per_tok;
+  const long long n = (long long)blockIdx.x * tok_per_block + threadIdx.x / per_tok;
+  if (threadIdx.x / per_tok >= tok_per_block || n >= (long long)B * T) return;
+  const int b = (int)(n / T);
+  const int t = (int)(n % T);
+  const int p0 = pos0[b];
+  if (p0 < 0 || p0 > kMaxPos - T) {
+    if (t == 0 && j == 0) raise_error(kErrPosition, 0x100u | (unsigned)b);
+    return;
+  }
+  const int pos = p0 + t;
+  float c0, s0, c1, s1;
+  rope_angle(pos, freq[2 * j], c0, s0);
+  rope_angle(pos, freq[2 * j + 1], c1, s1);
+  __nv_bfloat16* row = x + n * H * kHeadDim;
+  for (int h = 0; h < H; ++h) {
+    uint32_t* lo_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + 2 * j);
+    uint32_t* hi_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + half + 2 * j);
+    uint32_t lo = *lo_p, hi = *hi_p;
+    float l0 = bf16_lo(lo), l1 = bf16_hi(lo), h0 = bf16_lo(hi), h1 = bf16_hi(hi);
+    *lo_p = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
+    *hi_p = pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);
+  }
+}
+
+// Append k/v [B][T][4][256] of T new tokens into caches [B][4][cap][256].
+// One block per written token, thread = (head, 16-byte chunk of 8 dims).
+// Sliding layers (ring of 512 rows) only write the last min(T, 512) tokens.
+__global__ void __launch_bounds__(128) kv_append_kernel(
+    __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache, int cap,
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int B, int T,
+    int t_first, const int* __restrict__ pos0, int sliding, int rope, double log2_theta, int rot) {
+  const int t = t_first + blockIdx.x;
+  const int b = blockIdx.y;
+  const int h = threadIdx.x >> 5;
+  const int ch = threadIdx.x & 31;
+  const int p0 = pos0[b];
+  const bool bad = p0 < 0 || p0 > kMaxPos - T || (!sliding && p0 + T > cap);
+  if (bad) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(kErrPosition, 0x200u | (unsigned)b);
+    return;
+  }
+  const int pos = p0 + t;
+  const long long row = sliding ? (pos & (kWindow - 1)) : pos;
+  const long long src = (((long long)b * T + t) * kNkv + h) * kHeadDim;
+  const long long dst = (((long long)b * kNkv + h) * cap + row) * kHeadDim;
+
+  const uint4* vs = reinterpret_cast<const uint4*>(v + src);
+  reinterpret_cast<uint4*>(v_cache + dst)[ch] = vs[ch];
+
+  const uint4* ks = reinterpret_cast<const uint4*>(k + src);
+  uint4* kd = reinterpret_cast<uint4*>(k_cache + dst);
+  const int half = rot >> 1;
+  if (!rope || ch * 8 >= rot) {
+    kd[ch] = ks[ch];
+    return;
+  }
+  if (ch * 8 >= half) return;                    // the partner thread writes this chunk
+  const int pc = ch + (half >> 3);               // chunk holding the partner dims
+  uint4 lo = ks[ch], hi = ks[pc];
+  uint32_t* l = reinterpret_cast<uint32_t*>(&lo);
+  uint32_t* hh = reinterpret_cast<uint32_t*>(&hi);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int i0 = ch * 8 + 2 * e;
+    float c0, s0, c1, s1;
+    rope_angle(pos, exp2(-(2.0 * i0 / rot) * log2_theta), c0, s0);
+    rope_angle(pos, exp2(-(2.0 * (i0 + 1) / rot) * log2_theta), c1, s1);
+    float l0 = bf16_lo(l[e]), l1 = bf16_hi(l[e]), h0 = bf16_lo(hh[e]), h1 = bf16_hi(hh[e]);
+    l[e] = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
+    hh[e] = pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);
+  }
+  kd[ch] = lo;
+  kd[pc] = hi;
+}
+
+}  // namespace spark

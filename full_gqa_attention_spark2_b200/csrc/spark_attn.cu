@@ -1,0 +1,429 @@
+// libspark_attn.so: host entry points of the C ABI declared in
+// include/spark_attn.h.  One translation unit: the kernels live in the .cuh
+// files included below, so the device error word is a single module symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "../../include/spark_attn.h"
+#include "decode.cuh"
+#include "prefill.cuh"
+#include "ptx.cuh"
+#include "rope_append.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(SPARK_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- devices ---
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  std::once_flag once;
+  int ok = 0;          // 1: sm_100 and attributes set
+  int sm_count = 148;
+  char why[160] = "";
+};
+DeviceInfo g_dev[kMaxDevices];
+
+int device_ready(int* dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SPARK_ERR_UNSUPPORTED, "device index %d", dev);
+  DeviceInfo& d = g_dev[dev];
+  std::call_once(d.once, [&]() {
+    int major = 0, minor = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (major != 10 || minor != 0) {
+      snprintf(d.why, sizeof(d.why), "device %d is sm_%d%d; this library is built for sm_100a", dev,
+               major, minor);
+      return;
+    }
+    d.sm_count = sms > 0 ? sms : 148;
+    cudaError_t a = cudaFuncSetAttribute(spark::decode_partial_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         spark::kDecSmemBytes);
+    cudaError_t b = cudaFuncSetAttribute(spark::prefill_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         spark::kPfSmemBytes);
+    if (a != cudaSuccess || b != cudaSuccess) {
+      snprintf(d.why, sizeof(d.why), "cudaFuncSetAttribute: %s",
+               cudaGetErrorString(a != cudaSuccess ? a : b));
+      return;
+    }
+    d.ok = 1;
+  });
+  if (!d.ok) return fail(SPARK_ERR_UNSUPPORTED, "%s", d.why);
+  *dev_out = dev;
+  return SPARK_OK;
+}
+
+// Wait limit of the kernels' bounded waits.  SPARK_WAIT_TIMEOUT_NS overrides
+// it (used by the tests that make a wait run out on purpose).
+unsigned long long wait_timeout_ns() {
+  static std::atomic<unsigned long long> cached{0};
+  unsigned long long v = cached.load();
+  if (v == 0) {
+    const char* s = getenv("SPARK_WAIT_TIMEOUT_NS");
+    v = s ? strtoull(s, nullptr, 10) : 0ull;
+    if (v == 0) v = 1000000000ull;   // 1 s
+    cached.store(v);
+  }
+  return v;
+}
+
+// ------------------------------------------------------------ tensor maps ---
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle, dims/strides innermost first (strides in bytes, rank-1 of them)
+int make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+             const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(SPARK_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SPARK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return SPARK_OK;
+}
+
+// -------------------------------------------------------------- checks -----
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cfg(const spark_layer_cfg* c) {
+  if (!c) return fail(SPARK_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->n_q != 16 || c->n_kv != 4 || c->head_dim != 256)
+    return fail(SPARK_ERR_UNSUPPORTED, "only n_q 16, n_kv 4, head_dim 256 are built");
+  if (fabsf(c->scale - 0.0625f) > 0.0f) return fail(SPARK_ERR_UNSUPPORTED, "scale must be 1/16");
+  if (c->kind == SPARK_SLIDING) {
+    if (c->window != 512 || c->rot_dim != 256 || c->theta != 1.0e4)
+      return fail(SPARK_ERR_INVALID_ARG, "sliding cfg must be window 512, rot 256, theta 1e4");
+  } else if (c->kind == SPARK_FULL) {
+    if (c->window != 0 || c->rot_dim != 64 || c->theta != 5.0e6)
+      return fail(SPARK_ERR_INVALID_ARG, "full cfg must be window 0, rot 64, theta 5e6");
+  } else {
+    return fail(SPARK_ERR_INVALID_ARG, "unknown layer kind %d", c->kind);
+  }
+  return SPARK_OK;
+}
+
+// ---------------------------------------------------------- decode plan ----
+struct DecodePlan {
+  int n_splits;
+  int tiles_per_split;
+};
+
+// Choose the number of key splits per (sequence, KV head): each block streams
+// tiles_per_split 64-key tiles; the grid runs in waves of one block per SM.
+// Minimise waves * (tiles per block + fixed per-block cost of ~2 tiles).
+DecodePlan decode_plan(int B, int cap, int sliding, int sm_count) {
+  const int max_keys = sliding ? spark::kWindow : cap;
+  const int tiles = (max_keys + spark::kDecNK - 1) / spark::kDecNK;
+  const long long units = (long long)B * spark::kNkv;
+  DecodePlan best{1, tiles};
+  double best_cost = 1e300;
+  const int s_max = tiles < 4096 ? tiles : 4096;
+  for (int s = 1; s <= s_max; ++s) {
+    const int tps = (tiles + s - 1) / s;
+    const int s_eff = (tiles + tps - 1) / tps;
+    const long long ctas = units * s_eff;
+    const long long waves = (ctas + sm_count - 1) / sm_count;
+    const double cost = (double)waves * (tps + 2.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best.n_splits = s_eff;
+      best.tiles_per_split = tps;
+    }
+  }
+  return best;
+}
+
+size_t decode_ws_bytes(int B, const DecodePlan& pl) {
+  const size_t rows = (size_t)B * spark::kNq * pl.n_splits;
+  return rows * spark::kHeadDim * sizeof(float) + rows * 2 * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+int spark_version(void) { return 100; }
+
+const char* spark_last_error(void) { return g_last_error; }
+
+int spark_layer_cfg_for_kind(int kind, spark_layer_cfg* out) {
+  if (!out) return fail(SPARK_ERR_INVALID_ARG, "out is NULL");
+  spark_layer_cfg c;
+  c.kind = kind;
+  c.n_q = 16;
+  c.n_kv = 4;
+  c.head_dim = 256;
+  c.scale = 0.0625f;
+  if (kind == SPARK_SLIDING) {
+    c.window = 512;
+    c.rot_dim = 256;
+    c.theta = 1.0e4;
+  } else if (kind == SPARK_FULL) {
+    c.window = 0;
+    c.rot_dim = 64;
+    c.theta = 5.0e6;
+  } else {
+    return fail(SPARK_ERR_INVALID_ARG, "unknown layer kind %d", kind);
+  }
+  *out = c;
+  return SPARK_OK;
+}
+
+int spark_layer_cfg_for_layer(int layer, spark_layer_cfg* out) {
+  if (layer < 0 || layer >= SPARK_N_LAYERS) return fail(SPARK_ERR_INVALID_ARG, "layer %d outside [0, 36)", layer);
+  return spark_layer_cfg_for_kind(layer % 4 == 3 ? SPARK_FULL : SPARK_SLIDING, out);
+}
+
+long long spark_kv_cache_bytes(const spark_layer_cfg* cfg, int B, long long cap) {
+  if (check_cfg(cfg) != SPARK_OK || B <= 0 || cap <= 0) return -1;
+  return 2LL * B * cfg->n_kv * cap * cfg->head_dim * 2LL;
+}
+
+long long spark_stack_kv_bytes(int B, long long ctx) {
+  if (B <= 0 || ctx < 0) return -1;
+  long long total = 0;
+  for (int l = 0; l < SPARK_N_LAYERS; ++l) {
+    const long long rows = (l % 4 == 3) ? ctx : (ctx < SPARK_WINDOW ? ctx : SPARK_WINDOW);
+    total += 2LL * B * SPARK_N_KV_HEADS * rows * SPARK_HEAD_DIM * 2LL;
+  }
+  return total;
+}
+
+int spark_rope_apply(void* x, int B, int T, int H, const int* pos0, const spark_layer_cfg* cfg,
+                     void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!x || !pos0) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || T <= 0 || T > SPARK_MAX_POSITION || (H != 16 && H != 4))
+    return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d H=%d", B, T, H);
+  if (!aligned16(x)) return fail(SPARK_ERR_INVALID_ARG, "x must be 16-byte aligned");
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  const int per_tok = cfg->rot_dim / 4;
+  const int tok_per_block = 128 / per_tok;
+  const long long n = (long long)B * T;
+  const long long grid = (n + tok_per_block - 1) / tok_per_block;
+  if (grid > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "too many tokens");
+  spark::rope_kernel<<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>(
+      (__nv_bfloat16*)x, B, T, H, pos0, log2(cfg->theta), cfg->rot_dim);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "rope_kernel launch");
+}
+
+int spark_kv_append(void* k_cache, void* v_cache, int cap, const void* k, const void* v, int B,
+                    int T, const int* pos0, const spark_layer_cfg* cfg, unsigned flags,
+                    void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!k_cache || !v_cache || !k || !v || !pos0) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B > 65535 || T <= 0 || T > SPARK_MAX_POSITION || cap <= 0)
+    return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d cap=%d", B, T, cap);
+  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
+  if (!sliding && cap > SPARK_MAX_POSITION) return fail(SPARK_ERR_INVALID_ARG, "cap above 2^20");
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v))
+    return fail(SPARK_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  const int t_first = sliding && T > SPARK_WINDOW ? T - SPARK_WINDOW : 0;
+  dim3 grid(T - t_first, B);
+  spark::kv_append_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
+      (__nv_bfloat16*)k_cache, (__nv_bfloat16*)v_cache, cap, (const __nv_bfloat16*)k,
+      (const __nv_bfloat16*)v, B, T, t_first, pos0, sliding, (flags & SPARK_ROPE_FUSED) ? 1 : 0,
+      log2(cfg->theta), cfg->rot_dim);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "kv_append_kernel launch");
+}
+
+size_t spark_decode_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg) {
+  if (check_cfg(cfg) != SPARK_OK || B <= 0 || cap <= 0) return 0;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  return decode_ws_bytes(B, decode_plan(B, sliding ? SPARK_WINDOW : cap, sliding, sms > 0 ? sms : 148));
+}
+
+int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_cache,
+                      const void* v_cache, int cap, int B, const int* pos,
+                      const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
+                      unsigned flags, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!out || !q || !gate || !k_cache || !v_cache || !pos || !workspace)
+    return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B > 65535 || cap <= 0) return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d cap=%d", B, cap);
+  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
+  if (!sliding && cap > SPARK_MAX_POSITION) return fail(SPARK_ERR_INVALID_ARG, "cap above 2^20");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(workspace))
+    return fail(SPARK_ERR_INVALID_ARG, "tensors and workspace must be 16-byte aligned");
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  const DecodePlan pl = decode_plan(B, cap, sliding, g_dev[dev].sm_count);
+  if (ws_bytes < decode_ws_bytes(B, pl))
+    return fail(SPARK_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu needed", ws_bytes,
+                decode_ws_bytes(B, pl));
+
+  CUtensorMap km, vm;
+  const cuuint64_t dims[3] = {256, (cuuint64_t)cap, (cuuint64_t)B * 4};
+  const cuuint64_t strides[2] = {512, (cuuint64_t)cap * 512};
+  const cuuint32_t box[3] = {64, (cuuint32_t)spark::kDecNK, 1};
+  if ((rc = make_map(&km, k_cache, 3, dims, strides, box))) return rc;
+  if ((rc = make_map(&vm, v_cache, 3, dims, strides, box))) return rc;
+
+  spark::DecodeParams P;
+  P.q = (const __nv_bfloat16*)q;
+  P.pos = pos;
+  P.o_part = (float*)workspace;
+  P.ml_part = (float*)workspace + (size_t)B * spark::kNq * pl.n_splits * spark::kHeadDim;
+  P.B = B;
+  P.cap = cap;
+  P.sliding = sliding;
+  P.n_splits = pl.n_splits;
+  P.tiles_per_split = pl.tiles_per_split;
+  P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
+  P.rot = cfg->rot_dim;
+  P.log2_theta = log2(cfg->theta);
+  P.timeout_ns = wait_timeout_ns();
+  dim3 grid(pl.n_splits, spark::kNkv, B);
+  spark::decode_partial_kernel<<<grid, spark::kDecThreads, spark::kDecSmemBytes, (cudaStream_t)stream>>>(
+      km, vm, P);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode_partial_kernel launch");
+  spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, (cudaStream_t)stream>>>(
+      (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_combine_kernel launch");
+}
+
+int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, const void* gate,
+                       const void* k_cache, const void* v_cache, int cap, int B, int T,
+                       const int* pos0, const spark_layer_cfg* cfg, unsigned flags, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!out || !q || !k || !v || !gate || !pos0) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if ((k_cache == nullptr) != (v_cache == nullptr))
+    return fail(SPARK_ERR_INVALID_ARG, "pass both caches or neither");
+  if (B <= 0 || B > 65535 || T <= 0 || T > SPARK_MAX_POSITION)
+    return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d", B, T);
+  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  if (k_cache) {
+    if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
+    if (!sliding && (cap <= 0 || cap > SPARK_MAX_POSITION)) return fail(SPARK_ERR_INVALID_ARG, "bad cap %d", cap);
+  }
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (k_cache && (!aligned16(k_cache) || !aligned16(v_cache))))
+    return fail(SPARK_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  if (flags & SPARK_ROPE_FUSED)
+    return fail(SPARK_ERR_UNSUPPORTED, "prefill takes rotated q; run spark_rope_apply first");
+
+  // Q, chunk K/V: [B][T][H][256] as 4-D (dim, head, token, batch); caches
+  // [B][4][cap][256] as 3-D (dim, row, batch*head).  128-byte swizzled boxes of 64 dims.
+  CUtensorMap qm, km, vm, kcm, vcm;
+  {
+    const cuuint64_t dq[4] = {256, 16, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t sq[3] = {512, 512ull * 16, 512ull * 16 * T};
+    const cuuint32_t bq[4] = {64, 1, (cuuint32_t)spark::kPfM, 1};
+    if ((rc = make_map(&qm, q, 4, dq, sq, bq))) return rc;
+    const cuuint64_t dk[4] = {256, 4, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t sk[3] = {512, 512ull * 4, 512ull * 4 * T};
+    const cuuint32_t bk[4] = {64, 1, (cuuint32_t)spark::kPfN, 1};
+    const cuuint32_t bv[4] = {64, 1, 32, 1};
+    if ((rc = make_map(&km, k, 4, dk, sk, bk))) return rc;
+    if ((rc = make_map(&vm, v, 4, dk, sk, bv))) return rc;
+    if (k_cache) {
+      const cuuint64_t dc[3] = {256, (cuuint64_t)cap, (cuuint64_t)B * 4};
+      const cuuint64_t sc[2] = {512, (cuuint64_t)cap * 512};
+      const cuuint32_t bkc[3] = {64, (cuuint32_t)spark::kPfN, 1};
+      const cuuint32_t bvc[3] = {64, 32, 1};
+      if ((rc = make_map(&kcm, k_cache, 3, dc, sc, bkc))) return rc;
+      if ((rc = make_map(&vcm, v_cache, 3, dc, sc, bvc))) return rc;
+    } else {
+      kcm = km;
+      vcm = vm;
+    }
+  }
+  spark::PrefillParams P;
+  P.out = (__nv_bfloat16*)out;
+  P.gate = (const __nv_bfloat16*)gate;
+  P.pos0 = pos0;
+  P.B = B;
+  P.T = T;
+  P.cap = k_cache ? cap : 0;
+  P.sliding = sliding;
+  P.has_cache = k_cache ? 1 : 0;
+  P.n_qt = (T + spark::kPfM - 1) / spark::kPfM;
+  P.timeout_ns = wait_timeout_ns();
+  const long long blocks = (long long)B * spark::kNq * P.n_qt;
+  if (blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");
+  spark::prefill_kernel<<<(unsigned)blocks, spark::kPfThreads, spark::kPfSmemBytes, (cudaStream_t)stream>>>(
+      qm, km, vm, kcm, vcm, P);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "prefill_kernel launch");
+}
+
+int spark_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned word = 0, info = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&word, spark::g_error_word, sizeof(word));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&info, spark::g_error_info, sizeof(info));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(spark::g_error_word, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (word & spark::kErrTimeout)
+    return fail(SPARK_ERR_TIMEOUT, "a bounded device wait expired (site 0x%x)", info);
+  if (word & spark::kErrPosition)
+    return fail(SPARK_ERR_DEVICE_ARG, "a position failed its device-side check (site 0x%x)", info);
+  return SPARK_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,172 @@
+/*
+ * spark_attn.h -- C ABI of libspark_attn.so, the attention core of the
+ * Spark2_5 layer (Spark-X2.5 / X2.6 4B) on NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  Causal grouped-query attention with 16 query heads that
+ * share 4 KV heads (q head h reads KV head h / 4) at head_dim 256 and score
+ * scale 1/sqrt(256), an fp32 softmax, and a per-head sigmoid output gate, over
+ * a 36-layer stack that repeats three sliding-window layers and one full layer:
+ *   - sliding layers: key j visible to query i iff i - 512 < j <= i; RoPE with
+ *     theta 1e4 over all 256 dims;
+ *   - full layers: key j visible iff j <= i; RoPE with theta 5e6 over the
+ *     first 64 dims only (partial rotary factor 0.25).
+ * Sources: "Spark-X2.6-4B-FP8 W8A8" page §一 (16/4 heads, head_dim 256,
+ * 36 layers); "Spark-X2.6-4B config.json" page §混合注意力 and §1M 上下文如何做到
+ * (3 sliding + 1 full, the two RoPE parameter sets); "Spark-X2.6-4B-Base"
+ * hybrid attention page §36 层混合注意力排布, §滑动窗口 512, §全局注意力 5M 基频
+ * RoPE, §配套效率设计 (masks, partial rotary, GQA, headwise gate);
+ * "星火 X2.5-4B F16 与 Q4 实测对比" page §一 (KV cache per token) and §三 (fp32
+ * softmax, sigmoid gate per head).
+ *
+ * RoPE convention (the pages give none): for i < rot/2 the pair
+ * (x_i, x_{i+rot/2}) turns by angle pos * theta^(-2i/rot).
+ *
+ * Conventions shared by every call:
+ *   - All tensors are bf16, contiguous, in device memory, allocated and owned
+ *     by the caller.  The library allocates and frees nothing.
+ *   - Positions are absolute (0 <= pos < 2^20).  Per-sequence positions live
+ *     in caller-owned device int32 arrays, so a captured CUDA graph can replay
+ *     with new positions.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ *     default stream) and runs on the current device, which must be sm_100.
+ *   - Host-side argument checks run before any launch; on failure nothing is
+ *     launched.  Positions are device data, so they are checked on the device:
+ *     a bad position makes the kernel skip that sequence and set the library's
+ *     device error word, which spark_check() reports.
+ *   - Layouts (element strides, innermost first):
+ *       q, out   [B][T][16][256]      k, v (new tokens)  [B][T][4][256]
+ *       gate     [B][T][16] (logits; the kernel applies the sigmoid)
+ *       k_cache, v_cache [B][4][cap][256]
+ *     Full layers use a linear cache: row = position, cap >= context.
+ *     Sliding layers use a ring of cap = 512 rows: row = position mod 512.
+ *   - Return value: SPARK_OK or a negative spark status.
+ */
+#ifndef SPARK_ATTN_H
+#define SPARK_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SPARK_OK                0
+#define SPARK_ERR_INVALID_ARG  (-1)  /* null pointer, bad size, bad cfg */
+#define SPARK_ERR_UNSUPPORTED  (-2)  /* not an sm_100 device, or dims other than 16/4/256 */
+#define SPARK_ERR_CUDA         (-3)  /* a CUDA runtime call failed; see spark_last_error() */
+#define SPARK_ERR_TIMEOUT      (-4)  /* a bounded device-side wait expired (reported by spark_check) */
+#define SPARK_ERR_DEVICE_ARG   (-5)  /* a position checked on the device was out of range (spark_check) */
+
+#define SPARK_N_LAYERS     36
+#define SPARK_N_Q_HEADS    16
+#define SPARK_N_KV_HEADS   4
+#define SPARK_HEAD_DIM     256
+#define SPARK_WINDOW       512
+#define SPARK_MAX_POSITION (1 << 20)
+
+typedef enum { SPARK_SLIDING = 0, SPARK_FULL = 1 } spark_kind;
+
+/* Per-layer attention parameters.  Only the values the pages fix are
+ * accepted: n_q 16, n_kv 4, head_dim 256, scale 1/16, and per kind
+ * (window 512, rot_dim 256, theta 1e4) or (window 0, rot_dim 64, theta 5e6). */
+typedef struct {
+  int kind;       /* spark_kind */
+  int window;     /* 512 for sliding layers, 0 (unbounded) for full layers */
+  int rot_dim;    /* rotated leading dims: 256 sliding, 64 full */
+  int n_q;        /* 16 */
+  int n_kv;       /* 4 */
+  int head_dim;   /* 256 */
+  double theta;   /* RoPE base: 1e4 sliding, 5e6 full */
+  float scale;    /* 1/sqrt(head_dim) = 0.0625 */
+} spark_layer_cfg;
+
+/* Flags */
+#define SPARK_ROPE_FUSED 1u  /* the call rotates its raw q (prefill, decode) or k (kv_append) itself */
+
+/* Parameters of 0-based layer `layer` of the 36-layer stack: layer l is full
+ * iff l % 4 == 3 ("3 sliding + 1 full", the last layer full).
+ * Errors: SPARK_ERR_INVALID_ARG for layer outside [0, 36) or out == NULL. */
+int spark_layer_cfg_for_layer(int layer, spark_layer_cfg* out);
+
+/* Parameters of a layer kind (SPARK_SLIDING or SPARK_FULL). */
+int spark_layer_cfg_for_kind(int kind, spark_layer_cfg* out);
+
+/* Bytes of one layer's K+V cache for B sequences of capacity cap rows:
+ * 2 * B * 4 * cap * 256 * 2.  Per token and full layer this is the 4 KB the
+ * "星火 X2.5-4B F16 与 Q4" page §一 derives.  Returns -1 on bad arguments. */
+long long spark_kv_cache_bytes(const spark_layer_cfg* cfg, int B, long long cap);
+
+/* Bytes of the whole 36-layer stack's caches at context ctx: 9 linear caches
+ * of ctx rows plus 27 rings of min(ctx, 512) rows ("Sharp-Spark-X2.5-4B-GGUF"
+ * page §三: only the 9 full layers grow).  Returns -1 on bad arguments. */
+long long spark_stack_kv_bytes(int B, long long ctx);
+
+/* Rotate x [B][T][H][256] in place; token t of sequence b is at position
+ * pos0[b] + t (pos0: device int32 [B]).  H is 16 (queries) or 4 (keys).
+ * Dims >= cfg->rot_dim are not touched. */
+int spark_rope_apply(void* x, int B, int T, int H, const int* pos0, const spark_layer_cfg* cfg,
+                     void* stream);
+
+/* Append T new tokens per sequence to a layer's K/V cache.  k, v
+ * [B][T][4][256]; token t of sequence b is at position pos0[b] + t.
+ * Full layer: row = position, requires pos0[b] + T <= cap.
+ * Sliding layer: cap must be 512; row = position mod 512; only the last
+ * min(T, 512) tokens are written (older ones would be overwritten anyway).
+ * With SPARK_ROPE_FUSED, k is raw and is rotated on its way into the cache
+ * (the k buffer itself is not modified); v is copied bit for bit. */
+int spark_kv_append(void* k_cache, void* v_cache, int cap, const void* k, const void* v, int B,
+                    int T, const int* pos0, const spark_layer_cfg* cfg, unsigned flags,
+                    void* stream);
+
+/* Attention of a chunk of T queries per sequence (prefill).
+ *   q [B][T][16][256] (rotated, or raw with SPARK_ROPE_FUSED), k [B][T][4][256]
+ *   rotated, v [B][T][4][256], gate [B][T][16]; out [B][T][16][256].
+ *   Token t of sequence b is at position pos0[b] + t (pos0: device int32 [B]).
+ *   The chunk's own keys come from k/v.  Earlier keys (the history,
+ *   positions < pos0[b]) come from the cache: full layers read rows
+ *   [0, pos0[b]); sliding layers read the ring rows of positions
+ *   [max(0, pos0[b] - 511), pos0[b]).  Pass k_cache = v_cache = NULL when no
+ *   sequence has history.  The cache is only read: append the chunk after
+ *   this call on sliding layers (the ring rows are still needed here), before
+ *   or after it on full layers.
+ * Device requirements: sm_100a, about 225 KB of shared memory per block. */
+int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, const void* gate,
+                       const void* k_cache, const void* v_cache, int cap, int B, int T,
+                       const int* pos0, const spark_layer_cfg* cfg, unsigned flags, void* stream);
+
+/* Workspace bytes spark_attn_decode needs for B sequences and cache capacity
+ * cap (split-KV partials: per sequence, query head and split, 256 + 2 fp32).
+ * Returns 0 on bad arguments. */
+size_t spark_decode_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg);
+
+/* Attention of one new token per sequence (decode, append-then-attend).
+ *   q [B][16][256] (rotated, or raw with SPARK_ROPE_FUSED), gate [B][16];
+ *   out [B][16][256].  The new token of sequence b is at position pos[b]
+ *   (device int32 [B]) and its k/v must already be in the cache.
+ *   Full layer: attends to cache rows 0..pos[b] (pos[b] < cap).
+ *   Sliding layer (cap 512): attends to ring rows 0..min(pos[b], 511), which
+ *   then hold exactly positions max(0, pos[b] - 511)..pos[b].
+ *   workspace: caller-owned device scratch of at least
+ *   spark_decode_workspace_bytes(B, cap, cfg) bytes, 16-byte aligned; calls
+ *   that share a workspace must not overlap on the device. */
+int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_cache,
+                      const void* v_cache, int cap, int B, const int* pos,
+                      const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
+                      unsigned flags, void* stream);
+
+/* Synchronise `stream`, then read and clear the library's device error word
+ * on the current device.  Returns SPARK_OK, SPARK_ERR_TIMEOUT,
+ * SPARK_ERR_DEVICE_ARG or SPARK_ERR_CUDA. */
+int spark_check(void* stream);
+
+/* Text of the last error of the calling thread ("" if none). */
+const char* spark_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int spark_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARK_ATTN_H */

@@ -1,0 +1,68 @@
+"""The C-ABI library loads and exports every symbol the headers declare (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in sorted(os.listdir(inc)):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f), encoding="utf-8").read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w \*]*?\b(spark_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import __graft_entry__
+    __graft_entry__.build()
+    import full_gqa_attention_spark2_b200 as sa
+    return ctypes.CDLL(sa.lib_path())
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 12, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_binding_covers_the_header():
+    import full_gqa_attention_spark2_b200 as sa
+    assert set(sa.exported_symbols()) <= set(_declared())
+
+
+def test_host_helpers_without_a_gpu(lib):
+    import full_gqa_attention_spark2_b200 as sa
+    from oracle import spark_oracle as O
+    for layer in range(36):
+        c = sa.spark_layer_cfg_for_layer(layer)
+        assert c.kind == O.layer_kind(layer)
+        p = O.layer_params(c.kind)
+        assert c.rot_dim == p["rot"] and c.theta == p["theta"]
+        assert c.n_q == 16 and c.n_kv == 4 and c.head_dim == 256 and c.scale == 0.0625
+    with pytest.raises(sa.SparkError):
+        sa.spark_layer_cfg_for_layer(36)
+    for ctx in (1, 511, 512, 4096, 131072, 1 << 20):
+        assert sa.spark_stack_kv_bytes(1, ctx) == O.stack_kv_bytes(ctx)
+    full = sa.spark_layer_cfg_for_kind(sa.SPARK_FULL)
+    assert sa.spark_kv_cache_bytes(full, 1, 1) == O.kv_bytes_per_token_full_layer()
+    assert sa.spark_kv_cache_bytes(full, 1, 1 << 20) == 4 * 2 ** 30
+
+
+def test_calls_fail_loudly_without_a_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    import full_gqa_attention_spark2_b200 as sa
+    cfg = sa.spark_layer_cfg_for_kind(sa.SPARK_SLIDING)
+    x = torch.zeros(1, 1, 16, 256, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        sa.spark_rope_apply(x, torch.zeros(1, dtype=torch.int32), cfg)
