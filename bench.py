@@ -1,0 +1,509 @@
+"""Benchmark of the Spark2_5 hybrid GQA attention core on B200.
+
+Headline workload (one step): prefill of B=4 sequences of T=8192 tokens
+through one sliding-window layer and one full layer, q/k/v bf16 ~N(0,1) with
+k scaled 0.5, gate logits ~N(0, 2^2), positions 0..8191, seed 1.  A step runs
+the whole hot path: RoPE on q and k, the attention prefill, and the KV-cache
+append, for both layer kinds.  Secondary workload: one decode step of the
+36-layer stack for B=64 sequences with 32768 cached tokens (27 sliding layers
+with 512-slot rings, 9 full layers with linear caches), captured in one CUDA
+graph.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun each rank runs its own replica (independent sequences, no
+collective on the data path); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+SLIDING, FULL = 0, 1
+HQ, HKV, D, WINDOW = 16, 4, 256, 512
+PREFILL_B, PREFILL_T, PREFILL_SEED = 4, 8192, 1
+DECODE_B, DECODE_CTX, DECODE_SEED = 64, 32768, 3
+N_LAYERS = 36
+
+
+# ----------------------------------------------------------- work models ----
+
+def visible_pairs(T: int, pos0: int, kind: int, with_history: bool = True) -> int:
+    """Exact number of visible (query, key) pairs of a chunk of T queries at pos0."""
+    first = pos0 if not with_history else 0
+    if kind == FULL:
+        # query at pos0+t sees keys first..pos0+t
+        return T * (pos0 - first + 1) + T * (T - 1) // 2
+    total = 0
+    for t in range(T):
+        qp = pos0 + t
+        total += qp - max(first, qp - WINDOW + 1) + 1
+    return total
+
+
+def prefill_flops(B: int, T: int, pos0: int, kind: int, with_history: bool = True) -> int:
+    """Algorithmic FLOPs: 2*256 for QK^T plus 2*256 for PV per visible pair and query head."""
+    return B * visible_pairs(T, pos0, kind, with_history) * HQ * 4 * D
+
+
+def decode_kv_bytes(B: int, p: int, kind: int) -> int:
+    """Algorithmic KV bytes a decode step reads: visible keys x 4 heads x (K+V) x 256 x 2 B."""
+    keys = p + 1 if kind == FULL else min(p + 1, WINDOW)
+    return B * keys * HKV * 2 * D * 2
+
+
+# ------------------------------------------------------------- plumbing -----
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "full_gqa_attention_spark2_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernels."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(kernel)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------ our arm -------
+
+def prefill_workload(torch, sa, synth, dev):
+    """Device buffers of the headline workload for both layer kinds."""
+    B, T = PREFILL_B, PREFILL_T
+    W = {}
+    for kind, layer in ((SLIDING, 0), (FULL, 3)):
+        cfg = sa.spark_layer_cfg_for_kind(kind)
+        q = torch.empty(B, T, HQ, D, dtype=torch.bfloat16, device=dev)
+        k = torch.empty(B, T, HKV, D, dtype=torch.bfloat16, device=dev)
+        v = torch.empty_like(k)
+        g = torch.empty(B, T, HQ, dtype=torch.bfloat16, device=dev)
+        synth.fill_tokens(q, PREFILL_SEED, synth.tensor_id(layer, synth.ROLE_Q), 0)
+        synth.fill_tokens(k, PREFILL_SEED, synth.tensor_id(layer, synth.ROLE_K), 0, sigma=0.5)
+        synth.fill_tokens(v, PREFILL_SEED, synth.tensor_id(layer, synth.ROLE_V), 0)
+        synth.fill_tokens(g, PREFILL_SEED, synth.tensor_id(layer, synth.ROLE_GATE), 0, sigma=2.0)
+        cap = WINDOW if kind == SLIDING else T
+        kc = torch.empty(B, HKV, cap, D, dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+        W[kind] = dict(cfg=cfg, q=q, k=k, v=v, g=g, out=torch.empty_like(q), kc=kc, vc=vc)
+    pos0 = torch.zeros(B, dtype=torch.int32, device=dev)
+    return W, pos0
+
+
+def prefill_step(sa, W, pos0, events=None):
+    """One pass of the hot path over the batch: RoPE, prefill, append, for both layer kinds."""
+    for kind in (SLIDING, FULL):
+        w = W[kind]
+        sa.spark_rope_apply(w["q"], pos0, w["cfg"])
+        sa.spark_rope_apply(w["k"], pos0, w["cfg"])
+        if events is not None and kind == FULL:
+            events[0].record()
+        sa.spark_attn_prefill(w["out"], w["q"], w["k"], w["v"], w["g"], None, None, pos0, w["cfg"])
+        if events is not None and kind == FULL:
+            events[1].record()
+        sa.spark_kv_append(w["kc"], w["vc"], w["k"], w["v"], pos0, w["cfg"])
+
+
+def timed_region(torch, dist, fn, steps):
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        fn(i)
+    t1.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    if dist is not None:
+        x = torch.tensor([ms], device="cuda")
+        dist.all_reduce(x, op=dist.ReduceOp.MAX)
+        ms = float(x.item())
+    return ms
+
+
+def run_prefill(torch, sa, synth, dist, args, peaks, world):
+    dev = torch.device("cuda")
+    W, pos0 = prefill_workload(torch, sa, synth, dev)
+    for _ in range(args.warmup):
+        prefill_step(sa, W, pos0)
+    sa.spark_check()
+    # per-launch duration of the full-layer prefill kernel, on its stream
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    ms = timed_region(torch, dist, lambda i: prefill_step(sa, W, pos0, pairs[i]), args.steps)
+    clk = clocks.stop()
+    sa.spark_check()
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+    B, T = PREFILL_B, PREFILL_T
+    f_full = prefill_flops(B, T, 0, FULL, False)
+    f_slide = prefill_flops(B, T, 0, SLIDING, False)
+    ms_step = ms / args.steps
+    tokens = B * T * world
+    achieved = f_full / (kern_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+
+    # end to end: pinned host inputs -> device, the path, outputs -> pinned host
+    host_in = {kind: {n: torch.empty(W[kind][n].shape, dtype=torch.bfloat16, pin_memory=True)
+                      for n in ("q", "k", "v", "g")} for kind in W}
+    host_out = {kind: torch.empty(W[kind]["out"].shape, dtype=torch.bfloat16, pin_memory=True) for kind in W}
+    for kind in W:
+        for n in ("q", "k", "v", "g"):
+            host_in[kind][n].copy_(W[kind][n])
+    h2d = sum(t.numel() * 2 for kind in W for t in host_in[kind].values())
+    d2h = sum(t.numel() * 2 for t in host_out.values())
+
+    def e2e_step(i):
+        for kind in W:
+            for n in ("q", "k", "v", "g"):
+                W[kind][n].copy_(host_in[kind][n], non_blocking=True)
+        prefill_step(sa, W, pos0)
+        for kind in W:
+            host_out[kind].copy_(W[kind]["out"], non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step(0)
+    ms_e2e = timed_region(torch, dist, e2e_step, e2e_steps)
+    sa.spark_check()
+    del W
+    torch.cuda.empty_cache()
+    return {
+        "metric": "prefill attn tok/s & TFLOP/s; decode KV-read GB/s (36-layer stack); % roofline",
+        "value": tokens / (ms_step * 1e-3),
+        "unit": "tok/s",
+        "ms_per_step": ms_step,
+        "tflops": (f_full + f_slide) * world / (ms_step * 1e-3) / 1e12,
+        "prefill_full_kernel": {"ms": kern_ms, "tflops": achieved, "flops": f_full},
+        "roofline": {"bound": "tensor", "kernel": "prefill_kernel (full layer)", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"bf16_tflops burst, {peaks['source']}",
+                     "traffic": ncu_traffic("prefill_kernel_full")},
+        "e2e": {"value": tokens / (ms_e2e / e2e_steps * 1e-3), "unit": "tok/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk,
+        "gpu_launches": 8 * args.steps,
+    }
+
+
+def run_decode(torch, sa, synth, dist, args, peaks, world):
+    """One decode step of the 36-layer stack, B=64, 32768 cached tokens, in one CUDA graph."""
+    dev = torch.device("cuda")
+    B, p = DECODE_B, DECODE_CTX
+    layers = []
+    for l in range(N_LAYERS):
+        kind = FULL if l % 4 == 3 else SLIDING
+        cfg = sa.spark_layer_cfg_for_kind(kind)
+        cap = WINDOW if kind == SLIDING else p + 1
+        kc = torch.empty(B, HKV, cap, D, dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+        synth.fill_cache(kc, DECODE_SEED, synth.tensor_id(l, synth.ROLE_K), p, kind == SLIDING)
+        synth.fill_cache(vc, DECODE_SEED, synth.tensor_id(l, synth.ROLE_V), p, kind == SLIDING)
+        q = torch.empty(B, 1, HQ, D, dtype=torch.bfloat16, device=dev)
+        kn = torch.empty(B, 1, HKV, D, dtype=torch.bfloat16, device=dev)
+        vn = torch.empty_like(kn)
+        g = torch.empty(B, 1, HQ, dtype=torch.bfloat16, device=dev)
+        synth.fill_tokens(q, DECODE_SEED, synth.tensor_id(l, synth.ROLE_Q), p)
+        synth.fill_tokens(kn, DECODE_SEED, synth.tensor_id(l, synth.ROLE_K), p)
+        synth.fill_tokens(vn, DECODE_SEED, synth.tensor_id(l, synth.ROLE_V), p)
+        synth.fill_tokens(g, DECODE_SEED, synth.tensor_id(l, synth.ROLE_GATE), p)
+        layers.append(dict(kind=kind, cfg=cfg, cap=cap, kc=kc, vc=vc, q=q.view(B, HQ, D), kn=kn, vn=vn,
+                           g=g.view(B, HQ), out=torch.empty(B, HQ, D, dtype=torch.bfloat16, device=dev)))
+    pos = torch.full((B,), p, dtype=torch.int32, device=dev)
+    ws_bytes = max(sa.spark_decode_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def step():
+        for L in layers:
+            sa.spark_kv_append(L["kc"], L["vc"], L["kn"], L["vn"], pos, L["cfg"], flags=sa.SPARK_ROPE_FUSED)
+            sa.spark_attn_decode(L["out"], L["q"], L["g"], L["kc"], L["vc"], pos, L["cfg"], ws,
+                                 flags=sa.SPARK_ROPE_FUSED)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    sa.spark_check()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    dsteps = max(5, min(args.steps, 30))
+    ms = timed_region(torch, dist, lambda i: graph.replay(), dsteps)
+    sa.spark_check()
+    ms_step = ms / dsteps
+    # one full layer's decode alone (append + partial + combine), eager, for the roofline
+    full = layers[3]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    e0.record()
+    for _ in range(reps):
+        sa.spark_attn_decode(full["out"], full["q"], full["g"], full["kc"], full["vc"], pos, full["cfg"], ws,
+                             flags=sa.SPARK_ROPE_FUSED)
+    e1.record()
+    torch.cuda.synchronize()
+    k_ms = e0.elapsed_time(e1) / reps
+    total_bytes = sum(decode_kv_bytes(B, p, L["kind"]) for L in layers)
+    full_bytes = decode_kv_bytes(B, p, FULL)
+    del graph, layers, ws
+    torch.cuda.empty_cache()
+    return {
+        "value": total_bytes * world / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
+        "ms_per_step": ms_step, "steps_per_s": 1e3 / ms_step, "kv_bytes_per_step": total_bytes,
+        "workload": f"decode_b{B}_ctx{p}_36layers", "gpu_launches_per_step": 3 * N_LAYERS,
+        "roofline": {"bound": "hbm", "kernel": "decode_partial_kernel+combine (full layer)",
+                     "achieved": full_bytes / (k_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": full_bytes / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "traffic": ncu_traffic("decode_partial_kernel_full")},
+    }
+
+
+# ------------------------------------------------------- oracle timing -------
+
+def oracle_prefill_rate(budget_s: float = 15.0):
+    """The fp64 oracle on a bounded sample of the headline workload: query rows of
+    sequence 0 through both layers (all 16 heads); returns (tok/s, threads, description)."""
+    import synth
+    from oracle import spark_oracle as O
+    T = PREFILL_T
+    pos = np.arange(T)
+    layer_of = {SLIDING: 0, FULL: 3}
+
+    def get(kind, role, H, Dd, p, sig=1.0):
+        return synth.bf16_bits_to_f64(
+            synth.token_tensor(PREFILL_SEED, synth.tensor_id(layer_of[kind], role), 1, H, Dd, p, sig)[0])
+
+    kv = {kind: (get(kind, synth.ROLE_K, HKV, D, pos, 0.5), get(kind, synth.ROLE_V, HKV, D, pos)) for kind in layer_of}
+    rng = np.random.default_rng(0)
+    done, t_used = 0, 0.0
+    while t_used < budget_s or done < 2:
+        rows = np.sort(rng.integers(0, T, size=2))
+        for kind in (SLIDING, FULL):
+            q_rows = get(kind, synth.ROLE_Q, HQ, D, rows)
+            g_rows = get(kind, synth.ROLE_GATE, HQ, 1, rows, 2.0)
+            t0 = time.perf_counter()
+            O.layer_prefill_rows(q_rows, kv[kind][0], kv[kind][1], g_rows, pos, kind, rows)
+            t_used += time.perf_counter() - t0
+        done += len(rows)
+    threads = None
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        threads = os.cpu_count()
+    return done / t_used, threads, f"{done} random query rows of sequence 0 through both layers, {t_used:.1f} s"
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    rate, threads, sample = oracle_prefill_rate(budget_s=max(5.0, min(60.0, 3.0 * args.steps)))
+    line = {
+        "impl": "reference", "metric": "prefill attn tok/s & TFLOP/s; decode KV-read GB/s (36-layer stack); % roofline",
+        "value": rate, "unit": "tok/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": PREFILL_B * PREFILL_T / rate * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "prefill_b4_t8192_sliding+full", "B": PREFILL_B, "T": PREFILL_T},
+        "cpu_baseline": {"value": rate, "unit": "tok/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": rate, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- main -----
+
+def run_profile_case(torch, sa, synth, which: str):
+    """A small case for ncu: one warm-up and two launches of one kernel, nothing timed.
+
+    prefill_full / prefill_sliding: B=4, T=8192 (q alone 268 MB > L2);
+    decode_full: B=16, 32768 cached tokens, one full layer (2.1 GB of KV)."""
+    dev = torch.device("cuda")
+    if which.startswith("prefill"):
+        kind = FULL if which == "prefill_full" else SLIDING
+        W, pos0 = prefill_workload(torch, sa, synth, dev)
+        w = W[kind]
+        sa.spark_rope_apply(w["q"], pos0, w["cfg"])
+        sa.spark_rope_apply(w["k"], pos0, w["cfg"])
+        for _ in range(3):
+            sa.spark_attn_prefill(w["out"], w["q"], w["k"], w["v"], w["g"], None, None, pos0, w["cfg"])
+    elif which == "decode_full":
+        B, p = 16, DECODE_CTX
+        cfg = sa.spark_layer_cfg_for_kind(FULL)
+        kc = torch.empty(B, HKV, p + 1, D, dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+        synth.fill_cache(kc, DECODE_SEED, synth.tensor_id(3, synth.ROLE_K), p + 1, False)
+        synth.fill_cache(vc, DECODE_SEED, synth.tensor_id(3, synth.ROLE_V), p + 1, False)
+        q = torch.empty(B, 1, HQ, D, dtype=torch.bfloat16, device=dev)
+        g = torch.empty(B, 1, HQ, dtype=torch.bfloat16, device=dev)
+        synth.fill_tokens(q, DECODE_SEED, synth.tensor_id(3, synth.ROLE_Q), p)
+        synth.fill_tokens(g, DECODE_SEED, synth.tensor_id(3, synth.ROLE_GATE), p)
+        out = torch.empty(B, HQ, D, dtype=torch.bfloat16, device=dev)
+        pos = torch.full((B,), p, dtype=torch.int32, device=dev)
+        ws = torch.empty(sa.spark_decode_workspace_bytes(B, p + 1, cfg), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            sa.spark_attn_decode(out, q.view(B, HQ, D), g.view(B, HQ), kc, vc, pos, cfg, ws, flags=sa.SPARK_ROPE_FUSED)
+    else:
+        raise SystemExit(f"unknown profile case {which}")
+    sa.spark_check()
+    print(json.dumps({"profile_case": which, "ok": True}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["prefill_full", "prefill_sliding", "decode_full"], default=None,
+                    help="run a small case of one kernel for ncu and exit")
+    args = ap.parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+    import full_gqa_attention_spark2_b200 as sa
+    import synth
+    sa._lib()
+    synth.load_lib()
+    peaks = load_peaks()
+    if args.profile:
+        run_profile_case(torch, sa, synth, args.profile)
+        return
+
+    res = run_prefill(torch, sa, synth, dist, args, peaks, world)
+    dec = None if args.no_decode else run_decode(torch, sa, synth, dist, args, peaks, world)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, threads, sample = oracle_prefill_rate()
+        cpu = {"value": rate, "unit": "tok/s", "cores": threads, "kind": "oracle", "sample": sample}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": res["metric"], "value": res["value"], "unit": res["unit"], "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded counter generator, shapes of the pages' workloads)",
+        "config": {"workload": "prefill_b4_t8192_sliding+full", "B": PREFILL_B, "T": PREFILL_T,
+                   "layers": ["sliding (window 512, rope theta 1e4, 256 dims)",
+                              "full (rope theta 5e6, first 64 dims)"],
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (q alone is 268 MB per layer); no flush"},
+        "tflops": res["tflops"], "prefill_full_kernel": res["prefill_full_kernel"],
+        "roofline": res["roofline"], "e2e": res["e2e"], "clocks": res["clocks"],
+        "gpu_launches": res["gpu_launches"] + (0 if dec is None else 0),
+        "cpu_baseline": cpu, "decode": dec,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -202,16 +202,18 @@ def layer_prefill(q, k, v, gate, pos, kind: int, hist_k=None, hist_v=None, hist_
     return attention(qr, kr, v, gate, pos, kpos, kind)
 
 
-def layer_prefill_rows(q, k, v, gate, pos, kind: int, rows, hist_k=None, hist_v=None, hist_pos=None):
+def layer_prefill_rows(q_rows, k, v, gate_rows, pos, kind: int, rows, hist_k=None, hist_v=None, hist_pos=None):
     """``layer_prefill`` evaluated at the query rows ``rows`` only.
 
-    Each selected query is computed exactly as in ``layer_prefill``: it sees the
+    q_rows [len(rows),16,256] and gate_rows [len(rows),16] are the raw queries
+    and gate logits of those rows; k, v, pos are the whole chunk's.  Each
+    selected query is computed exactly as in ``layer_prefill``: it sees the
     same keys and gets the same rotation; the other queries are simply not
     evaluated.  Used where the full oracle would take too long.
     """
     rows = np.asarray(rows, dtype=np.int64)
     pos = np.asarray(pos, dtype=np.int64)
-    qr = rope(np.asarray(q)[rows], pos[rows], kind)
+    qr = rope(q_rows, pos[rows], kind)
     kr = rope(k, pos, kind)
     v = np.asarray(v, dtype=np.float64)
     if hist_k is not None and len(hist_pos) > 0:
@@ -220,7 +222,7 @@ def layer_prefill_rows(q, k, v, gate, pos, kind: int, rows, hist_k=None, hist_v=
         kpos = np.concatenate([np.asarray(hist_pos, dtype=np.int64), pos])
     else:
         kpos = pos
-    return attention(qr, kr, v, np.asarray(gate)[rows], pos[rows], kpos, kind)
+    return attention(qr, kr, v, gate_rows, pos[rows], kpos, kind)
 
 
 def layer_decode(q, k_new, v_new, gate, p: int, kind: int, hist_k, hist_v, hist_pos):

@@ -277,7 +277,8 @@ def test_chunked_prefill_equals_one_pass(kind):
     two = O.layer_prefill(q[c:], k[c:], v[c:], g[c:], pos[c:], kind, hist_k, v[:c], pos[:c])
     np.testing.assert_allclose(two, one[c:], rtol=1e-12, atol=1e-13)
     rows = np.array([0, 1, 255, 511, 512, 513, T - 1])
-    np.testing.assert_allclose(O.layer_prefill_rows(q, k, v, g, pos, kind, rows), one[rows], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(O.layer_prefill_rows(q[rows], k, v, g[rows], pos, kind, rows), one[rows],
+                               rtol=1e-12, atol=1e-14)
 
 
 # ------------------------------------------------------------- KV cache -----
