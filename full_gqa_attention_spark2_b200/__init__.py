@@ -66,6 +66,7 @@ def _lib():
         "spark_attn_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
         "spark_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
         "spark_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, cfgp, _P, ctypes.c_size_t, ctypes.c_uint, _P]),
+        "spark_attn_decode_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
         "spark_check": (_I, [_P]),
         "spark_last_error": (ctypes.c_char_p, []),
         "spark_version": (_I, []),
@@ -82,7 +83,8 @@ def exported_symbols():
     """Names of the C entry points this binding expects the library to export."""
     return ["spark_layer_cfg_for_layer", "spark_layer_cfg_for_kind", "spark_kv_cache_bytes",
             "spark_stack_kv_bytes", "spark_rope_apply", "spark_kv_append", "spark_attn_prefill",
-            "spark_decode_workspace_bytes", "spark_attn_decode", "spark_check", "spark_last_error",
+            "spark_decode_workspace_bytes", "spark_attn_decode", "spark_attn_decode_static", "spark_check",
+            "spark_last_error",
             "spark_version"]
 
 
@@ -190,6 +192,20 @@ def spark_attn_decode(out, q, gate, k_cache, v_cache, pos, cfg: SparkLayerCfg, w
     cap = k_cache.shape[2]
     _raise(_lib().spark_attn_decode(po, pq, pg, pkc, pvc, cap, B, pp, ctypes.byref(cfg), workspace.data_ptr(),
                                     ws_bytes, flags, _stream(stream)))
+
+
+def spark_attn_decode_static(out, q, gate, k_cache, v_cache, pos, cfg: SparkLayerCfg, flags: int = 0,
+                             stream=None) -> None:
+    """Decode like spark_attn_decode, but without a workspace: for callers that cannot allocate.
+
+    The split partials live in the library's fixed device scratch array, shared
+    by all calls; calls that overlap on the device race on it."""
+    po, pq = _dev(out, "out", ndim=3), _dev(q, "q", ndim=3)
+    pg = _dev(gate, "gate", ndim=2)
+    pkc, pvc = _dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4)
+    pp = _dev(pos, "pos", torch.int32, 1)
+    _raise(_lib().spark_attn_decode_static(po, pq, pg, pkc, pvc, k_cache.shape[2], q.shape[0], pp,
+                                           ctypes.byref(cfg), flags, _stream(stream)))
 
 
 def spark_check(stream=None) -> None:

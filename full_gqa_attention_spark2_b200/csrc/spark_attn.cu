@@ -181,6 +181,37 @@ size_t decode_ws_bytes(int B, const DecodePlan& pl) {
   return rows * spark::kHeadDim * sizeof(float) + rows * 2 * sizeof(float);
 }
 
+// ------------------------------------------------- decode without workspace ----
+// Some callers cannot allocate device memory when they run attention: a
+// serving runtime that plans all of its memory at start-up and forbids any
+// allocation afterwards, a host application that only lends the library its
+// input and output buffers, or code that runs while a stream is being recorded
+// into a CUDA graph, where cudaMalloc cannot be recorded.  For them
+// spark_attn_decode_static keeps the split-KV partials in this fixed array of
+// the library's own device memory instead of a caller workspace.  Every GPU
+// that loads the library holds these 16 MiB until the process exits.
+constexpr size_t kStaticScratchBytes = (size_t)SPARK_STATIC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+struct StaticScratch {
+  std::once_flag once;
+  void* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+StaticScratch g_scratch[kMaxDevices];
+
+// Device address of the scratch array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is asked of the
+// runtime once per device, with that device current.
+int static_scratch(int dev, void** out) {
+  StaticScratch& s = g_scratch[dev];
+  std::call_once(s.once, [&]() { s.err = cudaGetSymbolAddress(&s.ptr, g_decode_scratch); });
+  if (s.err != cudaSuccess || s.ptr == nullptr)
+    return cuda_fail(s.err != cudaSuccess ? s.err : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
+  *out = s.ptr;
+  return SPARK_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -409,6 +440,70 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
       qm, km, vm, kcm, vcm, P);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "prefill_kernel launch");
+}
+
+int spark_attn_decode_static(void* out, const void* q, const void* gate, const void* k_cache,
+                             const void* v_cache, int cap, int B, const int* pos,
+                             const spark_layer_cfg* cfg, unsigned flags, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!out || !q || !gate || !k_cache || !v_cache || !pos) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B > 65535 || cap <= 0) return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d cap=%d", B, cap);
+  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
+  if (!sliding && cap > SPARK_MAX_POSITION) return fail(SPARK_ERR_INVALID_ARG, "cap above 2^20");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(SPARK_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  // one split needs a partial row (256 + 2 floats) per sequence and query head
+  const size_t per_split = (size_t)B * spark::kNq * (spark::kHeadDim + 2) * sizeof(float);
+  if (per_split > kStaticScratchBytes)
+    return fail(SPARK_ERR_INVALID_ARG,
+                "B=%d needs %zu bytes of scratch, above the %zu-byte static scratch (at most %zu sequences)",
+                B, per_split, kStaticScratchBytes,
+                kStaticScratchBytes / ((size_t)spark::kNq * (spark::kHeadDim + 2) * sizeof(float)));
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  void* scratch = nullptr;
+  if ((rc = static_scratch(dev, &scratch))) return rc;
+  // the usual split plan, with fewer splits when its partials would not fit
+  DecodePlan pl = decode_plan(B, cap, sliding, g_dev[dev].sm_count);
+  if (decode_ws_bytes(B, pl) > kStaticScratchBytes) {
+    const int tiles = ((sliding ? SPARK_WINDOW : cap) + spark::kDecNK - 1) / spark::kDecNK;
+    const int s_fit = (int)(kStaticScratchBytes / per_split);
+    pl.tiles_per_split = (tiles + s_fit - 1) / s_fit;
+    pl.n_splits = (tiles + pl.tiles_per_split - 1) / pl.tiles_per_split;
+  }
+
+  CUtensorMap km, vm;
+  const cuuint64_t dims[3] = {256, (cuuint64_t)cap, (cuuint64_t)B * 4};
+  const cuuint64_t strides[2] = {512, (cuuint64_t)cap * 512};
+  const cuuint32_t box[3] = {64, (cuuint32_t)spark::kDecNK, 1};
+  if ((rc = make_map(&km, k_cache, 3, dims, strides, box))) return rc;
+  if ((rc = make_map(&vm, v_cache, 3, dims, strides, box))) return rc;
+
+  spark::DecodeParams P;
+  P.q = (const __nv_bfloat16*)q;
+  P.pos = pos;
+  P.o_part = (float*)scratch;
+  P.ml_part = (float*)scratch + (size_t)B * spark::kNq * pl.n_splits * spark::kHeadDim;
+  P.B = B;
+  P.cap = cap;
+  P.sliding = sliding;
+  P.n_splits = pl.n_splits;
+  P.tiles_per_split = pl.tiles_per_split;
+  P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
+  P.rot = cfg->rot_dim;
+  P.log2_theta = log2(cfg->theta);
+  P.timeout_ns = wait_timeout_ns();
+  spark::decode_partial_kernel<<<dim3(pl.n_splits, spark::kNkv, B), spark::kDecThreads, spark::kDecSmemBytes,
+                                 (cudaStream_t)stream>>>(km, vm, P);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode_partial_kernel launch");
+  spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, (cudaStream_t)stream>>>(
+      (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_combine_kernel launch");
 }
 
 int spark_check(void* stream) {

@@ -154,6 +154,32 @@ int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_
                       const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
                       unsigned flags, void* stream);
 
+/* Size of the fixed scratch array spark_attn_decode_static uses. */
+#define SPARK_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* Decode for callers that cannot allocate device memory (no counterpart on the
+ * pages; it exists for such callers).  Some hosts plan all device memory up
+ * front and forbid allocation later, some only lend the library their inputs
+ * and outputs, and code recording a CUDA graph cannot record cudaMalloc.  This
+ * call computes exactly what spark_attn_decode computes, with the same
+ * arguments minus the workspace: the split-KV partials go to a fixed
+ * SPARK_STATIC_SCRATCH_BYTES array in the library's own device memory, which
+ * every GPU that loads the library holds until the process exits.  It calls no
+ * allocating routine.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, once per device, with that device current); make
+ *     that first call before any stream capture.
+ *   - One split needs B * 16 * 258 * 4 bytes, so B may be at most 1016; larger
+ *     batches are rejected with SPARK_ERR_INVALID_ARG.  When the usual split
+ *     plan does not fit, fewer splits are used.
+ *   - All calls share the array and it keeps the last call's contents; nothing
+ *     in it needs to start at zero, because every partial a call reads is
+ *     written by the same call.  Calls that overlap on the device (other
+ *     streams, or other host threads) race on it: serialise them. */
+int spark_attn_decode_static(void* out, const void* q, const void* gate, const void* k_cache,
+                             const void* v_cache, int cap, int B, const int* pos,
+                             const spark_layer_cfg* cfg, unsigned flags, void* stream);
+
 /* Synchronise `stream`, then read and clear the library's device error word
  * on the current device.  Returns SPARK_OK, SPARK_ERR_TIMEOUT,
  * SPARK_ERR_DEVICE_ARG or SPARK_ERR_CUDA. */
