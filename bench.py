@@ -276,38 +276,49 @@ def run_prefill(torch, sa, synth, dist, args, peaks, world):
     }
 
 
-def run_decode(torch, sa, synth, dist, args, peaks, world):
-    """One decode step of the 36-layer stack, B=64, 32768 cached tokens, in one CUDA graph."""
-    dev = torch.device("cuda")
-    B, p = DECODE_B, DECODE_CTX
+def decode_layers(torch, sa, synth, dev, B: int, p: int, layer_ids=range(N_LAYERS), seed: int = DECODE_SEED):
+    """Caches holding positions 0..p-1 and the new token's q/k/v/gate at p, per layer."""
     layers = []
-    for l in range(N_LAYERS):
+    for l in layer_ids:
         kind = FULL if l % 4 == 3 else SLIDING
         cfg = sa.spark_layer_cfg_for_kind(kind)
         cap = WINDOW if kind == SLIDING else p + 1
         kc = torch.empty(B, HKV, cap, D, dtype=torch.bfloat16, device=dev)
         vc = torch.empty_like(kc)
-        synth.fill_cache(kc, DECODE_SEED, synth.tensor_id(l, synth.ROLE_K), p, kind == SLIDING)
-        synth.fill_cache(vc, DECODE_SEED, synth.tensor_id(l, synth.ROLE_V), p, kind == SLIDING)
+        synth.fill_cache(kc, seed, synth.tensor_id(l, synth.ROLE_K), p, kind == SLIDING)
+        synth.fill_cache(vc, seed, synth.tensor_id(l, synth.ROLE_V), p, kind == SLIDING)
         q = torch.empty(B, 1, HQ, D, dtype=torch.bfloat16, device=dev)
         kn = torch.empty(B, 1, HKV, D, dtype=torch.bfloat16, device=dev)
         vn = torch.empty_like(kn)
         g = torch.empty(B, 1, HQ, dtype=torch.bfloat16, device=dev)
-        synth.fill_tokens(q, DECODE_SEED, synth.tensor_id(l, synth.ROLE_Q), p)
-        synth.fill_tokens(kn, DECODE_SEED, synth.tensor_id(l, synth.ROLE_K), p)
-        synth.fill_tokens(vn, DECODE_SEED, synth.tensor_id(l, synth.ROLE_V), p)
-        synth.fill_tokens(g, DECODE_SEED, synth.tensor_id(l, synth.ROLE_GATE), p)
-        layers.append(dict(kind=kind, cfg=cfg, cap=cap, kc=kc, vc=vc, q=q.view(B, HQ, D), kn=kn, vn=vn,
+        synth.fill_tokens(q, seed, synth.tensor_id(l, synth.ROLE_Q), p)
+        synth.fill_tokens(kn, seed, synth.tensor_id(l, synth.ROLE_K), p)
+        synth.fill_tokens(vn, seed, synth.tensor_id(l, synth.ROLE_V), p)
+        synth.fill_tokens(g, seed, synth.tensor_id(l, synth.ROLE_GATE), p)
+        layers.append(dict(layer=l, kind=kind, cfg=cfg, cap=cap, kc=kc, vc=vc, q=q.view(B, HQ, D), kn=kn, vn=vn,
                            g=g.view(B, HQ), out=torch.empty(B, HQ, D, dtype=torch.bfloat16, device=dev)))
+    return layers
+
+
+def decode_step(sa, layers, pos, ws):
+    """One decode step: per layer, append the new token (RoPE fused on k), then attend (RoPE fused on q)."""
+    for L in layers:
+        sa.spark_kv_append(L["kc"], L["vc"], L["kn"], L["vn"], pos, L["cfg"], flags=sa.SPARK_ROPE_FUSED)
+        sa.spark_attn_decode(L["out"], L["q"], L["g"], L["kc"], L["vc"], pos, L["cfg"], ws,
+                             flags=sa.SPARK_ROPE_FUSED)
+
+
+def run_decode(torch, sa, synth, dist, args, peaks, world):
+    """One decode step of the 36-layer stack, B=64, 32768 cached tokens, in one CUDA graph."""
+    dev = torch.device("cuda")
+    B, p = DECODE_B, DECODE_CTX
+    layers = decode_layers(torch, sa, synth, dev, B, p)
     pos = torch.full((B,), p, dtype=torch.int32, device=dev)
     ws_bytes = max(sa.spark_decode_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
 
     def step():
-        for L in layers:
-            sa.spark_kv_append(L["kc"], L["vc"], L["kn"], L["vn"], pos, L["cfg"], flags=sa.SPARK_ROPE_FUSED)
-            sa.spark_attn_decode(L["out"], L["q"], L["g"], L["kc"], L["vc"], pos, L["cfg"], ws,
-                                 flags=sa.SPARK_ROPE_FUSED)
+        decode_step(sa, layers, pos, ws)
 
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())

@@ -113,11 +113,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         issued = i + 1;
       }
       // Never leave with copies in flight: wait for the last issued tiles to land.
-      for (int i = max(0, issued - kDecStages); i < issued; ++i) {
-        volatile int no_abort = 0;
-        if (!mbar_wait(bar_full + 8 * (i % kDecStages), (i / kDecStages) & 1, &no_abort, 200000000ull, 0x11u))
-          break;
-      }
+      for (int i = max(0, issued - kDecStages); i < issued; ++i)
+        if (!mbar_drain(bar_full + 8 * (i % kDecStages), (i / kDecStages) & 1, 200000000ull)) break;
     }
     return;
   }
@@ -170,7 +167,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   for (int i = 0; i < n_tiles; ++i) {
     const int s = i % kDecStages;
-    if (!mbar_wait(bar_full + 8 * s, (i / kDecStages) & 1, abort_flag, P.timeout_ns, 0x12u)) break;
+    // warp-uniform outcome: ldmatrix / mma.sync below need every lane
+    if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, (i / kDecStages) & 1, abort_flag, P.timeout_ns, 0x12u)))
+      break;
     const uint32_t kt = base + s * kDecStageBytes;
     const uint32_t vt = kt + kDecTileBytes;
 

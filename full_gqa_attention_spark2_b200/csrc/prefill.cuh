@@ -214,11 +214,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
       }
       // never leave with copies in flight
-      volatile int no_abort = 0;
-      if (mbar_wait(bar_q, 0, &no_abort, 200000000ull, 0x21u)) {
+      if (mbar_drain(bar_q, 0, 200000000ull)) {
         for (int i = max(0, li - kPfSlots); i < li; ++i)
-          if (!mbar_wait(bar_slot_full + 8 * (i % kPfSlots), (i / kPfSlots) & 1, &no_abort, 200000000ull, 0x22u))
-            break;
+          if (!mbar_drain(bar_slot_full + 8 * (i % kPfSlots), (i / kPfSlots) & 1, 200000000ull)) break;
       }
     }
     __syncwarp();
@@ -274,8 +272,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       // every MMA issued so far has completed before TMEM is released
       umma_commit(bar_done);
-      volatile int no_abort = 0;
-      mbar_wait(bar_done, 0, &no_abort, 200000000ull, 0x34u);
+      mbar_drain(bar_done, 0, 200000000ull);
     }
     __syncwarp();
   } else if (n > 0 && warp >= 4) {
@@ -289,7 +286,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     float m_ref = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      if (!mbar_wait(bar_s + 8 * (j & 1), (j >> 1) & 1, abort_flag, P.timeout_ns, 0x40u)) {
+      // warp-uniform outcomes: tcgen05.ld / st below need every lane of the warp
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s + 8 * (j & 1), (j >> 1) & 1, abort_flag, P.timeout_ns, 0x40u))) {
         ok = false;
         break;
       }
@@ -334,7 +332,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const bool need_o = resc && l_run > 0.f;
       if (__any_sync(0xffffffffu, need_o)) {
         // O must hold PV_{j-1} before it is rescaled
-        if (!mbar_wait(bar_o + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, P.timeout_ns, 0x41u)) {
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(bar_o + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, P.timeout_ns, 0x41u))) {
           ok = false;
           break;
         }
@@ -370,7 +369,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p + 8 * (j & 1));
     }
-    if (ok && mbar_wait(bar_o + 8 * ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, P.timeout_ns, 0x42u)) {
+    if (ok && __all_sync(0xffffffffu,
+                         mbar_wait(bar_o + 8 * ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, P.timeout_ns, 0x42u))) {
       tc_fence_after();
       float scale = 0.f;
       __nv_bfloat16* dst = nullptr;

@@ -183,6 +183,31 @@ def attention(q, k, v, gate, qpos, kpos, kind: int) -> np.ndarray:
     return out
 
 
+def attention_group(q, k, v, gate, qpos, kpos, kind: int) -> np.ndarray:
+    """The same gated attention for one GQA group only: the 4 query heads that share one KV head.
+
+    q [Tq,4,256] and k [Tk,256] already rotated, v [Tk,256], gate [Tq,4];
+    returns [Tq,4,256].  Identical, head by head, to ``attention`` restricted
+    to heads 4g..4g+3 with KV head g; it exists so that long contexts need the
+    keys of one KV head only.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    vis = visible(qpos, kpos, kind)
+    scale = 1.0 / np.sqrt(HEAD_DIM)
+    g = sigmoid(gate)
+    out = np.zeros((q.shape[0], GROUP, HEAD_DIM), dtype=np.float64)
+    for j in range(GROUP):
+        s = (q[:, j, :] @ k.T) * scale
+        s = np.where(vis, s, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        e = np.where(vis, np.exp(s - m), 0.0)
+        p = e / e.sum(axis=1, keepdims=True)
+        out[:, j, :] = (p @ v) * g[:, j][:, None]
+    return out
+
+
 def layer_prefill(q, k, v, gate, pos, kind: int, hist_k=None, hist_v=None, hist_pos=None):
     """One layer's attention for a chunk of tokens with raw (unrotated) q, k.
 

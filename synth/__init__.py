@@ -87,8 +87,22 @@ def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
 
 
 def bf16_values(seed: int, tid: int, index: np.ndarray, sigma: float = 1.0) -> np.ndarray:
-    """bf16 bit patterns (uint16) at the given flat indices."""
-    return f32_to_bf16_bits(values_f32(seed, tid, index, sigma))
+    """bf16 bit patterns (uint16) at the given flat indices (large requests run on a thread pool)."""
+    idx = np.asarray(index, dtype=np.uint64)
+    n = idx.size
+    chunk = 1 << 20
+    if n <= 2 * chunk:
+        return f32_to_bf16_bits(values_f32(seed, tid, idx, sigma))
+    from concurrent.futures import ThreadPoolExecutor
+    flat = idx.reshape(-1)
+    out = np.empty(n, dtype=np.uint16)
+
+    def work(lo):
+        out[lo:lo + chunk] = f32_to_bf16_bits(values_f32(seed, tid, flat[lo:lo + chunk], sigma))
+
+    with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        list(ex.map(work, range(0, n, chunk)))
+    return out.reshape(idx.shape)
 
 
 def token_index(B: int, H: int, D: int, pos: np.ndarray, b_idx=None, h_idx=None) -> np.ndarray:

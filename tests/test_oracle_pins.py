@@ -326,3 +326,15 @@ def test_ring_after_append_holds_exactly_the_sliding_window(p):
     window = set(int(j) for j in np.nonzero(O.visible(np.array([p]), np.arange(p + 1), O.SLIDING)[0])[0])
     assert held == window
     assert all(O.cache_slot(j, O.FULL) == j for j in (0, 5, (1 << 20) - 1))
+
+
+@pytest.mark.parametrize("kind", [O.SLIDING, O.FULL])
+def test_group_attention_equals_the_full_form(kind):
+    T = 530
+    pos = np.arange(T) + 7
+    q, k, v, g = _rand(T, 16, 256), _rand(T, 4, 256), _rand(T, 4, 256), _rand(T, 16)
+    full = O.attention(q, k, v, g, pos, pos, kind)
+    for grp in range(4):
+        hs = slice(4 * grp, 4 * grp + 4)
+        part = O.attention_group(q[:, hs], k[:, grp], v[:, grp], g[:, hs], pos, pos, kind)
+        np.testing.assert_allclose(part, full[:, hs], rtol=1e-12, atol=1e-14)
