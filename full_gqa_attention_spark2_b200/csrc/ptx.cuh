@@ -67,14 +67,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
       : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+// One potentially suspending test of an mbarrier phase; the thread sleeps at
+// most `hint_ns` nanoseconds (the suspendTimeHint operand) before it returns.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uint32_t hint_ns = 10000000u) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -85,10 +87,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // role of the block leaves its loop instead of waiting forever.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t timeout_ns, unsigned where) {
-  if (mbar_try_wait(bar, parity)) return true;
+  // never sleep inside one test for longer than the whole wait may last
+  const uint32_t hint = timeout_ns < 10000000ull ? (uint32_t)timeout_ns : 10000000u;
+  if (mbar_try_wait(bar, parity, hint)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity, hint)) return true;
     if ((it & 63u) == 0u) {
       if (*abort) return false;
       if (*reinterpret_cast<volatile unsigned*>(&g_error_word) & kErrTimeout) {
