@@ -67,6 +67,7 @@ def _lib():
         "spark_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
         "spark_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, cfgp, _P, ctypes.c_size_t, ctypes.c_uint, _P]),
         "spark_attn_decode_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
+        "spark_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
         "spark_check": (_I, [_P]),
         "spark_last_error": (ctypes.c_char_p, []),
         "spark_version": (_I, []),
@@ -83,7 +84,7 @@ def exported_symbols():
     """Names of the C entry points this binding expects the library to export."""
     return ["spark_layer_cfg_for_layer", "spark_layer_cfg_for_kind", "spark_kv_cache_bytes",
             "spark_stack_kv_bytes", "spark_rope_apply", "spark_kv_append", "spark_attn_prefill",
-            "spark_decode_workspace_bytes", "spark_attn_decode", "spark_attn_decode_static", "spark_check",
+            "spark_decode_workspace_bytes", "spark_attn_decode", "spark_attn_decode_static", "spark_selftest_wait_timeout", "spark_check",
             "spark_last_error",
             "spark_version"]
 
@@ -206,6 +207,11 @@ def spark_attn_decode_static(out, q, gate, k_cache, v_cache, pos, cfg: SparkLaye
     pp = _dev(pos, "pos", torch.int32, 1)
     _raise(_lib().spark_attn_decode_static(po, pq, pg, pkc, pvc, k_cache.shape[2], q.shape[0], pp,
                                            ctypes.byref(cfg), flags, _stream(stream)))
+
+
+def spark_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:
+    """Launch a block whose bounded wait cannot complete; spark_check() then reports a timeout."""
+    _raise(_lib().spark_selftest_wait_timeout(timeout_ns, _stream(stream)))
 
 
 def spark_check(stream=None) -> None:

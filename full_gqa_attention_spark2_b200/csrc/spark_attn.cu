@@ -18,6 +18,23 @@
 #include "ptx.cuh"
 #include "rope_append.cuh"
 
+namespace spark {
+// One block waits, with the library's bounded wait, on a barrier phase that
+// nothing ever completes: the wait must run out, set the device error word and
+// let the kernel return.  Used to test the failure-detection path.
+__global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, timeout_ns, 0x7Fu);
+}
+}  // namespace spark
+
 namespace {
 
 thread_local char g_last_error[512] = "";
@@ -504,6 +521,16 @@ int spark_attn_decode_static(void* out, const void* q, const void* gate, const v
       (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
   e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_combine_kernel launch");
+}
+
+int spark_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull)
+    return fail(SPARK_ERR_INVALID_ARG, "timeout_ns must be in (0, 10 s]");
+  int rc, dev;
+  if ((rc = device_ready(&dev))) return rc;
+  spark::selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(timeout_ns);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "selftest_wait_kernel launch");
 }
 
 int spark_check(void* stream) {

@@ -180,6 +180,13 @@ int spark_attn_decode_static(void* out, const void* q, const void* gate, const v
                              const void* v_cache, int cap, int B, const int* pos,
                              const spark_layer_cfg* cfg, unsigned flags, void* stream);
 
+/* Self-test of the failure-detection path: launches one block that waits,
+ * with the same bounded wait every kernel of the library uses, on a barrier
+ * phase that nothing completes.  The wait runs out after timeout_ns
+ * (0 < timeout_ns <= 10 s), the block returns, and the next spark_check()
+ * reports SPARK_ERR_TIMEOUT.  The GPU context stays usable. */
+int spark_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
+
 /* Synchronise `stream`, then read and clear the library's device error word
  * on the current device.  Returns SPARK_OK, SPARK_ERR_TIMEOUT,
  * SPARK_ERR_DEVICE_ARG or SPARK_ERR_CUDA. */

@@ -52,6 +52,24 @@ print("RESULT " + json.dumps(res))
 
 
 @pytest.mark.gpu
+def test_a_wait_that_nothing_completes_times_out(cuda_device):
+    import time
+    sa.spark_check()
+    t0 = time.perf_counter()
+    sa.spark_selftest_wait_timeout(50_000_000)          # 50 ms
+    with pytest.raises(sa.SparkError) as e:
+        sa.spark_check()
+    assert e.value.status == -4
+    assert 0.04 < time.perf_counter() - t0 < 5.0
+    sa.spark_check()                                     # the word was cleared; the context is usable
+    from tests.test_gpu_kernels import _decode_case
+    from tests.helpers import assert_close
+    from oracle import spark_oracle as O
+    got, ref = _decode_case(O.SLIDING, 2, [700, 700])
+    assert_close(got, ref, "decode after a timed-out wait")
+
+
+@pytest.mark.gpu
 def test_expired_waits_report_timeout_and_return(cuda_device):
     env = dict(os.environ, SPARK_WAIT_TIMEOUT_NS="1")
     r = subprocess.run([sys.executable, "-c", CHILD % ROOT], env=env, capture_output=True, text=True, timeout=300)
