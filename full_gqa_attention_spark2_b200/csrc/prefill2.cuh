@@ -1,0 +1,356 @@
+// Flash-attention prefill on a pair of SMs (tcgen05 cta_group::2, M = 256).
+//
+// A cluster of two blocks computes two query heads of the same KV group over
+// the same 128-query tile, so both need exactly the same K/V tiles and masks.
+// Each UMMA instruction of the pair is issued once, by the even block, with
+// M = 256 rows: rows 0..127 (block 0's head) come from block 0's shared memory
+// and tensor memory, rows 128..255 from block 1's, and the B operand is split
+// in halves between the two blocks.  So each block stages only half of every
+// K tile (64 of its 128 keys) and half of every V tile (128 of its 256 dims):
+// 64 KB of K/V per 128-key tile per SM instead of 128 KB, which doubles the
+// loads in flight that the shared-memory ring can hold and halves the L2->SM
+// traffic.
+//
+// Per block: Q tile 64 KB; ring of 20 slots of 8 KB.  K slot = one 64-dim box of
+// this block's 64 keys; V slot = 32 keys x this block's 128 dims.  TMEM per
+// block as in the single-SM kernel: O [0,256), S buffers [256,384) and
+// [384,512), P (bf16 pairs) over the first 64 columns of its S buffer.
+//
+// Synchronisation of the pair:
+//   - both producers load into their own shared memory; their TMA bytes complete
+//     on the even block's slot barrier, which only the even producer arms;
+//   - the even block's MMA thread commits with a two-block multicast to the
+//     slot-empty, S-ready and O-ready barriers of both blocks;
+//   - both blocks' softmax warps arrive on the even block's P-ready barrier.
+#pragma once
+#include <cuda.h>
+#include "prefill.cuh"
+#include "ptx.cuh"
+
+namespace spark {
+
+constexpr int kP2Slots = 20;
+constexpr int kP2SlotBytes = 8192;
+constexpr int kP2SmemBytes = 1024 + kPfQBytes + kP2Slots * kP2SlotBytes + 1024;
+constexpr uint32_t kIdescQK2 = umma_idesc_bf16(256, 128, false, false);
+constexpr uint32_t kIdescPV2 = umma_idesc_bf16(256, 256, false, true);
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
+    prefill2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kcmap,
+                    const __grid_constant__ CUtensorMap vcmap, const PrefillParams P) {
+  extern __shared__ uint8_t dsmem[];
+  const uint32_t raw = smem_u32(dsmem);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = dsmem + (base - raw);
+  const uint32_t q_s = base;
+  const uint32_t slots = base + kPfQBytes;
+  uint8_t* gmisc = gbase + kPfQBytes + kP2Slots * kP2SlotBytes;
+  const uint32_t misc = smem_u32(gmisc);
+  const uint32_t bar_slot_full = misc;              // [20], even block's are used
+  const uint32_t bar_slot_empty = misc + 160;       // [20], both blocks
+  const uint32_t bar_q = misc + 320;                // even block's is used
+  const uint32_t bar_s = misc + 328;                // [2], both
+  const uint32_t bar_p = misc + 344;                // [2], even block's is used
+  const uint32_t bar_o = misc + 360;                // [2], both
+  const uint32_t bar_done = misc + 376;             // even block's
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gmisc + 384);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gmisc + 388);
+
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  // cluster -> (head pair, query tile (heaviest first), KV head, sequence)
+  int id = blockIdx.x >> 1;
+  const int hp = id & 1;
+  id >>= 1;
+  const int qt = P.n_qt - 1 - (id % P.n_qt);
+  id /= P.n_qt;
+  const int kvh = id & 3;
+  const int b = id >> 2;
+  const int h = kvh * 4 + hp * 2 + (int)rank;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int pos0 = P.pos0[b];
+  const bool bad = pos0 < 0 || pos0 > kMaxPos - P.T || (P.has_cache && !P.sliding && pos0 > P.cap);
+  PfSchedule S = pf_schedule(P, qt, bad ? 0 : pos0);
+  if (bad) {
+    S.n_tiles = 0;
+    if (threadIdx.x == 0 && qt == 0 && h == 0) raise_error(kErrPosition, 0x500u | (unsigned)b);
+  }
+  const int n = S.n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kP2Slots; ++s) {
+      mbar_init(bar_slot_full + 8 * s, 1);
+      mbar_init(bar_slot_empty + 8 * s, 1);
+    }
+    mbar_init(bar_q, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar_s + 8 * x, 1);
+      mbar_init(bar_p + 8 * x, 8);        // 4 softmax warps of each block
+      mbar_init(bar_o + 8 * x, 1);
+    }
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc2(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish2();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (n > 0 && warp == 0) {
+    // ------------------------------------------------------ producers (both)
+    if (lane == 0) {
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      if (P.has_cache) {
+        tma_prefetch_desc(&kcmap);
+        tma_prefetch_desc(&vcmap);
+      }
+      const uint32_t q_full0 = mapa_shared(bar_q, 0);
+      if (leader) mbar_arrive_expect_tx(bar_q, 2 * kPfQBytes);
+      for (int d = 0; d < 4; ++d) tma2_load_4d(q_s + d * 16384, &qmap, q_full0, d * 64, h, qt * kPfM, b);
+      const int plane = b * kNkv + kvh;
+      const int key_half = 64 * (int)rank;       // this block's keys of a K tile
+      const int dim_half = 128 * (int)rank;      // this block's dims of a V tile
+      int li = 0;
+      bool ok = true;
+      for (int step = 0; step <= n && ok; ++step) {
+        for (int part = 0; part < 2 && ok; ++part) {
+          const bool is_k = (part == 0);
+          const int j = is_k ? step : step - 1;
+          if (j < 0 || j >= n) continue;
+          const PfTile t = pf_tile(S, P, j);
+          for (int x = 0; x < 4; ++x) {
+            const int s = li % kP2Slots;
+            if (li >= kP2Slots &&
+                !mbar_wait(bar_slot_empty + 8 * s, ((li / kP2Slots) - 1) & 1, abort_flag, P.timeout_ns, 0x50u)) {
+              ok = false;
+              break;
+            }
+            const uint32_t dst = slots + s * kP2SlotBytes;
+            const uint32_t full0 = mapa_shared(bar_slot_full + 8 * s, 0);
+            if (leader) mbar_arrive_expect_tx(bar_slot_full + 8 * s, 2 * kP2SlotBytes);
+            if (is_k) {        // x = 64-dim box of this block's 64 keys
+              if (t.hist) tma2_load_3d(dst, &kcmap, full0, x * 64, t.row + key_half, plane);
+              else tma2_load_4d(dst, &kmap, full0, x * 64, kvh, t.row + key_half, b);
+            } else {           // x = 32-key sub-tile, this block's two 64-dim boxes
+              for (int d = 0; d < 2; ++d) {
+                const int dim = dim_half + 64 * d;
+                if (t.hist) tma2_load_3d(dst + d * 4096, &vcmap, full0, dim, t.row + 32 * x, plane);
+                else tma2_load_4d(dst + d * 4096, &vmap, full0, dim, kvh, t.row + 32 * x, b);
+              }
+            }
+            ++li;
+          }
+        }
+      }
+      if (leader) {
+        // the even block's barriers count both blocks' bytes: wait for all copies in flight
+        if (mbar_drain(bar_q, 0, 200000000ull)) {
+          for (int i = max(0, li - kP2Slots); i < li; ++i)
+            if (!mbar_drain(bar_slot_full + 8 * (i % kP2Slots), (i / kP2Slots) & 1, 200000000ull)) break;
+        }
+      } else if (!ok) {
+        __nanosleep(200000);   // aborted: let this block's last copies land before the pair leaves
+      }
+    }
+    __syncwarp();
+  } else if (n > 0 && warp == 1) {
+    // --------------------------------------------------- MMA issuer (even block)
+    if (lane == 0 && leader) {
+      const uint64_t dq = smem_desc_sw128(q_s, 16, 1024);
+      bool ok = mbar_wait(bar_q, 0, abort_flag, P.timeout_ns, 0x60u);
+      tc_fence_after();
+      int li = 0;
+      auto issue_s = [&](int j) -> bool {
+        const uint32_t dcol = tmem + kSCol + 128u * (j & 1);
+        for (int d = 0; d < 4; ++d) {
+          const int s = li % kP2Slots;
+          if (!mbar_wait(bar_slot_full + 8 * s, (li / kP2Slots) & 1, abort_flag, P.timeout_ns, 0x61u))
+            return false;
+          tc_fence_after();
+          const uint64_t dk = smem_desc_sw128(slots + s * kP2SlotBytes, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma2_ss(dcol, dq + (uint64_t)((d * 16384 + kk * 32) >> 4), dk + (uint64_t)((kk * 32) >> 4),
+                     kIdescQK2, (d | kk) != 0);
+          umma2_commit_mc(bar_slot_empty + 8 * s, 3);
+          ++li;
+        }
+        umma2_commit_mc(bar_s + 8 * (j & 1), 3);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        if (!mbar_wait_cluster(bar_p + 8 * (j & 1), (j >> 1) & 1, abort_flag, P.timeout_ns, 0x62u)) return false;
+        tc_fence_after();
+        const uint32_t pcol = tmem + kSCol + 128u * (j & 1);
+        for (int v = 0; v < 4; ++v) {
+          const int s = li % kP2Slots;
+          if (!mbar_wait(bar_slot_full + 8 * s, (li / kP2Slots) & 1, abort_flag, P.timeout_ns, 0x63u))
+            return false;
+          tc_fence_after();
+          const uint64_t dv = smem_desc_sw128(slots + s * kP2SlotBytes, 4096, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            umma2_ts(tmem + kOCol, pcol + 16u * v + 8u * kk, dv + (uint64_t)((kk * 2048) >> 4), kIdescPV2,
+                     (j > 0 || v > 0 || kk > 0) ? 1u : 0u);
+          umma2_commit_mc(bar_slot_empty + 8 * s, 3);
+          ++li;
+        }
+        umma2_commit_mc(bar_o + 8 * (j & 1), 3);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < n && ok; ++j) {
+        if (j + 1 < n) ok = issue_s(j + 1);
+        if (ok) ok = issue_pv(j);
+      }
+      umma2_commit_mc(bar_done, 1);
+      mbar_drain(bar_done, 0, 200000000ull);
+    }
+    __syncwarp();
+  } else if (n > 0 && warp >= 4) {
+    // ------------------------------------------------- softmax warps (both)
+    const int r = threadIdx.x - 128;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t ocol = tmem + lane_base + kOCol;
+    const int qp = S.qp0 + r;
+    const bool row_valid = qp < S.pos0 + P.T;
+    const float c_scale = 0.0625f * 1.4426950408889634f;    // 1/sqrt(256) * log2(e)
+    const uint32_t p_ready0 = mapa_shared(bar_p, 0);
+    float m_ref = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      // warp-uniform outcomes: tcgen05.ld / st below need every lane of the warp
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s + 8 * (j & 1), (j >> 1) & 1, abort_flag, P.timeout_ns, 0x70u))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t scol = tmem + lane_base + kSCol + 128u * (j & 1);
+      uint32_t sv[128];
+      tmem_ld32(scol, sv);
+      tmem_ld32(scol + 32, sv + 32);
+      tmem_ld32(scol + 64, sv + 64);
+      tmem_ld32(scol + 96, sv + 96);
+      tmem_wait_ld();
+
+      const PfTile t = pf_tile(S, P, j);
+      const bool full_tile = t.kt0 >= t.v_lo && t.kt0 + kPfN <= t.v_hi && t.kt0 + kPfN - 1 <= S.qp0 &&
+                             (!P.sliding || t.kt0 > S.qp0 + kPfM - 1 - kWindow);
+      float mx = -INFINITY;
+      if (full_tile) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const float x = __uint_as_float(sv[i]) * c_scale;
+          sv[i] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      } else {
+        const int lo = max(t.v_lo, P.sliding ? qp - (kWindow - 1) : t.v_lo) - t.kt0;
+        const int hi = min(t.v_hi - 1, qp) - t.kt0;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const float x = (i >= lo && i <= hi) ? __uint_as_float(sv[i]) * c_scale : -INFINITY;
+          sv[i] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      }
+      float factor = 1.f;
+      const bool resc = mx > m_ref + 8.f;
+      if (resc) {
+        factor = fast_exp2(m_ref - mx);
+        m_ref = mx;
+      }
+      const bool need_o = resc && l_run > 0.f;
+      if (__any_sync(0xffffffffu, need_o)) {
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(bar_o + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, P.timeout_ns, 0x71u))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float f = need_o ? factor : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(ocol + 32 * c, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+          tmem_st32(ocol + 32 * c, ov);
+        }
+        tmem_wait_st();
+      }
+      l_run *= factor;
+      const float mr = (m_ref == -INFINITY) ? 0.f : m_ref;
+      float ls = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = fast_exp2(__uint_as_float(sv[2 * i]) - mr);
+        const float p1 = fast_exp2(__uint_as_float(sv[2 * i + 1]) - mr);
+        ls += p0 + p1;
+        pk[i] = pack_bf16(p0, p1);
+      }
+      l_run += ls;
+      tmem_st32(scol, pk);
+      tmem_st32(scol + 32, pk + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(bar_p + 8 * (j & 1));
+        else mbar_arrive_remote(p_ready0 + 8 * (j & 1));
+      }
+    }
+    if (ok && __all_sync(0xffffffffu,
+                         mbar_wait(bar_o + 8 * ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, P.timeout_ns, 0x72u))) {
+      tc_fence_after();
+      float scale = 0.f;
+      __nv_bfloat16* dst = nullptr;
+      if (row_valid) {
+        const long long tok = (long long)b * P.T + (qp - S.pos0);
+        const float gl = __bfloat162float(P.gate[tok * kNq + h]);
+        scale = (l_run > 0.f ? 1.f / l_run : 0.f) * (1.f / (1.f + expf(-gl)));
+        dst = P.out + (tok * kNq + h) * kHeadDim;
+      }
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(ocol + 32 * c, ov);
+        tmem_wait_ld();
+        if (row_valid) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(ov[8 * e + 0]) * scale, __uint_as_float(ov[8 * e + 1]) * scale);
+            w.y = pack_bf16(__uint_as_float(ov[8 * e + 2]) * scale, __uint_as_float(ov[8 * e + 3]) * scale);
+            w.z = pack_bf16(__uint_as_float(ov[8 * e + 4]) * scale, __uint_as_float(ov[8 * e + 5]) * scale);
+            w.w = pack_bf16(__uint_as_float(ov[8 * e + 6]) * scale, __uint_as_float(ov[8 * e + 7]) * scale);
+            d4[e] = w;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  }
+
+  // both blocks: no TMEM, shared memory or barrier of either block is in use past this point
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem, kTmemCols);
+  }
+}
+
+}  // namespace spark

@@ -15,6 +15,7 @@
 #include "../../include/spark_attn.h"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "prefill2.cuh"
 #include "ptx.cuh"
 #include "rope_append.cuh"
 
@@ -81,9 +82,9 @@ int device_ready(int* dev_out) {
     cudaError_t a = cudaFuncSetAttribute(spark::decode_partial_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          spark::kDecSmemBytes);
-    cudaError_t b = cudaFuncSetAttribute(spark::prefill_kernel,
+    cudaError_t b = cudaFuncSetAttribute(spark::prefill2_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         spark::kPfSmemBytes);
+                                         spark::kP2SmemBytes);
     if (a != cudaSuccess || b != cudaSuccess) {
       snprintf(d.why, sizeof(d.why), "cudaFuncSetAttribute: %s",
                cudaGetErrorString(a != cudaSuccess ? a : b));
@@ -424,14 +425,14 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
     if ((rc = make_map(&qm, q, 4, dq, sq, bq))) return rc;
     const cuuint64_t dk[4] = {256, 4, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t sk[3] = {512, 512ull * 4, 512ull * 4 * T};
-    const cuuint32_t bk[4] = {64, 1, (cuuint32_t)spark::kPfN, 1};
+    const cuuint32_t bk[4] = {64, 1, (cuuint32_t)(spark::kPfN / 2), 1};   // each block of the pair: 64 keys
     const cuuint32_t bv[4] = {64, 1, 32, 1};
     if ((rc = make_map(&km, k, 4, dk, sk, bk))) return rc;
     if ((rc = make_map(&vm, v, 4, dk, sk, bv))) return rc;
     if (k_cache) {
       const cuuint64_t dc[3] = {256, (cuuint64_t)cap, (cuuint64_t)B * 4};
       const cuuint64_t sc[2] = {512, (cuuint64_t)cap * 512};
-      const cuuint32_t bkc[3] = {64, (cuuint32_t)spark::kPfN, 1};
+      const cuuint32_t bkc[3] = {64, (cuuint32_t)(spark::kPfN / 2), 1};
       const cuuint32_t bvc[3] = {64, 32, 1};
       if ((rc = make_map(&kcm, k_cache, 3, dc, sc, bkc))) return rc;
       if ((rc = make_map(&vcm, v_cache, 3, dc, sc, bvc))) return rc;
@@ -453,10 +454,11 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   P.timeout_ns = wait_timeout_ns();
   const long long blocks = (long long)B * spark::kNq * P.n_qt;
   if (blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");
-  spark::prefill_kernel<<<(unsigned)blocks, spark::kPfThreads, spark::kPfSmemBytes, (cudaStream_t)stream>>>(
+  // clusters of two blocks (an SM pair): two query heads of a KV group, same query tile
+  spark::prefill2_kernel<<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
       qm, km, vm, kcm, vcm, P);
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "prefill_kernel launch");
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "prefill2_kernel launch");
 }
 
 int spark_attn_decode_static(void* out, const void* q, const void* gate, const void* k_cache,
