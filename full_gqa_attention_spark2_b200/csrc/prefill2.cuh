@@ -11,8 +11,11 @@
 // loads in flight that the shared-memory ring can hold and halves the L2->SM
 // traffic.
 //
-// Per block: Q tile 64 KB; ring of 20 slots of 8 KB.  K slot = one 64-dim box of
-// this block's 64 keys; V slot = 32 keys x this block's 128 dims.  TMEM per
+// Per block: Q tile 64 KB; ring of 5 slots of 32 KB.  A K slot holds this
+// block's 64 keys of a K tile (four 64-dim boxes); a V slot holds this block's
+// 128 dims of a V tile (four 32-key sub-tiles of two 64-dim boxes).  One
+// barrier wait per slot keeps the single MMA-issuing thread ahead of the
+// tensor core.  TMEM per
 // block as in the single-SM kernel: O [0,256), S buffers [256,384) and
 // [384,512), P (bf16 pairs) over the first 64 columns of its S buffer.
 //
@@ -29,8 +32,8 @@
 
 namespace spark {
 
-constexpr int kP2Slots = 20;
-constexpr int kP2SlotBytes = 8192;
+constexpr int kP2Slots = 5;
+constexpr int kP2SlotBytes = 32768;
 constexpr int kP2SmemBytes = 1024 + kPfQBytes + kP2Slots * kP2SlotBytes + 1024;
 constexpr uint32_t kIdescQK2 = umma_idesc_bf16(256, 128, false, false);
 constexpr uint32_t kIdescPV2 = umma_idesc_bf16(256, 256, false, true);
@@ -47,15 +50,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   const uint32_t slots = base + kPfQBytes;
   uint8_t* gmisc = gbase + kPfQBytes + kP2Slots * kP2SlotBytes;
   const uint32_t misc = smem_u32(gmisc);
-  const uint32_t bar_slot_full = misc;              // [20], even block's are used
-  const uint32_t bar_slot_empty = misc + 160;       // [20], both blocks
-  const uint32_t bar_q = misc + 320;                // even block's is used
-  const uint32_t bar_s = misc + 328;                // [2], both
-  const uint32_t bar_p = misc + 344;                // [2], even block's is used
-  const uint32_t bar_o = misc + 360;                // [2], both
-  const uint32_t bar_done = misc + 376;             // even block's
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gmisc + 384);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gmisc + 388);
+  const uint32_t bar_slot_full = misc;              // [5], even block's are used
+  const uint32_t bar_slot_empty = misc + 40;        // [5], both blocks
+  const uint32_t bar_q = misc + 80;                 // even block's is used
+  const uint32_t bar_s = misc + 88;                 // [2], both
+  const uint32_t bar_p = misc + 104;                // [2], even block's is used
+  const uint32_t bar_o = misc + 120;                // [2], both
+  const uint32_t bar_done = misc + 136;             // even block's
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gmisc + 144);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gmisc + 148);
 
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -127,28 +130,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
           const int j = is_k ? step : step - 1;
           if (j < 0 || j >= n) continue;
           const PfTile t = pf_tile(S, P, j);
-          for (int x = 0; x < 4; ++x) {
-            const int s = li % kP2Slots;
-            if (li >= kP2Slots &&
-                !mbar_wait(bar_slot_empty + 8 * s, ((li / kP2Slots) - 1) & 1, abort_flag, P.timeout_ns, 0x50u)) {
-              ok = false;
-              break;
+          const int s = li % kP2Slots;
+          if (li >= kP2Slots &&
+              !mbar_wait(bar_slot_empty + 8 * s, ((li / kP2Slots) - 1) & 1, abort_flag, P.timeout_ns, 0x50u)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = slots + s * kP2SlotBytes;
+          const uint32_t full0 = mapa_shared(bar_slot_full + 8 * s, 0);
+          if (leader) mbar_arrive_expect_tx(bar_slot_full + 8 * s, 2 * kP2SlotBytes);
+          if (is_k) {          // four 64-dim boxes of this block's 64 keys, 8 KB each
+            for (int x = 0; x < 4; ++x) {
+              if (t.hist) tma2_load_3d(dst + x * 8192, &kcmap, full0, x * 64, t.row + key_half, plane);
+              else tma2_load_4d(dst + x * 8192, &kmap, full0, x * 64, kvh, t.row + key_half, b);
             }
-            const uint32_t dst = slots + s * kP2SlotBytes;
-            const uint32_t full0 = mapa_shared(bar_slot_full + 8 * s, 0);
-            if (leader) mbar_arrive_expect_tx(bar_slot_full + 8 * s, 2 * kP2SlotBytes);
-            if (is_k) {        // x = 64-dim box of this block's 64 keys
-              if (t.hist) tma2_load_3d(dst, &kcmap, full0, x * 64, t.row + key_half, plane);
-              else tma2_load_4d(dst, &kmap, full0, x * 64, kvh, t.row + key_half, b);
-            } else {           // x = 32-key sub-tile, this block's two 64-dim boxes
+          } else {             // four 32-key sub-tiles x this block's two 64-dim boxes, 4 KB each
+            for (int x = 0; x < 4; ++x)
               for (int d = 0; d < 2; ++d) {
                 const int dim = dim_half + 64 * d;
-                if (t.hist) tma2_load_3d(dst + d * 4096, &vcmap, full0, dim, t.row + 32 * x, plane);
-                else tma2_load_4d(dst + d * 4096, &vmap, full0, dim, kvh, t.row + 32 * x, b);
+                const uint32_t o = dst + x * 8192 + d * 4096;
+                if (t.hist) tma2_load_3d(o, &vcmap, full0, dim, t.row + 32 * x, plane);
+                else tma2_load_4d(o, &vmap, full0, dim, kvh, t.row + 32 * x, b);
               }
-            }
-            ++li;
           }
+          ++li;
         }
       }
       if (leader) {
@@ -171,40 +176,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       int li = 0;
       auto issue_s = [&](int j) -> bool {
         const uint32_t dcol = tmem + kSCol + 128u * (j & 1);
-        for (int d = 0; d < 4; ++d) {
-          const int s = li % kP2Slots;
-          if (!mbar_wait(bar_slot_full + 8 * s, (li / kP2Slots) & 1, abort_flag, P.timeout_ns, 0x61u))
-            return false;
-          tc_fence_after();
-          const uint64_t dk = smem_desc_sw128(slots + s * kP2SlotBytes, 16, 1024);
+        const int s = li % kP2Slots;
+        if (!mbar_wait(bar_slot_full + 8 * s, (li / kP2Slots) & 1, abort_flag, P.timeout_ns, 0x61u)) return false;
+        tc_fence_after();
+        const uint64_t dk = smem_desc_sw128(slots + s * kP2SlotBytes, 16, 1024);
+#pragma unroll
+        for (int d = 0; d < 4; ++d)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma2_ss(dcol, dq + (uint64_t)((d * 16384 + kk * 32) >> 4), dk + (uint64_t)((kk * 32) >> 4),
+            umma2_ss(dcol, dq + (uint64_t)((d * 16384 + kk * 32) >> 4), dk + (uint64_t)((d * 8192 + kk * 32) >> 4),
                      kIdescQK2, (d | kk) != 0);
-          umma2_commit_mc(bar_slot_empty + 8 * s, 3);
-          ++li;
-        }
+        umma2_commit_mc(bar_slot_empty + 8 * s, 3);
         umma2_commit_mc(bar_s + 8 * (j & 1), 3);
+        ++li;
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
         if (!mbar_wait_cluster(bar_p + 8 * (j & 1), (j >> 1) & 1, abort_flag, P.timeout_ns, 0x62u)) return false;
+        const int s = li % kP2Slots;
+        if (!mbar_wait(bar_slot_full + 8 * s, (li / kP2Slots) & 1, abort_flag, P.timeout_ns, 0x63u)) return false;
         tc_fence_after();
         const uint32_t pcol = tmem + kSCol + 128u * (j & 1);
-        for (int v = 0; v < 4; ++v) {
-          const int s = li % kP2Slots;
-          if (!mbar_wait(bar_slot_full + 8 * s, (li / kP2Slots) & 1, abort_flag, P.timeout_ns, 0x63u))
-            return false;
-          tc_fence_after();
-          const uint64_t dv = smem_desc_sw128(slots + s * kP2SlotBytes, 4096, 1024);
+        const uint64_t dv = smem_desc_sw128(slots + s * kP2SlotBytes, 4096, 1024);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            umma2_ts(tmem + kOCol, pcol + 16u * v + 8u * kk, dv + (uint64_t)((kk * 2048) >> 4), kIdescPV2,
+            umma2_ts(tmem + kOCol, pcol + 16u * v + 8u * kk, dv + (uint64_t)((v * 8192 + kk * 2048) >> 4), kIdescPV2,
                      (j > 0 || v > 0 || kk > 0) ? 1u : 0u);
-          umma2_commit_mc(bar_slot_empty + 8 * s, 3);
-          ++li;
-        }
+        umma2_commit_mc(bar_slot_empty + 8 * s, 3);
         umma2_commit_mc(bar_o + 8 * (j & 1), 3);
+        ++li;
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -245,24 +247,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       const PfTile t = pf_tile(S, P, j);
       const bool full_tile = t.kt0 >= t.v_lo && t.kt0 + kPfN <= t.v_hi && t.kt0 + kPfN - 1 <= S.qp0 &&
                              (!P.sliding || t.kt0 > S.qp0 + kPfM - 1 - kWindow);
-      float mx = -INFINITY;
+      // row max over the raw scores in four independent chains (scale applied after: c_scale > 0)
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (full_tile) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const float x = __uint_as_float(sv[i]) * c_scale;
-          sv[i] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
+        for (int i = 0; i < 128; ++i) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(sv[i]));
       } else {
         const int lo = max(t.v_lo, P.sliding ? qp - (kWindow - 1) : t.v_lo) - t.kt0;
         const int hi = min(t.v_hi - 1, qp) - t.kt0;
 #pragma unroll
         for (int i = 0; i < 128; ++i) {
-          const float x = (i >= lo && i <= hi) ? __uint_as_float(sv[i]) * c_scale : -INFINITY;
+          const float x = (i >= lo && i <= hi) ? __uint_as_float(sv[i]) : -INFINITY;
           sv[i] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+          m4[i & 3] = fmaxf(m4[i & 3], x);
         }
       }
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c_scale;
       float factor = 1.f;
       const bool resc = mx > m_ref + 8.f;
       if (resc) {
@@ -290,17 +290,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         tmem_wait_st();
       }
       l_run *= factor;
-      const float mr = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float ls = 0.f;
+      const float nmr = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        const float p0 = fast_exp2(__uint_as_float(sv[2 * i]) - mr);
-        const float p1 = fast_exp2(__uint_as_float(sv[2 * i + 1]) - mr);
-        ls += p0 + p1;
+        const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * i]), c_scale, nmr));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * i + 1]), c_scale, nmr));
+        l4[i & 3] += p0 + p1;
         pk[i] = pack_bf16(p0, p1);
       }
-      l_run += ls;
+      l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       tmem_st32(scol, pk);
       tmem_st32(scol + 32, pk + 32);
       tmem_wait_st();
