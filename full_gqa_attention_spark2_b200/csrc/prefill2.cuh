@@ -41,7 +41,8 @@ constexpr uint32_t kIdescPV2 = umma_idesc_bf16(256, 256, false, true);
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     prefill2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kcmap,
-                    const __grid_constant__ CUtensorMap vcmap, const PrefillParams P) {
+                    const __grid_constant__ CUtensorMap vcmap, const __grid_constant__ CUtensorMap omap,
+                    const PrefillParams P) {
   extern __shared__ uint8_t dsmem[];
   const uint32_t raw = smem_u32(dsmem);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -311,35 +312,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         else mbar_arrive_remote(p_ready0 + 8 * (j & 1));
       }
     }
-    if (ok && __all_sync(0xffffffffu,
-                         mbar_wait(bar_o + 8 * ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, P.timeout_ns, 0x72u))) {
+    const bool ep_ok = ok && __all_sync(0xffffffffu, mbar_wait(bar_o + 8 * ((n - 1) & 1), ((n - 1) >> 1) & 1,
+                                                               abort_flag, P.timeout_ns, 0x72u));
+    if (ep_ok) {
       tc_fence_after();
+      // out = O / l * sigmoid(gate) in bf16, staged in the Q buffer (free: every S
+      // MMA has completed) in the 128-byte swizzled layout of four [128 x 64] boxes,
+      // then written with TMA tensor stores (rows past the chunk are clipped)
       float scale = 0.f;
-      __nv_bfloat16* dst = nullptr;
       if (row_valid) {
         const long long tok = (long long)b * P.T + (qp - S.pos0);
         const float gl = __bfloat162float(P.gate[tok * kNq + h]);
         scale = (l_run > 0.f ? 1.f / l_run : 0.f) * (1.f / (1.f + expf(-gl)));
-        dst = P.out + (tok * kNq + h) * kHeadDim;
       }
+      uint8_t* q_gen = gbase;                     // generic view of the Q buffer
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         uint32_t ov[32];
         tmem_ld32(ocol + 32 * c, ov);
         tmem_wait_ld();
-        if (row_valid) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+        uint8_t* box = q_gen + (c >> 1) * 16384 + r * 128;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(ov[8 * e + 0]) * scale, __uint_as_float(ov[8 * e + 1]) * scale);
-            w.y = pack_bf16(__uint_as_float(ov[8 * e + 2]) * scale, __uint_as_float(ov[8 * e + 3]) * scale);
-            w.z = pack_bf16(__uint_as_float(ov[8 * e + 4]) * scale, __uint_as_float(ov[8 * e + 5]) * scale);
-            w.w = pack_bf16(__uint_as_float(ov[8 * e + 6]) * scale, __uint_as_float(ov[8 * e + 7]) * scale);
-            d4[e] = w;
-          }
+        for (int e = 0; e < 4; ++e) {
+          uint4 w;
+          w.x = pack_bf16(__uint_as_float(ov[8 * e + 0]) * scale, __uint_as_float(ov[8 * e + 1]) * scale);
+          w.y = pack_bf16(__uint_as_float(ov[8 * e + 2]) * scale, __uint_as_float(ov[8 * e + 3]) * scale);
+          w.z = pack_bf16(__uint_as_float(ov[8 * e + 4]) * scale, __uint_as_float(ov[8 * e + 5]) * scale);
+          w.w = pack_bf16(__uint_as_float(ov[8 * e + 6]) * scale, __uint_as_float(ov[8 * e + 7]) * scale);
+          const int chunk = (c & 1) * 4 + e;      // 16-byte chunk within the 128-byte row of the box
+          *reinterpret_cast<uint4*>(box + ((chunk ^ (r & 7)) << 4)) = w;
         }
       }
+      fence_proxy_async_smem();                   // make the generic writes visible to TMA
+    }
+    // every softmax thread reaches this barrier, aborted or not; store only if all staged their row
+    uint32_t all_ok;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(all_ok)
+        : "r"((uint32_t)ep_ok)
+        : "memory");
+    if (all_ok && threadIdx.x == 128) {
+      for (int d = 0; d < 4; ++d) tma_store_4d(&omap, q_s + d * 16384, d * 64, h, qt * kPfM, b);
+      bulk_commit_group();
+      bulk_wait_group0();
     }
     __syncwarp();
   }

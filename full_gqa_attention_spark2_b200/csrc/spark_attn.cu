@@ -417,12 +417,13 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
 
   // Q, chunk K/V: [B][T][H][256] as 4-D (dim, head, token, batch); caches
   // [B][4][cap][256] as 3-D (dim, row, batch*head).  128-byte swizzled boxes of 64 dims.
-  CUtensorMap qm, km, vm, kcm, vcm;
+  CUtensorMap qm, km, vm, kcm, vcm, om;
   {
     const cuuint64_t dq[4] = {256, 16, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t sq[3] = {512, 512ull * 16, 512ull * 16 * T};
     const cuuint32_t bq[4] = {64, 1, (cuuint32_t)spark::kPfM, 1};
     if ((rc = make_map(&qm, q, 4, dq, sq, bq))) return rc;
+    if ((rc = make_map(&om, out, 4, dq, sq, bq))) return rc;    // the output has q's layout
     const cuuint64_t dk[4] = {256, 4, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t sk[3] = {512, 512ull * 4, 512ull * 4 * T};
     const cuuint32_t bk[4] = {64, 1, (cuuint32_t)(spark::kPfN / 2), 1};   // each block of the pair: 64 keys
@@ -456,7 +457,7 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   if (blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");
   // clusters of two blocks (an SM pair): two query heads of a KV group, same query tile
   spark::prefill2_kernel<<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
-      qm, km, vm, kcm, vcm, P);
+      qm, km, vm, kcm, vcm, om, P);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "prefill2_kernel launch");
 }
