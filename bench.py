@@ -191,7 +191,22 @@ def prefill_step(sa, W, pos0, events=None):
         sa.spark_kv_append(w["kc"], w["vc"], w["k"], w["v"], pos0, w["cfg"])
 
 
+def max_over_ranks(torch, dist, ms: float, device: str = "cuda") -> float:
+    """The slowest rank's time: every rank reports its own device-timed milliseconds."""
+    if dist is None:
+        return ms
+    x = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(x, op=dist.ReduceOp.MAX)
+    return float(x.item())
+
+
+def weak_scaling_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank processed its own units in at most `ms`."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 def timed_region(torch, dist, fn, steps):
+    """Time `steps` calls of fn on the device, bracketed by a barrier and a synchronize; max over ranks."""
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -204,12 +219,7 @@ def timed_region(torch, dist, fn, steps):
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    ms = t0.elapsed_time(t1)
-    if dist is not None:
-        x = torch.tensor([ms], device="cuda")
-        dist.all_reduce(x, op=dist.ReduceOp.MAX)
-        ms = float(x.item())
-    return ms
+    return max_over_ranks(torch, dist, t0.elapsed_time(t1))
 
 
 def run_prefill(torch, sa, synth, dist, args, peaks, world):
@@ -260,7 +270,7 @@ def run_prefill(torch, sa, synth, dist, args, peaks, world):
     torch.cuda.empty_cache()
     return {
         "metric": "prefill attn tok/s & TFLOP/s; decode KV-read GB/s (36-layer stack); % roofline",
-        "value": tokens / (ms_step * 1e-3),
+        "value": weak_scaling_rate(B * T, world, ms_step),
         "unit": "tok/s",
         "ms_per_step": ms_step,
         "tflops": (f_full + f_slide) * world / (ms_step * 1e-3) / 1e12,
@@ -362,6 +372,82 @@ def run_decode(torch, sa, synth, dist, args, peaks, world):
     }
 
 
+def run_long_prefill(torch, sa, synth, dist, args, peaks, world):
+    """B=1, T=131072 in 16 chunks of 8192 over the growing cache, one full and one sliding layer."""
+    dev = torch.device("cuda")
+    T, C, seed = 131072, 8192, 4
+    L = {}
+    for kind, layer in ((SLIDING, 0), (FULL, 3)):
+        cfg = sa.spark_layer_cfg_for_kind(kind)
+        q = torch.empty(1, T, HQ, D, dtype=torch.bfloat16, device=dev)
+        k = torch.empty(1, T, HKV, D, dtype=torch.bfloat16, device=dev)
+        v = torch.empty_like(k)
+        g = torch.empty(1, T, HQ, dtype=torch.bfloat16, device=dev)
+        synth.fill_tokens(q, seed, synth.tensor_id(layer, synth.ROLE_Q), 0)
+        synth.fill_tokens(k, seed, synth.tensor_id(layer, synth.ROLE_K), 0)
+        synth.fill_tokens(v, seed, synth.tensor_id(layer, synth.ROLE_V), 0)
+        synth.fill_tokens(g, seed, synth.tensor_id(layer, synth.ROLE_GATE), 0)
+        cap = WINDOW if kind == SLIDING else T
+        kc = torch.empty(1, HKV, cap, D, dtype=torch.bfloat16, device=dev)
+        L[kind] = dict(cfg=cfg, q=q, k=k, v=v, g=g, out=torch.empty_like(q), kc=kc, vc=torch.empty_like(kc))
+    pos = [torch.full((1,), c * C, dtype=torch.int32, device=dev) for c in range(T // C)]
+
+    def step(i=0):
+        for kind in (SLIDING, FULL):
+            w = L[kind]
+            for c in range(T // C):
+                sl = slice(c * C, (c + 1) * C)
+                q, k = w["q"][:, sl], w["k"][:, sl]
+                sa.spark_rope_apply(q, pos[c], w["cfg"])
+                sa.spark_rope_apply(k, pos[c], w["cfg"])
+                sa.spark_attn_prefill(w["out"][:, sl], q, k, w["v"][:, sl], w["g"][:, sl],
+                                      w["kc"] if c else None, w["vc"] if c else None, pos[c], w["cfg"])
+                sa.spark_kv_append(w["kc"], w["vc"], k, w["v"][:, sl], pos[c], w["cfg"])
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        step()
+    sa.spark_check()
+    steps = max(2, min(args.steps, 5))
+    ms = timed_region(torch, dist, step, steps) / steps
+    sa.spark_check()
+    f_full = sum(prefill_flops(1, C, c * C, FULL, True) for c in range(T // C))
+    f_slide = sum(prefill_flops(1, C, c * C, SLIDING, True) for c in range(T // C))
+    del L
+    torch.cuda.empty_cache()
+    return {"workload": "long_prefill_b1_t131072_chunks8192_sliding+full", "value": T * world / (ms * 1e-3),
+            "unit": "tok/s", "ms_per_step": ms, "tflops": (f_full + f_slide) * world / (ms * 1e-3) / 1e12,
+            "gpu_launches_per_step": 2 * (T // C) * 4}
+
+
+def run_long_decode(torch, sa, synth, dist, args, peaks, world):
+    """One 36-layer decode step at long context: B=1 at 2^20 and B=16 at 131072 (positions at the end)."""
+    dev = torch.device("cuda")
+    out = {}
+    for B, ctx in ((1, 1 << 20), (16, 131072)):
+        p = ctx - 1
+        layers = decode_layers(torch, sa, synth, dev, B, p, seed=5)
+        pos = torch.full((B,), p, dtype=torch.int32, device=dev)
+        ws = torch.empty(max(sa.spark_decode_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers),
+                         dtype=torch.uint8, device=dev)
+        graph = torch.cuda.CUDAGraph()
+        decode_step(sa, layers, pos, ws)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            decode_step(sa, layers, pos, ws)
+        for _ in range(3):
+            graph.replay()
+        steps = max(5, min(args.steps, 20))
+        ms = timed_region(torch, dist, lambda i: graph.replay(), steps) / steps
+        sa.spark_check()
+        total = sum(decode_kv_bytes(B, p, L["kind"]) for L in layers)
+        out[f"b{B}_ctx{ctx}"] = {"value": total * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+                                 "steps_per_s": 1e3 / ms, "kv_bytes_per_step": total,
+                                 "frac_of_hbm": total / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        del graph, layers, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------- oracle timing -------
 
 def oracle_prefill_rate(budget_s: float = 15.0):
@@ -460,6 +546,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-long", action="store_true", help="skip the long-context prefill and decode workloads")
     ap.add_argument("--profile", choices=["prefill_full", "prefill_sliding", "decode_full"], default=None,
                     help="run a small case of one kernel for ncu and exit")
     args = ap.parse_args()
@@ -489,6 +576,8 @@ def main():
 
     res = run_prefill(torch, sa, synth, dist, args, peaks, world)
     dec = None if args.no_decode else run_decode(torch, sa, synth, dist, args, peaks, world)
+    long_pf = None if args.no_long else run_long_prefill(torch, sa, synth, dist, args, peaks, world)
+    long_dec = None if (args.no_long or args.no_decode) else run_long_decode(torch, sa, synth, dist, args, peaks, world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, threads, sample = oracle_prefill_rate()
@@ -511,7 +600,7 @@ def main():
         "tflops": res["tflops"], "prefill_full_kernel": res["prefill_full_kernel"],
         "roofline": res["roofline"], "e2e": res["e2e"], "clocks": res["clocks"],
         "gpu_launches": res["gpu_launches"] + (0 if dec is None else 0),
-        "cpu_baseline": cpu, "decode": dec,
+        "cpu_baseline": cpu, "decode": dec, "long_prefill": long_pf, "long_decode": long_dec,
     }
     print(json.dumps(line), flush=True)
 
