@@ -33,6 +33,8 @@ struct PrefillParams {
   const __nv_bfloat16* gate;     // [B][T][16]
   const int* pos0;               // [B]
   int B, T, cap, sliding, has_cache, n_qt;
+  int rope, rot;                 // rope: q is raw and is rotated in shared memory
+  double log2_theta;
   unsigned long long timeout_ns;
 };
 

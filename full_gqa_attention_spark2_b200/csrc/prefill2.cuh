@@ -53,13 +53,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   const uint32_t misc = smem_u32(gmisc);
   const uint32_t bar_slot_full = misc;              // [5], even block's are used
   const uint32_t bar_slot_empty = misc + 40;        // [5], both blocks
-  const uint32_t bar_q = misc + 80;                 // even block's is used
+  const uint32_t bar_q = misc + 80;                 // this block's Q landed (each block's own)
   const uint32_t bar_s = misc + 88;                 // [2], both
   const uint32_t bar_p = misc + 104;                // [2], even block's is used
   const uint32_t bar_o = misc + 120;                // [2], both
   const uint32_t bar_done = misc + 136;             // even block's
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gmisc + 144);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gmisc + 148);
+  const uint32_t bar_q_ready = misc + 144;          // both blocks' Q rotated / checked (even block's)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gmisc + 160);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gmisc + 164);
 
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -95,6 +96,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       mbar_init(bar_o + 8 * x, 1);
     }
     mbar_init(bar_done, 1);
+    mbar_init(bar_q_ready, 8);          // 4 softmax warps of each block
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -117,9 +119,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         tma_prefetch_desc(&kcmap);
         tma_prefetch_desc(&vcmap);
       }
-      const uint32_t q_full0 = mapa_shared(bar_q, 0);
-      if (leader) mbar_arrive_expect_tx(bar_q, 2 * kPfQBytes);
-      for (int d = 0; d < 4; ++d) tma2_load_4d(q_s + d * 16384, &qmap, q_full0, d * 64, h, qt * kPfM, b);
+      // Q lands on this block's own barrier: its softmax warps rotate it (RoPE at load) or
+      // just see it arrive, then tell the even block's MMA thread
+      mbar_arrive_expect_tx(bar_q, kPfQBytes);
+      for (int d = 0; d < 4; ++d) tma_load_4d(q_s + d * 16384, &qmap, bar_q, d * 64, h, qt * kPfM, b);
       const int plane = b * kNkv + kvh;
       const int key_half = 64 * (int)rank;       // this block's keys of a K tile
       const int dim_half = 128 * (int)rank;      // this block's dims of a V tile
@@ -157,9 +160,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
           ++li;
         }
       }
+      const bool q_landed = mbar_drain(bar_q, 0, 200000000ull);
       if (leader) {
-        // the even block's barriers count both blocks' bytes: wait for all copies in flight
-        if (mbar_drain(bar_q, 0, 200000000ull)) {
+        // the even block's slot barriers count both blocks' bytes: wait for all copies in flight
+        if (q_landed) {
           for (int i = max(0, li - kP2Slots); i < li; ++i)
             if (!mbar_drain(bar_slot_full + 8 * (i % kP2Slots), (i / kP2Slots) & 1, 200000000ull)) break;
         }
@@ -172,7 +176,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     // --------------------------------------------------- MMA issuer (even block)
     if (lane == 0 && leader) {
       const uint64_t dq = smem_desc_sw128(q_s, 16, 1024);
-      bool ok = mbar_wait(bar_q, 0, abort_flag, P.timeout_ns, 0x60u);
+      bool ok = mbar_wait_cluster(bar_q_ready, 0, abort_flag, P.timeout_ns, 0x60u);
       tc_fence_after();
       int li = 0;
       auto issue_s = [&](int j) -> bool {
@@ -228,9 +232,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     const bool row_valid = qp < S.pos0 + P.T;
     const float c_scale = 0.0625f * 1.4426950408889634f;    // 1/sqrt(256) * log2(e)
     const uint32_t p_ready0 = mapa_shared(bar_p, 0);
-    float m_ref = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
+    {
+      // Q: wait for this block's tile, rotate it in place when q is raw, hand it to the MMA
+      // thread.  Thread t rotates pairs (2 pp, 2 pp + 1) over a group of consecutive rows; the
+      // angle of the group's first row is exact (fp64 reduction), the next rows advance by
+      // the rotation by f_i (complex multiplication).
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort_flag, P.timeout_ns, 0x73u));
+      if (ok && P.rope) {
+        const int tq = threadIdx.x - 128;
+        const int half = P.rot >> 1;
+        const int n_pp = half >> 1;                       // pair-pairs: 64 (sliding) or 16 (full)
+        const int pp = tq % n_pp;
+        const int rows_per = 128 / (128 / n_pp);          // rows per thread: n_pp
+        const int r0 = (tq / n_pp) * rows_per;
+        float c[2], sn[2], cf[2], sf[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = 2 * pp + e;
+          const double f = exp2(-(2.0 * i / P.rot) * P.log2_theta);
+          rope_angle(S.qp0 + r0, f, c[e], sn[e]);
+          rope_angle(1, f, cf[e], sf[e]);
+        }
+        const int dlo = 2 * pp, dhi = 2 * pp + half;
+        uint8_t* qg = gbase;
+        for (int rr = 0; rr < rows_per; ++rr) {
+          const int row = r0 + rr;
+          uint32_t* plo = reinterpret_cast<uint32_t*>(qg + (dlo >> 6) * 16384 + row * 128 +
+                                                      (((((dlo & 63) >> 3) ^ (row & 7))) << 4) + (dlo & 7) * 2);
+          uint32_t* phi = reinterpret_cast<uint32_t*>(qg + (dhi >> 6) * 16384 + row * 128 +
+                                                      (((((dhi & 63) >> 3) ^ (row & 7))) << 4) + (dhi & 7) * 2);
+          const uint32_t lo = *plo, hi = *phi;
+          const float l0 = bf16_lo(lo), l1 = bf16_hi(lo), h0 = bf16_lo(hi), h1 = bf16_hi(hi);
+          *plo = pack_bf16(l0 * c[0] - h0 * sn[0], l1 * c[1] - h1 * sn[1]);
+          *phi = pack_bf16(h0 * c[0] + l0 * sn[0], h1 * c[1] + l1 * sn[1]);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float cn = c[e] * cf[e] - sn[e] * sf[e];
+            sn[e] = sn[e] * cf[e] + c[e] * sf[e];
+            c[e] = cn;
+          }
+        }
+        fence_proxy_async_smem();                         // the tensor core reads Q next
+      }
+      __syncwarp();
+      if (lane == 0 && ok) {
+        if (leader) mbar_arrive(bar_q_ready);
+        else mbar_arrive_remote_cluster(mapa_shared(bar_q_ready, 0));
+      }
+    }
+    float m_ref = -INFINITY, l_run = 0.f;
+    for (int j = 0; j < n && ok; ++j) {
       // warp-uniform outcomes: tcgen05.ld / st below need every lane of the warp
       if (!__all_sync(0xffffffffu, mbar_wait(bar_s + 8 * (j & 1), (j >> 1) & 1, abort_flag, P.timeout_ns, 0x70u))) {
         ok = false;

@@ -412,8 +412,6 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
     return fail(SPARK_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   int dev;
   if ((rc = device_ready(&dev))) return rc;
-  if (flags & SPARK_ROPE_FUSED)
-    return fail(SPARK_ERR_UNSUPPORTED, "prefill takes rotated q; run spark_rope_apply first");
 
   // Q, chunk K/V: [B][T][H][256] as 4-D (dim, head, token, batch); caches
   // [B][4][cap][256] as 3-D (dim, row, batch*head).  128-byte swizzled boxes of 64 dims.
@@ -452,6 +450,9 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   P.sliding = sliding;
   P.has_cache = k_cache ? 1 : 0;
   P.n_qt = (T + spark::kPfM - 1) / spark::kPfM;
+  P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
+  P.rot = cfg->rot_dim;
+  P.log2_theta = log2(cfg->theta);
   P.timeout_ns = wait_timeout_ns();
   const long long blocks = (long long)B * spark::kNq * P.n_qt;
   if (blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");

@@ -119,8 +119,10 @@ int spark_kv_append(void* k_cache, void* v_cache, int cap, const void* k, const 
                     void* stream);
 
 /* Attention of a chunk of T queries per sequence (prefill).
- *   q [B][T][16][256] (rotated, or raw with SPARK_ROPE_FUSED), k [B][T][4][256]
- *   rotated, v [B][T][4][256], gate [B][T][16]; out [B][T][16][256].
+ *   q [B][T][16][256] (rotated, or raw with SPARK_ROPE_FUSED: the kernel then
+ *   rotates each Q tile in shared memory after loading it; q itself is not
+ *   modified), k [B][T][4][256] rotated, v [B][T][4][256], gate [B][T][16];
+ *   out [B][T][16][256].
  *   Token t of sequence b is at position pos0[b] + t (pos0: device int32 [B]).
  *   The chunk's own keys come from k/v.  Earlier keys (the history,
  *   positions < pos0[b]) come from the cache: full layers read rows

@@ -209,7 +209,7 @@ def test_decode_rejects_position_beyond_cache():
 
 # --------------------------------------------------------------- prefill ----
 
-def _prefill_case(kind, B, T, pos0_list, seed=21, layer=0, sigma_k=1.0, sigma_g=1.0):
+def _prefill_case(kind, B, T, pos0_list, seed=21, layer=0, sigma_k=1.0, sigma_g=1.0, fused_q=False):
     sliding = kind == O.SLIDING
     has_hist = max(pos0_list) > 0
     assert not (sliding and has_hist) or len(set(pos0_list)) == 1
@@ -221,7 +221,8 @@ def _prefill_case(kind, B, T, pos0_list, seed=21, layer=0, sigma_k=1.0, sigma_g=
     cfg = _cfg(kind)
     p0 = _pos_tensor(pos0_list)
     q, k = to_dev(qb), to_dev(kb)
-    sa.spark_rope_apply(q, p0, cfg)
+    if not fused_q:
+        sa.spark_rope_apply(q, p0, cfg)
     sa.spark_rope_apply(k, p0, cfg)
     kc = vc = None
     if has_hist:
@@ -232,7 +233,8 @@ def _prefill_case(kind, B, T, pos0_list, seed=21, layer=0, sigma_k=1.0, sigma_g=
         synth.fill_cache(kc, seed, tid(layer, synth.ROLE_K), n_hist, sliding, sigma_k)
         synth.fill_cache(vc, seed, tid(layer, synth.ROLE_V), n_hist, sliding)
     out = torch.full((B, T, 16, 256), float("nan"), dtype=torch.bfloat16, device="cuda")
-    sa.spark_attn_prefill(out, q, k, to_dev(vb), to_dev(gb), kc, vc, p0, cfg)
+    sa.spark_attn_prefill(out, q, k, to_dev(vb), to_dev(gb), kc, vc, p0, cfg,
+                          flags=sa.SPARK_ROPE_FUSED if fused_q else 0)
     sa.spark_check()
     got = dev_to_f64(out)
     refs = []
@@ -280,3 +282,16 @@ def test_prefill_tiny_config_all_elements(kind):
     layer = 0 if kind == O.SLIDING else 3
     got, ref = _prefill_case(kind, 1, 1024, [0], seed=0, layer=layer)
     assert_close(got, ref, f"tiny prefill {KIND_NAME[kind]}")
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("T,pos0", [(1, 0), (129, 0), (640, 0), (200, 700), (256, (1 << 20) - 256)])
+def test_prefill_rope_fused_at_load(kind, T, pos0):
+    """q is raw; the prefill block rotates its Q tile in shared memory before the first MMA."""
+    got, ref = _prefill_case(kind, 1, T, [pos0], fused_q=True)
+    assert_close(got, ref, f"prefill {KIND_NAME[kind]} fused RoPE T={T} pos0={pos0}")
+
+
+def test_prefill_rope_fused_batch_positions():
+    got, ref = _prefill_case(O.FULL, 3, 300, [0, 128, 5000], fused_q=True)
+    assert_close(got, ref, "prefill full fused RoPE, per-sequence pos0")

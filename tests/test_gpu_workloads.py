@@ -52,9 +52,9 @@ def test_prefill_b4_t8192_sampled_rows():
                                      rng.integers(0, T, 4)]))
     for kind, layer in ((O.SLIDING, 0), (O.FULL, 3)):
         w = W[kind]
-        sa.spark_rope_apply(w["q"], pos0, w["cfg"])
-        sa.spark_rope_apply(w["k"], pos0, w["cfg"])
-        sa.spark_attn_prefill(w["out"], w["q"], w["k"], w["v"], w["g"], None, None, pos0, w["cfg"])
+        sa.spark_rope_apply(w["k"], pos0, w["cfg"])                  # as in bench.prefill_step:
+        sa.spark_attn_prefill(w["out"], w["q"], w["k"], w["v"], w["g"], None, None, pos0, w["cfg"],
+                              flags=sa.SPARK_ROPE_FUSED)              # q raw, rotated at load
         sa.spark_check()
         for b in (0, 3):
             got = dev_to_f64(w["out"][b, torch.as_tensor(rows, device=dev)])
@@ -135,9 +135,9 @@ def test_long_prefill_chunked_sampled_rows():
             synth.fill_tokens(v, seed, tid(layer, synth.ROLE_V), p0)
             synth.fill_tokens(gt, seed, tid(layer, synth.ROLE_GATE), p0)
             pos0 = torch.full((1,), p0, dtype=torch.int32, device=dev)
-            sa.spark_rope_apply(q, pos0, cfg)
             sa.spark_rope_apply(k, pos0, cfg)
-            sa.spark_attn_prefill(out, q, k, v, gt, kc if c else None, vc if c else None, pos0, cfg)
+            sa.spark_attn_prefill(out, q, k, v, gt, kc if c else None, vc if c else None, pos0, cfg,
+                                  flags=sa.SPARK_ROPE_FUSED)
             sa.spark_kv_append(kc, vc, k, v, pos0, cfg)
             if c in check_chunks:
                 got[c] = dev_to_f64(out[0, torch.as_tensor(rel, device=dev)])
