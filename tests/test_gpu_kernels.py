@@ -209,9 +209,11 @@ def test_decode_rejects_position_beyond_cache():
 
 # --------------------------------------------------------------- prefill ----
 
-def _prefill_case(kind, B, T, pos0_list, seed=21, layer=0, sigma_k=1.0, sigma_g=1.0, fused_q=False):
+def _prefill_case(kind, B, T, pos0_list, seed=21, layer=0, sigma_k=1.0, sigma_g=1.0, fused_q=False,
+                  history=True):
+    """history=False: positions start at pos0 but no cache is passed, so each chunk sees only itself."""
     sliding = kind == O.SLIDING
-    has_hist = max(pos0_list) > 0
+    has_hist = history and max(pos0_list) > 0
     assert not (sliding and has_hist) or len(set(pos0_list)) == 1
     pos = np.array([[p + t for t in range(T)] for p in pos0_list])
     qb = synth.token_tensor(seed, tid(layer, synth.ROLE_Q), B, 16, 256, pos)
@@ -239,7 +241,7 @@ def _prefill_case(kind, B, T, pos0_list, seed=21, layer=0, sigma_k=1.0, sigma_g=
     got = dev_to_f64(out)
     refs = []
     for b, p0b in enumerate(pos0_list):
-        hp = np.arange(max(0, p0b - 511) if sliding else 0, p0b)
+        hp = np.arange(max(0, p0b - 511) if sliding else 0, p0b) if has_hist else np.arange(0)
         hist_k = hist_v = None
         if len(hp):
             hist_k = np.stack([f64(synth.head_slice(seed, tid(layer, synth.ROLE_K), b, g, 4, 256, hp, sigma_k))
@@ -285,10 +287,13 @@ def test_prefill_tiny_config_all_elements(kind):
 
 
 @pytest.mark.parametrize("kind", KINDS)
-@pytest.mark.parametrize("T,pos0", [(1, 0), (129, 0), (640, 0), (200, 700), (256, (1 << 20) - 256)])
-def test_prefill_rope_fused_at_load(kind, T, pos0):
-    """q is raw; the prefill block rotates its Q tile in shared memory before the first MMA."""
-    got, ref = _prefill_case(kind, 1, T, [pos0], fused_q=True)
+@pytest.mark.parametrize("T,pos0,history", [(1, 0, True), (129, 0, True), (640, 0, True), (200, 700, True),
+                                            (256, (1 << 20) - 256, False), (300, 777777, False)])
+def test_prefill_rope_fused_at_load(kind, T, pos0, history):
+    """q is raw; the prefill block rotates its Q tile in shared memory before the first MMA.
+    The cases near position 2^20 pass no cache (the chunk sees only itself) to keep the
+    oracle's work small while still exercising the largest rotation angles."""
+    got, ref = _prefill_case(kind, 1, T, [pos0], fused_q=True, history=history)
     assert_close(got, ref, f"prefill {KIND_NAME[kind]} fused RoPE T={T} pos0={pos0}")
 
 
