@@ -308,3 +308,47 @@ def stack_kv_bytes(n_ctx: int, bytes_per_elem: float = 2.0) -> float:
     n_slide = N_LAYERS - n_full
     per_tok = kv_bytes_per_token_full_layer(bytes_per_elem)
     return n_full * per_tok * n_ctx + n_slide * per_tok * min(n_ctx, WINDOW)
+
+
+# ---------------------------------------------------------------------------
+# 8-bit block-quantised KV cache (q8_0-style): 32-value blocks, one fp16 scale
+# ---------------------------------------------------------------------------
+
+Q8_BLOCK = 32
+
+
+def quantize_q8(x):
+    """Quantise rows of 256 values into 8 blocks of 32: codes and fp16 scales.
+
+    [GGUF] §四: the KV cache can be stored as q8_0, 8-bit values in blocks that
+    carry one scale each, cutting 36 KB per token to 19 KB.  The pages give the
+    format's name and byte count only; the reading taken here: per block,
+    amax = max |x|, scale d = fp16(amax / 127), code c = round-half-away-from-
+    zero(x * (127 / amax)) in [-127, 127], stored offset by 128 as a byte.  All
+    arithmetic before the rounding is float32 (the same operations the device
+    performs), so the codes are exact integers both sides agree on.
+    Returns (u8 codes [..., 256], fp16 scales [..., 8]).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    blocks = x.reshape(x.shape[:-1] + (x.shape[-1] // Q8_BLOCK, Q8_BLOCK))
+    amax = np.max(np.abs(blocks), axis=-1, keepdims=True).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        inv = np.where(amax > 0, np.float32(127.0) / amax, np.float32(0.0)).astype(np.float32)
+    y = (blocks * inv).astype(np.float32)
+    c = np.sign(y) * np.floor(np.abs(y) + np.float32(0.5))
+    codes = (c + 128).astype(np.uint8).reshape(x.shape)
+    scales = (amax[..., 0] / np.float32(127.0)).astype(np.float32).astype(np.float16)
+    return codes, scales
+
+
+def dequantize_q8(codes, scales):
+    """Values of a quantised row: scale * code, in float64."""
+    c = np.asarray(codes, dtype=np.float64) - 128.0
+    d = np.asarray(scales, dtype=np.float64)
+    blocks = c.reshape(c.shape[:-1] + (c.shape[-1] // Q8_BLOCK, Q8_BLOCK))
+    return (blocks * d[..., None]).reshape(c.shape)
+
+
+def q8_bytes_per_value() -> float:
+    """34 bytes per 32 values: 32 codes and a 2-byte scale."""
+    return (Q8_BLOCK + 2) / Q8_BLOCK

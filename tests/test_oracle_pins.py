@@ -338,3 +338,40 @@ def test_group_attention_equals_the_full_form(kind):
         hs = slice(4 * grp, 4 * grp + 4)
         part = O.attention_group(q[:, hs], k[:, grp], v[:, grp], g[:, hs], pos, pos, kind)
         np.testing.assert_allclose(part, full[:, hs], rtol=1e-12, atol=1e-14)
+
+
+# ----------------------------------------------------- 8-bit KV blocks -----
+
+def test_q8_worked_example():
+    """Hand-computed block: amax 1 -> scale 1/127; -0.5 * 127 = -63.5 rounds away from zero to -64."""
+    x = np.zeros(256, dtype=np.float32)
+    x[:4] = [1.0, -0.5, 0.25, -1.0]
+    codes, scales = O.quantize_q8(x)
+    assert list(codes[:4].astype(int) - 128) == [127, -64, 32, -127]
+    assert np.all(codes[4:32] == 128)
+    assert scales[0] == np.float16(1.0 / 127.0)
+    assert np.all(scales[1:] == 0) and np.all(codes[32:] == 128)        # all-zero blocks
+
+
+def test_q8_round_trip_bound_and_code_range():
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((64, 256)) * rng.uniform(0.01, 5, (64, 1))).astype(np.float32)
+    codes, scales = O.quantize_q8(x)
+    c = codes.astype(int) - 128
+    assert c.min() >= -127 and c.max() <= 127
+    blocks = np.abs(x).reshape(64, 8, 32)
+    # the largest magnitude of every block maps to +-127
+    arg = blocks.argmax(axis=-1)
+    assert np.all(np.abs(np.take_along_axis(c.reshape(64, 8, 32), arg[..., None], -1)) == 127)
+    # |x - dequant| <= half a step plus the fp16 rounding of the scale
+    amax = blocks.max(axis=-1)
+    step = amax / 127.0
+    err = np.abs(x.astype(np.float64) - O.dequantize_q8(codes, scales)).reshape(64, 8, 32)
+    bound = step[..., None] * 0.5 * (1 + 2 ** -10) + amax[..., None] * 2 ** -11
+    assert np.all(err <= bound)
+
+
+def test_q8_bytes_match_the_pages():
+    g = _golden("pages_numbers.txt")
+    per_tok_q8 = O.kv_bytes_per_token_full_layer(O.q8_bytes_per_value()) * 9
+    assert round(per_tok_q8 / 1024) == float(g["kv_kb_per_token_q8_0_stack"][0])   # 36 KB -> 19 KB
