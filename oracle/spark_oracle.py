@@ -326,14 +326,17 @@ def quantize_q8(x):
     amax = max |x|, scale d = fp16(amax / 127), code c = round-half-away-from-
     zero(x * (127 / amax)) in [-127, 127], stored offset by 128 as a byte.  All
     arithmetic before the rounding is float32 (the same operations the device
-    performs), so the codes are exact integers both sides agree on.
+    performs), so the codes are exact integers both sides agree on.  A block
+    whose 127 / amax is not a finite float32 (amax below ~3.7e-37, so its fp16
+    scale is 0 anyway) gets code 0 throughout, like an all-zero block.
     Returns (u8 codes [..., 256], fp16 scales [..., 8]).
     """
     x = np.asarray(x, dtype=np.float32)
     blocks = x.reshape(x.shape[:-1] + (x.shape[-1] // Q8_BLOCK, Q8_BLOCK))
     amax = np.max(np.abs(blocks), axis=-1, keepdims=True).astype(np.float32)
-    with np.errstate(divide="ignore", invalid="ignore"):
-        inv = np.where(amax > 0, np.float32(127.0) / amax, np.float32(0.0)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+        inv = (np.float32(127.0) / amax).astype(np.float32)
+        inv = np.where((amax > 0) & np.isfinite(inv), inv, np.float32(0.0)).astype(np.float32)
     y = (blocks * inv).astype(np.float32)
     c = np.sign(y) * np.floor(np.abs(y) + np.float32(0.5))
     codes = (c + 128).astype(np.uint8).reshape(x.shape)

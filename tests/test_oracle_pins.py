@@ -353,6 +353,20 @@ def test_q8_worked_example():
     assert np.all(scales[1:] == 0) and np.all(codes[32:] == 128)        # all-zero blocks
 
 
+def test_q8_tiny_block_quantises_to_zero():
+    """127 / amax overflows float32 for a block of denormal values: codes 0, scale 0 (no inf or NaN)."""
+    x = np.zeros(256, dtype=np.float32)
+    x[0] = np.float32(1e-40)
+    x[40] = np.float32(-3e-38)
+    codes, scales = O.quantize_q8(x)
+    assert np.all(codes == 128) and np.all(scales == 0)
+    assert np.all(O.dequantize_q8(codes, scales) == 0)
+    # just above the overflow threshold the block still quantises normally
+    x[64] = np.float32(1e-36)
+    codes, scales = O.quantize_q8(x)
+    assert codes[64] == 255 and scales[2] == 0          # the fp16 scale itself underflows
+
+
 def test_q8_round_trip_bound_and_code_range():
     rng = np.random.default_rng(3)
     x = (rng.standard_normal((64, 256)) * rng.uniform(0.01, 5, (64, 1))).astype(np.float32)
