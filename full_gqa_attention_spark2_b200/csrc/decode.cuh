@@ -172,6 +172,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       break;
     const uint32_t kt = base + s * kDecStageBytes;
     const uint32_t vt = kt + kDecTileBytes;
+    const int tile_key0 = key_begin + i * kDecNK;
+    if (tile_key0 + kDecNK > key_end) {
+      // Rows past the last key may hold anything, NaN included, and a zero
+      // probability does not cancel a NaN.  Each warp clears the V rows of its
+      // own keys there (its P.V reads no other rows).  This is the split's
+      // last tile, so no later copy lands in this stage.
+      for (int e = lane; e < 16 * 32; e += 32) {
+        const int key = warp * 16 + (e >> 5);
+        if (tile_key0 + key >= key_end)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(swz_addr(vt, key, (e & 31) * 8)), "r"(0)
+                       : "memory");
+      }
+      __syncwarp();
+    }
 
     // S = Q K^T for this warp's 16 keys, two accumulation chains per n-tile
     float sa[2][2][4];

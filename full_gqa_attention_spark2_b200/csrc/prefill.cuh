@@ -74,9 +74,18 @@ __device__ __forceinline__ PfTile pf_tile(const PfSchedule& S, const PrefillPara
   if (j < S.n_hist) {
     t.hist = 1;
     t.kt0 = S.a0 + j * kPfN;
-    t.row = P.sliding ? (t.kt0 & (kWindow - 1)) : t.kt0;
     t.v_lo = S.need_lo;
     t.v_hi = S.pos0;
+    // Cache rows at and past pos0 may never have been written, and a masked
+    // score does not cancel a NaN there (0 * NaN).  So the last history tile
+    // is moved back to end exactly at pos0, and the keys it shares with the
+    // tile before it are masked.  Rows before 0 are the TMA's zero fill.  A
+    // ring that has wrapped (pos0 >= 512) holds written rows everywhere.
+    if (j == S.n_hist - 1 && t.kt0 + kPfN > S.pos0 && (!P.sliding || S.pos0 < kWindow)) {
+      t.v_lo = max(S.need_lo, t.kt0);
+      t.kt0 = S.pos0 - kPfN;
+    }
+    t.row = (P.sliding && t.kt0 >= 0) ? (t.kt0 & (kWindow - 1)) : t.kt0;
   } else {
     const int c = S.c_lo + (j - S.n_hist);
     t.hist = 0;

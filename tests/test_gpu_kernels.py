@@ -139,8 +139,9 @@ def test_host_side_argument_checks():
 
 # ---------------------------------------------------------------- decode ----
 
-def _decode_case(kind, B, p_list, seed=11, layer=0, fused_q=True, cap_extra=5):
-    """Append the new token (rope fused) and decode; return (out, reference)."""
+def _decode_case(kind, B, p_list, seed=11, layer=0, fused_q=True, cap_extra=5, poison=False):
+    """Append the new token (rope fused) and decode; return (out, reference).
+    poison: cache rows past each sequence's new token hold NaN (memory the caller never wrote)."""
     sliding = kind == O.SLIDING
     assert not sliding or len(set(p_list)) == 1
     cap = 512 if sliding else max(p_list) + 1 + cap_extra
@@ -158,6 +159,11 @@ def _decode_case(kind, B, p_list, seed=11, layer=0, fused_q=True, cap_extra=5):
     pos = _pos_tensor(p_list)
     cfg = _cfg(kind)
     sa.spark_kv_append(kc, vc, to_dev(kb), to_dev(vb), pos, cfg, flags=sa.SPARK_ROPE_FUSED)
+    if poison:
+        for b, p in enumerate(p_list):
+            if not sliding or p < 511:
+                kc[b, :, p + 1:] = float("nan")
+                vc[b, :, p + 1:] = float("nan")
     q = to_dev(qb)
     if not fused_q:
         q4 = q.view(B, 1, 16, 256)
@@ -189,6 +195,16 @@ def test_decode_full(p_list):
     assert_close(got, ref, f"decode full p={p_list}")
 
 
+@pytest.mark.parametrize("kind,p_list", [(O.FULL, [5, 64, 65]), (O.FULL, [127, 128, 129, 3000]),
+                                         (O.SLIDING, [0]), (O.SLIDING, [63]), (O.SLIDING, [64]),
+                                         (O.SLIDING, [200])])
+def test_decode_ignores_nan_past_the_last_key(kind, p_list):
+    """Rows the caller never wrote may hold NaN; a zero probability must not multiply them."""
+    got, ref = _decode_case(kind, len(p_list), p_list, cap_extra=100, poison=True)
+    assert np.isfinite(got).all()
+    assert_close(got, ref, f"decode {KIND_NAME[kind]} p={p_list}, NaN past the last key")
+
+
 def test_decode_unfused_q_matches_fused():
     got, ref = _decode_case(O.FULL, 2, [700, 1500], fused_q=False)
     assert_close(got, ref, "decode full, q rotated by spark_rope_apply")
@@ -210,8 +226,9 @@ def test_decode_rejects_position_beyond_cache():
 # --------------------------------------------------------------- prefill ----
 
 def _prefill_case(kind, B, T, pos0_list, seed=21, layer=0, sigma_k=1.0, sigma_g=1.0, fused_q=False,
-                  history=True):
-    """history=False: positions start at pos0 but no cache is passed, so each chunk sees only itself."""
+                  history=True, poison=False, cap_extra=7):
+    """history=False: positions start at pos0 but no cache is passed, so each chunk sees only itself.
+    poison: cache rows that hold no history position are NaN (memory the caller never wrote)."""
     sliding = kind == O.SLIDING
     has_hist = history and max(pos0_list) > 0
     assert not (sliding and has_hist) or len(set(pos0_list)) == 1
@@ -229,11 +246,16 @@ def _prefill_case(kind, B, T, pos0_list, seed=21, layer=0, sigma_k=1.0, sigma_g=
     kc = vc = None
     if has_hist:
         n_hist = max(pos0_list)
-        cap = 512 if sliding else n_hist + 7
+        cap = 512 if sliding else n_hist + cap_extra
         kc = torch.empty(B, 4, cap, 256, dtype=torch.bfloat16, device="cuda")
         vc = torch.empty_like(kc)
         synth.fill_cache(kc, seed, tid(layer, synth.ROLE_K), n_hist, sliding, sigma_k)
         synth.fill_cache(vc, seed, tid(layer, synth.ROLE_V), n_hist, sliding)
+        if poison:
+            for b, p0b in enumerate(pos0_list):
+                if not sliding or p0b < 512:
+                    kc[b, :, p0b:] = float("nan")
+                    vc[b, :, p0b:] = float("nan")
     out = torch.full((B, T, 16, 256), float("nan"), dtype=torch.bfloat16, device="cuda")
     sa.spark_attn_prefill(out, q, k, to_dev(vb), to_dev(gb), kc, vc, p0, cfg,
                           flags=sa.SPARK_ROPE_FUSED if fused_q else 0)
@@ -300,3 +322,13 @@ def test_prefill_rope_fused_at_load(kind, T, pos0, history):
 def test_prefill_rope_fused_batch_positions():
     got, ref = _prefill_case(O.FULL, 3, 300, [0, 128, 5000], fused_q=True)
     assert_close(got, ref, "prefill full fused RoPE, per-sequence pos0")
+
+
+@pytest.mark.parametrize("kind,T,pos0_list", [(O.FULL, 100, [333]), (O.FULL, 129, [1]), (O.FULL, 256, [256]),
+                                              (O.FULL, 160, [0, 200, 900]), (O.SLIDING, 300, [200]),
+                                              (O.SLIDING, 129, [1]), (O.SLIDING, 64, [130])])
+def test_prefill_ignores_nan_past_the_history(kind, T, pos0_list):
+    """Cache rows at and past pos0 may hold NaN; the last history tile must not read them."""
+    got, ref = _prefill_case(kind, len(pos0_list), T, pos0_list, poison=True, cap_extra=200)
+    assert np.isfinite(got).all()
+    assert_close(got, ref, f"prefill {KIND_NAME[kind]} T={T} pos0={pos0_list}, NaN past the history")
