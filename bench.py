@@ -63,6 +63,12 @@ def decode_kv_bytes(B: int, p: int, kind: int) -> int:
     return B * keys * HKV * 2 * D * 2
 
 
+def decode_q8_kv_bytes(B: int, p: int, kind: int) -> int:
+    """The same for the 8-bit cache: per key and KV head, K and V codes (256 B each) and scales (16 B each)."""
+    keys = p + 1 if kind == FULL else min(p + 1, WINDOW)
+    return B * keys * HKV * 2 * (D + 2 * (D // 32))
+
+
 # ------------------------------------------------------------- plumbing -----
 
 def dist_env():
@@ -373,6 +379,99 @@ def run_decode(torch, sa, synth, dist, args, peaks, world):
     }
 
 
+def decode_q8_layers(torch, sa, synth, dev, B: int, p: int, layer_ids=range(N_LAYERS), seed: int = DECODE_SEED,
+                     chunk: int = 2048):
+    """8-bit caches holding positions 0..p-1 (quantised by spark_kv_append_q8 from the generator's
+    tokens, keys taken as rotated) and the new token's q/k/v/gate at p, per layer."""
+    layers = []
+    for l in layer_ids:
+        kind = FULL if l % 4 == 3 else SLIDING
+        cfg = sa.spark_layer_cfg_for_kind(kind)
+        cap = WINDOW if kind == SLIDING else p + 1
+        kc = torch.empty(B, HKV, cap, D, dtype=torch.uint8, device=dev)
+        vc = torch.empty_like(kc)
+        ks = torch.empty(B, HKV, cap, D // 32, dtype=torch.float16, device=dev)
+        vs = torch.empty_like(ks)
+        first = 0 if kind == FULL else max(0, p - WINDOW)
+        for c0 in range(first, p, chunk):
+            n = min(chunk, p - c0)
+            kt = torch.empty(B, n, HKV, D, dtype=torch.bfloat16, device=dev)
+            vt = torch.empty_like(kt)
+            synth.fill_tokens(kt, seed, synth.tensor_id(l, synth.ROLE_K), c0)
+            synth.fill_tokens(vt, seed, synth.tensor_id(l, synth.ROLE_V), c0)
+            sa.spark_kv_append_q8(kc, ks, vc, vs, kt, vt, torch.full((B,), c0, dtype=torch.int32, device=dev), cfg)
+            del kt, vt
+        q = torch.empty(B, 1, HQ, D, dtype=torch.bfloat16, device=dev)
+        kn = torch.empty(B, 1, HKV, D, dtype=torch.bfloat16, device=dev)
+        vn = torch.empty_like(kn)
+        g = torch.empty(B, 1, HQ, dtype=torch.bfloat16, device=dev)
+        synth.fill_tokens(q, seed, synth.tensor_id(l, synth.ROLE_Q), p)
+        synth.fill_tokens(kn, seed, synth.tensor_id(l, synth.ROLE_K), p)
+        synth.fill_tokens(vn, seed, synth.tensor_id(l, synth.ROLE_V), p)
+        synth.fill_tokens(g, seed, synth.tensor_id(l, synth.ROLE_GATE), p)
+        layers.append(dict(layer=l, kind=kind, cfg=cfg, cap=cap, kc=kc, vc=vc, ks=ks, vs=vs, q=q.view(B, HQ, D),
+                           kn=kn, vn=vn, g=g.view(B, HQ),
+                           out=torch.empty(B, HQ, D, dtype=torch.bfloat16, device=dev)))
+    sa.spark_check()
+    return layers
+
+
+def decode_q8_step(sa, layers, pos, ws):
+    """One decode step over 8-bit caches: per layer, quantise-append the new token (RoPE fused on k),
+    then attend (RoPE fused on q)."""
+    for L in layers:
+        sa.spark_kv_append_q8(L["kc"], L["ks"], L["vc"], L["vs"], L["kn"], L["vn"], pos, L["cfg"],
+                              flags=sa.SPARK_ROPE_FUSED)
+        sa.spark_attn_decode_q8(L["out"], L["q"], L["g"], L["kc"], L["ks"], L["vc"], L["vs"], pos, L["cfg"], ws,
+                                flags=sa.SPARK_ROPE_FUSED)
+
+
+def run_decode_q8(torch, sa, synth, dist, args, peaks, world):
+    """The decode step of run_decode (36 layers, B=64, 32768 cached tokens, one CUDA graph) over the
+    8-bit KV cache."""
+    dev = torch.device("cuda")
+    B, p = DECODE_B, DECODE_CTX
+    layers = decode_q8_layers(torch, sa, synth, dev, B, p)
+    pos = torch.full((B,), p, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(sa.spark_decode_q8_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers),
+                     dtype=torch.uint8, device=dev)
+    decode_q8_step(sa, layers, pos, ws)
+    torch.cuda.synchronize()
+    sa.spark_check()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        decode_q8_step(sa, layers, pos, ws)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    dsteps = max(5, min(args.steps, 30))
+    ms_step = timed_region(torch, dist, lambda i: graph.replay(), dsteps) / dsteps
+    sa.spark_check()
+    full = layers[3]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    e0.record()
+    for _ in range(reps):
+        sa.spark_attn_decode_q8(full["out"], full["q"], full["g"], full["kc"], full["ks"], full["vc"], full["vs"],
+                                pos, full["cfg"], ws, flags=sa.SPARK_ROPE_FUSED)
+    e1.record()
+    torch.cuda.synchronize()
+    k_ms = e0.elapsed_time(e1) / reps
+    total_bytes = sum(decode_q8_kv_bytes(B, p, L["kind"]) for L in layers)
+    full_bytes = decode_q8_kv_bytes(B, p, FULL)
+    del graph, layers, ws
+    torch.cuda.empty_cache()
+    return {
+        "value": total_bytes * world / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
+        "ms_per_step": ms_step, "steps_per_s": 1e3 / ms_step, "kv_bytes_per_step": total_bytes,
+        "workload": f"decode_q8_b{B}_ctx{p}_36layers", "gpu_launches_per_step": 3 * N_LAYERS,
+        "roofline": {"bound": "hbm", "kernel": "decode_q8_partial_kernel+combine (full layer)",
+                     "achieved": full_bytes / (k_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": full_bytes / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "traffic": ncu_traffic("decode_q8_partial_kernel_full")},
+    }
+
+
 def run_long_prefill(torch, sa, synth, dist, args, peaks, world):
     """B=1, T=131072 in 16 chunks of 8192 over the growing cache, one full and one sliding layer."""
     dev = torch.device("cuda")
@@ -533,6 +632,14 @@ def run_profile_case(torch, sa, synth, which: str):
         ws = torch.empty(sa.spark_decode_workspace_bytes(B, p + 1, cfg), dtype=torch.uint8, device=dev)
         for _ in range(3):
             sa.spark_attn_decode(out, q.view(B, HQ, D), g.view(B, HQ), kc, vc, pos, cfg, ws, flags=sa.SPARK_ROPE_FUSED)
+    elif which == "decode_q8_full":
+        B, p = 16, DECODE_CTX
+        L = decode_q8_layers(torch, sa, synth, dev, B, p, layer_ids=(3,))[0]
+        pos = torch.full((B,), p, dtype=torch.int32, device=dev)
+        ws = torch.empty(sa.spark_decode_q8_workspace_bytes(B, L["cap"], L["cfg"]), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            sa.spark_attn_decode_q8(L["out"], L["q"], L["g"], L["kc"], L["ks"], L["vc"], L["vs"], pos, L["cfg"], ws,
+                                    flags=sa.SPARK_ROPE_FUSED)
     else:
         raise SystemExit(f"unknown profile case {which}")
     sa.spark_check()
@@ -548,7 +655,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context prefill and decode workloads")
-    ap.add_argument("--profile", choices=["prefill_full", "prefill_sliding", "decode_full"], default=None,
+    ap.add_argument("--profile", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_q8_full"],
+                    default=None,
                     help="run a small case of one kernel for ncu and exit")
     args = ap.parse_args()
     rank, world, local = dist_env()
@@ -577,6 +685,7 @@ def main():
 
     res = run_prefill(torch, sa, synth, dist, args, peaks, world)
     dec = None if args.no_decode else run_decode(torch, sa, synth, dist, args, peaks, world)
+    dec_q8 = None if args.no_decode else run_decode_q8(torch, sa, synth, dist, args, peaks, world)
     long_pf = None if args.no_long else run_long_prefill(torch, sa, synth, dist, args, peaks, world)
     long_dec = None if (args.no_long or args.no_decode) else run_long_decode(torch, sa, synth, dist, args, peaks, world)
     cpu = None
@@ -601,7 +710,7 @@ def main():
         "tflops": res["tflops"], "prefill_full_kernel": res["prefill_full_kernel"],
         "roofline": res["roofline"], "e2e": res["e2e"], "clocks": res["clocks"],
         "gpu_launches": res["gpu_launches"] + (0 if dec is None else 0),
-        "cpu_baseline": cpu, "decode": dec, "long_prefill": long_pf, "long_decode": long_dec,
+        "cpu_baseline": cpu, "decode": dec, "decode_q8": dec_q8, "long_prefill": long_pf, "long_decode": long_dec,
     }
     print(json.dumps(line), flush=True)
 

@@ -67,6 +67,11 @@ def _lib():
         "spark_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
         "spark_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, cfgp, _P, ctypes.c_size_t, ctypes.c_uint, _P]),
         "spark_attn_decode_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
+        "spark_kv_cache_q8_bytes": (ctypes.c_longlong, [cfgp, _I, ctypes.c_longlong]),
+        "spark_kv_append_q8": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
+        "spark_decode_q8_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
+        "spark_attn_decode_q8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _P, cfgp, _P, ctypes.c_size_t,
+                                      ctypes.c_uint, _P]),
         "spark_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
         "spark_check": (_I, [_P]),
         "spark_last_error": (ctypes.c_char_p, []),
@@ -84,8 +89,9 @@ def exported_symbols():
     """Names of the C entry points this binding expects the library to export."""
     return ["spark_layer_cfg_for_layer", "spark_layer_cfg_for_kind", "spark_kv_cache_bytes",
             "spark_stack_kv_bytes", "spark_rope_apply", "spark_kv_append", "spark_attn_prefill",
-            "spark_decode_workspace_bytes", "spark_attn_decode", "spark_attn_decode_static", "spark_selftest_wait_timeout", "spark_check",
-            "spark_last_error",
+            "spark_decode_workspace_bytes", "spark_attn_decode", "spark_attn_decode_static",
+            "spark_kv_cache_q8_bytes", "spark_kv_append_q8", "spark_decode_q8_workspace_bytes",
+            "spark_attn_decode_q8", "spark_selftest_wait_timeout", "spark_check", "spark_last_error",
             "spark_version"]
 
 
@@ -207,6 +213,51 @@ def spark_attn_decode_static(out, q, gate, k_cache, v_cache, pos, cfg: SparkLaye
     pp = _dev(pos, "pos", torch.int32, 1)
     _raise(_lib().spark_attn_decode_static(po, pq, pg, pkc, pvc, k_cache.shape[2], q.shape[0], pp,
                                            ctypes.byref(cfg), flags, _stream(stream)))
+
+
+def spark_kv_cache_q8_bytes(cfg: SparkLayerCfg, B: int, cap: int) -> int:
+    return int(_lib().spark_kv_cache_q8_bytes(ctypes.byref(cfg), B, cap))
+
+
+def _q8_pair(codes, scales, name):
+    pc = _dev(codes, f"{name}_codes", torch.uint8, 4)
+    ps = _dev(scales, f"{name}_scales", torch.float16, 4)
+    if tuple(scales.shape) != tuple(codes.shape[:3]) + (codes.shape[3] // 32,):
+        raise ValueError(f"{name}_scales must be [B, 4, cap, 8] beside codes [B, 4, cap, 256]")
+    return pc, ps
+
+
+def spark_kv_append_q8(k_codes, k_scales, v_codes, v_scales, k, v, pos0, cfg: SparkLayerCfg, flags: int = 0,
+                       stream=None) -> None:
+    """Quantise and append k, v [B, T, 4, 256] bf16 into 8-bit caches: codes uint8 [B, 4, cap, 256] and
+    scales float16 [B, 4, cap, 8] (see include/spark_attn.h)."""
+    pkc, pks = _q8_pair(k_codes, k_scales, "k")
+    pvc, pvs = _q8_pair(v_codes, v_scales, "v")
+    pk, pv = _dev(k, "k", ndim=4), _dev(v, "v", ndim=4)
+    pp = _dev(pos0, "pos0", torch.int32, 1)
+    B, T = k.shape[0], k.shape[1]
+    _raise(_lib().spark_kv_append_q8(pkc, pks, pvc, pvs, k_codes.shape[2], pk, pv, B, T, pp, ctypes.byref(cfg),
+                                     flags, _stream(stream)))
+
+
+def spark_decode_q8_workspace_bytes(B: int, cap: int, cfg: SparkLayerCfg) -> int:
+    return int(_lib().spark_decode_q8_workspace_bytes(B, cap, ctypes.byref(cfg)))
+
+
+def spark_attn_decode_q8(out, q, gate, k_codes, k_scales, v_codes, v_scales, pos, cfg: SparkLayerCfg,
+                         workspace: torch.Tensor, flags: int = 0, stream=None) -> None:
+    """spark_attn_decode over 8-bit caches (codes + scales per K and V)."""
+    po, pq = _dev(out, "out", ndim=3), _dev(q, "q", ndim=3)
+    pg = _dev(gate, "gate", ndim=2)
+    pkc, pks = _q8_pair(k_codes, k_scales, "k")
+    pvc, pvs = _q8_pair(v_codes, v_scales, "v")
+    pp = _dev(pos, "pos", torch.int32, 1)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _raise(_lib().spark_attn_decode_q8(po, pq, pg, pkc, pks, pvc, pvs, k_codes.shape[2], q.shape[0], pp,
+                                       ctypes.byref(cfg), workspace.data_ptr(), ws_bytes, flags,
+                                       _stream(stream)))
 
 
 def spark_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:

@@ -17,6 +17,7 @@
 #include "prefill.cuh"
 #include "prefill2.cuh"
 #include "ptx.cuh"
+#include "q8.cuh"
 #include "rope_append.cuh"
 
 namespace spark {
@@ -85,9 +86,12 @@ int device_ready(int* dev_out) {
     cudaError_t b = cudaFuncSetAttribute(spark::prefill2_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          spark::kP2SmemBytes);
-    if (a != cudaSuccess || b != cudaSuccess) {
+    cudaError_t c = cudaFuncSetAttribute(spark::decode_q8_partial_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         spark::kQ8SmemBytes);
+    if (a != cudaSuccess || b != cudaSuccess || c != cudaSuccess) {
       snprintf(d.why, sizeof(d.why), "cudaFuncSetAttribute: %s",
-               cudaGetErrorString(a != cudaSuccess ? a : b));
+               cudaGetErrorString(a != cudaSuccess ? a : b != cudaSuccess ? b : c));
       return;
     }
     d.ok = 1;
@@ -130,17 +134,24 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map, 128-byte swizzle, dims/strides innermost first (strides in bytes, rank-1 of them)
-int make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-             const cuuint32_t* box) {
+// Tensor map, dims/strides innermost first (strides in bytes, rank-1 of them).
+int make_map_t(CUtensorMap* m, CUtensorMapDataType dtype, CUtensorMapSwizzle swz, const void* ptr, int rank,
+               const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(SPARK_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), dims,
-                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(m, dtype, (cuuint32_t)rank, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SPARK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return SPARK_OK;
+}
+
+// bf16 tensor map with the 128-byte swizzle
+int make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+             const cuuint32_t* box) {
+  return make_map_t(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_128B, ptr, rank, dims, strides,
+                    box);
 }
 
 // -------------------------------------------------------------- checks -----
@@ -197,6 +208,11 @@ DecodePlan decode_plan(int B, int cap, int sliding, int sm_count) {
 size_t decode_ws_bytes(int B, const DecodePlan& pl) {
   const size_t rows = (size_t)B * spark::kNq * pl.n_splits;
   return rows * spark::kHeadDim * sizeof(float) + rows * 2 * sizeof(float);
+}
+
+// One q8 decode block per SM, like the bf16 one.
+DecodePlan decode_q8_plan(int B, int cap, int sliding, int sm_count) {
+  return decode_plan(B, cap, sliding, sm_count);
 }
 
 // ------------------------------------------------- decode without workspace ----
@@ -385,6 +401,116 @@ int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_
       km, vm, P);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_partial_kernel launch");
+  spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, (cudaStream_t)stream>>>(
+      (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_combine_kernel launch");
+}
+
+long long spark_kv_cache_q8_bytes(const spark_layer_cfg* cfg, int B, long long cap) {
+  if (check_cfg(cfg) != SPARK_OK || B <= 0 || cap <= 0) return -1;
+  return 2LL * B * cfg->n_kv * cap * (cfg->head_dim + 2LL * (cfg->head_dim / 32));
+}
+
+int spark_kv_append_q8(void* k_codes, void* k_scales, void* v_codes, void* v_scales, int cap,
+                       const void* k, const void* v, int B, int T, const int* pos0,
+                       const spark_layer_cfg* cfg, unsigned flags, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!k_codes || !k_scales || !v_codes || !v_scales || !k || !v || !pos0)
+    return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B > 65535 || T <= 0 || T > SPARK_MAX_POSITION || cap <= 0)
+    return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d cap=%d", B, T, cap);
+  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
+  if (!sliding && cap > SPARK_MAX_POSITION) return fail(SPARK_ERR_INVALID_ARG, "cap above 2^20");
+  if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(k_scales) || !aligned16(v_scales) ||
+      !aligned16(k) || !aligned16(v))
+    return fail(SPARK_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  const int t_first = sliding && T > SPARK_WINDOW ? T - SPARK_WINDOW : 0;
+  dim3 grid(T - t_first, B);
+  spark::kv_append_q8_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
+      (uint8_t*)k_codes, (__half*)k_scales, (uint8_t*)v_codes, (__half*)v_scales, cap,
+      (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, B, T, t_first, pos0, sliding,
+      (flags & SPARK_ROPE_FUSED) ? 1 : 0, log2(cfg->theta), cfg->rot_dim);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "kv_append_q8_kernel launch");
+}
+
+size_t spark_decode_q8_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg) {
+  if (check_cfg(cfg) != SPARK_OK || B <= 0 || cap <= 0) return 0;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  return decode_ws_bytes(B, decode_q8_plan(B, sliding ? SPARK_WINDOW : cap, sliding, sms > 0 ? sms : 148));
+}
+
+int spark_attn_decode_q8(void* out, const void* q, const void* gate, const void* k_codes,
+                         const void* k_scales, const void* v_codes, const void* v_scales, int cap,
+                         int B, const int* pos, const spark_layer_cfg* cfg, void* workspace,
+                         size_t ws_bytes, unsigned flags, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!out || !q || !gate || !k_codes || !k_scales || !v_codes || !v_scales || !pos || !workspace)
+    return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B > 65535 || cap <= 0) return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d cap=%d", B, cap);
+  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
+  if (!sliding && cap > SPARK_MAX_POSITION) return fail(SPARK_ERR_INVALID_ARG, "cap above 2^20");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(k_scales) ||
+      !aligned16(v_scales) || !aligned16(workspace))
+    return fail(SPARK_ERR_INVALID_ARG, "tensors and workspace must be 16-byte aligned");
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  const DecodePlan pl = decode_q8_plan(B, cap, sliding, g_dev[dev].sm_count);
+  if (ws_bytes < decode_ws_bytes(B, pl))
+    return fail(SPARK_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu needed", ws_bytes,
+                decode_ws_bytes(B, pl));
+
+  // codes [B*4][cap][256] u8 in two 128-byte swizzled boxes per row; scales [B*4][cap][8] fp16
+  CUtensorMap kcm, ksm, vcm, vsm;
+  const cuuint64_t cdims[3] = {256, (cuuint64_t)cap, (cuuint64_t)B * 4};
+  const cuuint64_t cstr[2] = {256, (cuuint64_t)cap * 256};
+  const cuuint32_t cbox[3] = {128, (cuuint32_t)spark::kQ8NK, 1};
+  const cuuint64_t sdims[3] = {8, (cuuint64_t)cap, (cuuint64_t)B * 4};
+  const cuuint64_t sstr[2] = {16, (cuuint64_t)cap * 16};
+  const cuuint32_t sbox[3] = {8, (cuuint32_t)spark::kQ8NK, 1};
+  if ((rc = make_map_t(&kcm, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_128B, k_codes, 3, cdims, cstr,
+                       cbox)))
+    return rc;
+  if ((rc = make_map_t(&vcm, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_128B, v_codes, 3, cdims, cstr,
+                       cbox)))
+    return rc;
+  if ((rc = make_map_t(&ksm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE, k_scales, 3, sdims,
+                       sstr, sbox)))
+    return rc;
+  if ((rc = make_map_t(&vsm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE, v_scales, 3, sdims,
+                       sstr, sbox)))
+    return rc;
+
+  spark::DecodeParams P;
+  P.q = (const __nv_bfloat16*)q;
+  P.pos = pos;
+  P.o_part = (float*)workspace;
+  P.ml_part = (float*)workspace + (size_t)B * spark::kNq * pl.n_splits * spark::kHeadDim;
+  P.B = B;
+  P.cap = cap;
+  P.sliding = sliding;
+  P.n_splits = pl.n_splits;
+  P.tiles_per_split = pl.tiles_per_split;
+  P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
+  P.rot = cfg->rot_dim;
+  P.log2_theta = log2(cfg->theta);
+  P.timeout_ns = wait_timeout_ns();
+  dim3 grid(pl.n_splits, spark::kNkv, B);
+  spark::decode_q8_partial_kernel<<<grid, spark::kQ8Threads, spark::kQ8SmemBytes, (cudaStream_t)stream>>>(
+      kcm, ksm, vcm, vsm, P);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode_q8_partial_kernel launch");
   spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, (cudaStream_t)stream>>>(
       (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
   e = cudaGetLastError();

@@ -22,8 +22,9 @@
  * (x_i, x_{i+rot/2}) turns by angle pos * theta^(-2i/rot).
  *
  * Conventions shared by every call:
- *   - All tensors are bf16, contiguous, in device memory, allocated and owned
- *     by the caller.  The library allocates and frees nothing.
+ *   - All tensors are bf16 (the q8 cache: uint8 codes and fp16 scales),
+ *     contiguous, in device memory, allocated and owned by the caller.  The
+ *     library allocates and frees nothing.
  *   - Positions are absolute (0 <= pos < 2^20).  Per-sequence positions live
  *     in caller-owned device int32 arrays, so a captured CUDA graph can replay
  *     with new positions.
@@ -181,6 +182,43 @@ int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_
 int spark_attn_decode_static(void* out, const void* q, const void* gate, const void* k_cache,
                              const void* v_cache, int cap, int B, const int* pos,
                              const spark_layer_cfg* cfg, unsigned flags, void* stream);
+
+/* ---- 8-bit block-quantised KV cache ("Sharp-Spark-X2.5-4B-GGUF" page §四:
+ * the K/V cache stored as q8_0, 36 -> 19 KB per token).  The block format is
+ * GGML's q8_0, which the page names but does not spell out: 32 consecutive
+ * values of a row share one fp16 scale, each value is an 8-bit code.
+ *   k_codes, v_codes    uint8 [B][4][cap][256]  byte = c + 128, c in [-127, 127]
+ *   k_scales, v_scales  fp16  [B][4][cap][8]    value ~ c * scale of its block
+ * Rows are placed as in the bf16 cache (ring of 512 for sliding layers).
+ * Quantising a block (float32): amax = max |x|; scale = fp16(amax / 127);
+ * c = x * (127 / amax) rounded half away from zero (IEEE single division and
+ * product); an all-zero block, or one where 127 / amax overflows, gives c = 0,
+ * scale 0.  Values are representable up to |x| = 127 * 65504 (fp16 scale).  Buffers are caller-owned
+ * device memory: codes 16-byte aligned, scales 16-byte aligned. */
+
+/* Bytes of one layer's q8 K and V caches (codes and scales), -1 on bad input. */
+long long spark_kv_cache_q8_bytes(const spark_layer_cfg* cfg, int B, long long cap);
+
+/* Quantise and append T new tokens per sequence (same positions, ring and
+ * checks as spark_kv_append; k/v [B][T][4][256] bf16, not modified).  With
+ * SPARK_ROPE_FUSED, k is rotated (and rounded to bf16) before quantisation. */
+int spark_kv_append_q8(void* k_codes, void* k_scales, void* v_codes, void* v_scales, int cap,
+                       const void* k, const void* v, int B, int T, const int* pos0,
+                       const spark_layer_cfg* cfg, unsigned flags, void* stream);
+
+/* Workspace bytes spark_attn_decode_q8 needs (0 on bad arguments). */
+size_t spark_decode_q8_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg);
+
+/* spark_attn_decode over a q8 cache: same arguments, positions, visibility
+ * and output as spark_attn_decode, with each cache given as codes + scales.
+ * The products use q and the probabilities in fp16 (q keeps its bf16 value
+ * exactly; a row with |q|/16 >= 2^15 is first scaled by a power of two) and
+ * accumulate in fp32.  Rows past the last visible key are never used, so
+ * they may hold anything. */
+int spark_attn_decode_q8(void* out, const void* q, const void* gate, const void* k_codes,
+                         const void* k_scales, const void* v_codes, const void* v_scales, int cap,
+                         int B, const int* pos, const spark_layer_cfg* cfg, void* workspace,
+                         size_t ws_bytes, unsigned flags, void* stream);
 
 /* Self-test of the failure-detection path: launches one block that waits,
  * with the same bounded wait every kernel of the library uses, on a barrier

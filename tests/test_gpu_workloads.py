@@ -108,6 +108,41 @@ def test_decode_sampled(B, p, layer_ids, check_b, groups):
     torch.cuda.empty_cache()
 
 
+def test_decode_q8_b64_ctx32768_sampled():
+    """The 8-bit-cache decode step in the launch configuration bench.py times (one sliding and one
+    full layer), sampled sequences and groups against the oracle over its own quantised history."""
+    dev = torch.device("cuda")
+    B, p = bench.DECODE_B, bench.DECODE_CTX
+    layers = bench.decode_q8_layers(torch, sa, synth, dev, B, p, (0, 3))
+    pos = torch.full((B,), p, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(sa.spark_decode_q8_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers),
+                     dtype=torch.uint8, device=dev)
+    bench.decode_q8_step(sa, layers, pos, ws)
+    sa.spark_check()
+    seed = bench.DECODE_SEED
+    for L in layers:
+        kind, layer = L["kind"], L["layer"]
+        got = dev_to_f64(L["out"])
+        hist = np.arange(max(0, p - 511) if kind == O.SLIDING else 0, p)
+        for b in (0, 63):
+            qb = f64(synth.token_tensor(seed, tid(layer, synth.ROLE_Q), B, 16, 256, np.full((B, 1), p))[b, 0])
+            gb = f64(synth.token_tensor(seed, tid(layer, synth.ROLE_GATE), B, 16, 1, np.full((B, 1), p))[b, 0])
+            for g in (0, 3):
+                hs = slice(4 * g, 4 * g + 4)
+                hk, hv = _group_kv(seed, layer, b, g, hist)
+                kn, vn = _group_kv(seed, layer, b, g, np.array([p]))
+                keys = np.concatenate([hk, _rope1(kn, np.array([p]), kind)]).astype(np.float32)
+                vals = np.concatenate([hv, vn]).astype(np.float32)
+                keys = O.dequantize_q8(*O.quantize_q8(keys))
+                vals = O.dequantize_q8(*O.quantize_q8(vals))
+                kpos = np.concatenate([hist, [p]])
+                q = O.rope(qb[None, hs], np.array([p]), kind)
+                ref = O.attention_group(q, keys, vals, gb[None, hs], np.array([p]), kpos, kind)[0]
+                assert_close(got[b, hs], ref, f"q8 decode B={B} p={p} layer={layer} b={b} group={g}")
+    del layers, ws
+    torch.cuda.empty_cache()
+
+
 # ------------------------------------ long prefill, 8192-token chunks ------
 
 def test_long_prefill_chunked_sampled_rows():
