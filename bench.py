@@ -317,6 +317,18 @@ def decode_layers(torch, sa, synth, dev, B: int, p: int, layer_ids=range(N_LAYER
     return layers
 
 
+def decode_launches(sa, B: int, layers, q8: bool = False) -> int:
+    """Kernels one decode step launches: per layer the append and the split kernel, plus the
+    combine kernel where the split plan has more than one split (read back from the workspace size,
+    B * 16 * splits * 258 fp32)."""
+    n = 0
+    for L in layers:
+        fn = sa.spark_decode_q8_workspace_bytes if q8 else sa.spark_decode_workspace_bytes
+        splits = fn(B, L["cap"], L["cfg"]) // (B * HQ * (D + 2) * 4)
+        n += 2 + (1 if splits > 1 else 0)
+    return n
+
+
 def decode_step(sa, layers, pos, ws):
     """One decode step: per layer, append the new token (RoPE fused on k), then attend (RoPE fused on q)."""
     for L in layers:
@@ -366,12 +378,13 @@ def run_decode(torch, sa, synth, dist, args, peaks, world):
     k_ms = e0.elapsed_time(e1) / reps
     total_bytes = sum(decode_kv_bytes(B, p, L["kind"]) for L in layers)
     full_bytes = decode_kv_bytes(B, p, FULL)
+    launches = decode_launches(sa, B, layers)
     del graph, layers, ws
     torch.cuda.empty_cache()
     return {
         "value": total_bytes * world / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
         "ms_per_step": ms_step, "steps_per_s": 1e3 / ms_step, "kv_bytes_per_step": total_bytes,
-        "workload": f"decode_b{B}_ctx{p}_36layers", "gpu_launches_per_step": 3 * N_LAYERS,
+        "workload": f"decode_b{B}_ctx{p}_36layers", "gpu_launches_per_step": launches,
         "roofline": {"bound": "hbm", "kernel": "decode_partial_kernel+combine (full layer)",
                      "achieved": full_bytes / (k_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": full_bytes / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
@@ -459,12 +472,13 @@ def run_decode_q8(torch, sa, synth, dist, args, peaks, world):
     k_ms = e0.elapsed_time(e1) / reps
     total_bytes = sum(decode_q8_kv_bytes(B, p, L["kind"]) for L in layers)
     full_bytes = decode_q8_kv_bytes(B, p, FULL)
+    launches = decode_launches(sa, B, layers, q8=True)
     del graph, layers, ws
     torch.cuda.empty_cache()
     return {
         "value": total_bytes * world / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
         "ms_per_step": ms_step, "steps_per_s": 1e3 / ms_step, "kv_bytes_per_step": total_bytes,
-        "workload": f"decode_q8_b{B}_ctx{p}_36layers", "gpu_launches_per_step": 3 * N_LAYERS,
+        "workload": f"decode_q8_b{B}_ctx{p}_36layers", "gpu_launches_per_step": launches,
         "roofline": {"bound": "hbm", "kernel": "decode_q8_partial_kernel+combine (full layer)",
                      "achieved": full_bytes / (k_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": full_bytes / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],

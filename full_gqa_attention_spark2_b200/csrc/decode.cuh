@@ -39,11 +39,20 @@ struct DecodeParams {
   const int* pos;             // [B]
   float* o_part;              // [B][16][splits][256]
   float* ml_part;             // [B][16][splits][2]
+  __nv_bfloat16* out;         // [B][16][256], written here when n_splits == 1
+  const __nv_bfloat16* gate;  // [B][16]
   int B, cap, sliding, n_splits, tiles_per_split;
   int rope, rot;
   double log2_theta;
   unsigned long long timeout_ns;
 };
+
+// Factor of the merged numerator: 1 / (softmax denominator) times the
+// sigmoid of the head's gate logit; 0 for a row that saw no key.
+__device__ __forceinline__ float decode_out_scale(float l, __nv_bfloat16 gate_logit) {
+  const float gl = __bfloat162float(gate_logit);
+  return (l > 0.f) ? (1.f / l) * (1.f / (1.f + expf(-gl))) : 0.f;
+}
 
 __device__ __forceinline__ uint32_t swz_addr(uint32_t tile, int key, int dim) {
   // byte address of (key, dim) in a tile of four [64 keys x 128 B] boxes, 128 B swizzle
@@ -287,6 +296,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       ls += ew[w] * sm_l[w * 4 + hh];
     }
     const long long row = ((long long)b * kNq + g * 4 + hh) * P.n_splits + split;
+    if (P.n_splits == 1) {
+      // a single split is the whole answer: normalise, gate and store it here
+      const float scale = decode_out_scale(ls, P.gate[(long long)b * kNq + g * 4 + hh]);
+      __nv_bfloat16* dst = P.out + ((long long)b * kNq + g * 4 + hh) * kHeadDim;
+      for (int d = (tid & 31); d < kHeadDim; d += 32) {
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecConsumerWarps; ++w) acc += ew[w] * mrg_o[(w * 4 + hh) * kHeadDim + d];
+        dst[d] = __float2bfloat16_rn(acc * scale);
+      }
+      return;
+    }
     float* dst = P.o_part + row * kHeadDim;
     for (int d = (tid & 31); d < kHeadDim; d += 32) {
       float acc = 0.f;
@@ -323,8 +344,7 @@ __global__ void __launch_bounds__(64) decode_combine_kernel(__nv_bfloat16* __res
     acc.z += e * v.z;
     acc.w += e * v.w;
   }
-  const float gl = __bfloat162float(gate[(long long)b * kNq + h]);
-  const float scale = (ls > 0.f) ? (1.f / ls) * (1.f / (1.f + expf(-gl))) : 0.f;
+  const float scale = decode_out_scale(ls, gate[(long long)b * kNq + h]);
   uint2 packed;
   packed.x = pack_bf16(acc.x * scale, acc.y * scale);
   packed.y = pack_bf16(acc.z * scale, acc.w * scale);

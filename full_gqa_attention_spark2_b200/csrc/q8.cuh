@@ -472,6 +472,18 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       ls += ew[w] * sm_l[w * 4 + hh];
     }
     const long long row = ((long long)b * kNq + g * 4 + hh) * P.n_splits + split;
+    if (P.n_splits == 1) {
+      // a single split is the whole answer: normalise, gate and store it here
+      const float scale = decode_out_scale(ls, P.gate[(long long)b * kNq + g * 4 + hh]);
+      __nv_bfloat16* dst = P.out + ((long long)b * kNq + g * 4 + hh) * kHeadDim;
+      for (int d = (tid & 63); d < kHeadDim; d += 64) {
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kQ8ConsumerWarps; ++w) acc += ew[w] * mrg_o[(w * 4 + hh) * kHeadDim + d];
+        dst[d] = __float2bfloat16_rn(acc * scale);
+      }
+      return;
+    }
     float* dst = P.o_part + row * kHeadDim;
     for (int d = (tid & 63); d < kHeadDim; d += 64) {
       float acc = 0.f;

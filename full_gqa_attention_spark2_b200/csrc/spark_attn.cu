@@ -396,11 +396,14 @@ int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_
   P.rot = cfg->rot_dim;
   P.log2_theta = log2(cfg->theta);
   P.timeout_ns = wait_timeout_ns();
+  P.out = (__nv_bfloat16*)out;
+  P.gate = (const __nv_bfloat16*)gate;
   dim3 grid(pl.n_splits, spark::kNkv, B);
   spark::decode_partial_kernel<<<grid, spark::kDecThreads, spark::kDecSmemBytes, (cudaStream_t)stream>>>(
       km, vm, P);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_partial_kernel launch");
+  if (pl.n_splits == 1) return SPARK_OK;      // the partial kernel wrote the output itself
   spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, (cudaStream_t)stream>>>(
       (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
   e = cudaGetLastError();
@@ -506,11 +509,14 @@ int spark_attn_decode_q8(void* out, const void* q, const void* gate, const void*
   P.rot = cfg->rot_dim;
   P.log2_theta = log2(cfg->theta);
   P.timeout_ns = wait_timeout_ns();
+  P.out = (__nv_bfloat16*)out;
+  P.gate = (const __nv_bfloat16*)gate;
   dim3 grid(pl.n_splits, spark::kNkv, B);
   spark::decode_q8_partial_kernel<<<grid, spark::kQ8Threads, spark::kQ8SmemBytes, (cudaStream_t)stream>>>(
       kcm, ksm, vcm, vsm, P);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_q8_partial_kernel launch");
+  if (pl.n_splits == 1) return SPARK_OK;      // the partial kernel wrote the output itself
   spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, (cudaStream_t)stream>>>(
       (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
   e = cudaGetLastError();
@@ -643,10 +649,13 @@ int spark_attn_decode_static(void* out, const void* q, const void* gate, const v
   P.rot = cfg->rot_dim;
   P.log2_theta = log2(cfg->theta);
   P.timeout_ns = wait_timeout_ns();
+  P.out = (__nv_bfloat16*)out;
+  P.gate = (const __nv_bfloat16*)gate;
   spark::decode_partial_kernel<<<dim3(pl.n_splits, spark::kNkv, B), spark::kDecThreads, spark::kDecSmemBytes,
                                  (cudaStream_t)stream>>>(km, vm, P);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_partial_kernel launch");
+  if (pl.n_splits == 1) return SPARK_OK;      // the partial kernel wrote the output itself
   spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, (cudaStream_t)stream>>>(
       (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
   e = cudaGetLastError();

@@ -151,7 +151,9 @@ size_t spark_decode_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg);
  *   then hold exactly positions max(0, pos[b] - 511)..pos[b].
  *   workspace: caller-owned device scratch of at least
  *   spark_decode_workspace_bytes(B, cap, cfg) bytes, 16-byte aligned; calls
- *   that share a workspace must not overlap on the device. */
+ *   that share a workspace must not overlap on the device.  When the split
+ *   plan has one split per (sequence, KV head), as for sliding layers at
+ *   B >= 37, one kernel writes `out` directly and the workspace is unused. */
 int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_cache,
                       const void* v_cache, int cap, int B, const int* pos,
                       const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
