@@ -43,6 +43,12 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int
 
 
+class SparkPagedKV(ctypes.Structure):
+    """spark_paged_kv of include/spark_attn.h; keeps the tensors it points to alive."""
+    _fields_ = [("k", _P), ("v", _P), ("k_scales", _P), ("v_scales", _P), ("block_table", _P),
+                ("page_size", _I), ("n_pages", _I), ("max_pages", _I)]
+
+
 def lib_path() -> str:
     return os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspark_attn.so")
 
@@ -72,6 +78,10 @@ def _lib():
         "spark_decode_q8_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
         "spark_attn_decode_q8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _P, cfgp, _P, ctypes.c_size_t,
                                       ctypes.c_uint, _P]),
+        "spark_kv_append_paged": (_I, [ctypes.POINTER(SparkPagedKV), _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
+        "spark_decode_paged_workspace_bytes": (ctypes.c_size_t, [_I, ctypes.POINTER(SparkPagedKV), cfgp]),
+        "spark_attn_decode_paged": (_I, [_P, _P, _P, ctypes.POINTER(SparkPagedKV), _I, _P, cfgp, _P,
+                                         ctypes.c_size_t, ctypes.c_uint, _P]),
         "spark_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
         "spark_check": (_I, [_P]),
         "spark_last_error": (ctypes.c_char_p, []),
@@ -91,7 +101,8 @@ def exported_symbols():
             "spark_stack_kv_bytes", "spark_rope_apply", "spark_kv_append", "spark_attn_prefill",
             "spark_decode_workspace_bytes", "spark_attn_decode", "spark_attn_decode_static",
             "spark_kv_cache_q8_bytes", "spark_kv_append_q8", "spark_decode_q8_workspace_bytes",
-            "spark_attn_decode_q8", "spark_selftest_wait_timeout", "spark_check", "spark_last_error",
+            "spark_attn_decode_q8", "spark_kv_append_paged", "spark_decode_paged_workspace_bytes",
+            "spark_attn_decode_paged", "spark_selftest_wait_timeout", "spark_check", "spark_last_error",
             "spark_version"]
 
 
@@ -258,6 +269,48 @@ def spark_attn_decode_q8(out, q, gate, k_codes, k_scales, v_codes, v_scales, pos
     _raise(_lib().spark_attn_decode_q8(po, pq, pg, pkc, pks, pvc, pvs, k_codes.shape[2], q.shape[0], pp,
                                        ctypes.byref(cfg), workspace.data_ptr(), ws_bytes, flags,
                                        _stream(stream)))
+
+
+def paged_kv(k_pool, v_pool, block_table, k_scales=None, v_scales=None) -> SparkPagedKV:
+    """Describe one layer's paged K/V: pools [n_pages, 4, page_size, 256] (bf16, or uint8 codes with
+    float16 scales [n_pages, 4, page_size, 8]) and block_table int32 [B, max_pages]."""
+    q8 = k_scales is not None
+    dt = torch.uint8 if q8 else torch.bfloat16
+    pk, pv = _dev(k_pool, "k_pool", dt, 4), _dev(v_pool, "v_pool", dt, 4)
+    pt = _dev(block_table, "block_table", torch.int32, 2)
+    if tuple(v_pool.shape) != tuple(k_pool.shape) or k_pool.shape[1] != 4 or k_pool.shape[3] != 256:
+        raise ValueError("pools must be [n_pages, 4, page_size, 256]")
+    pks = pvs = None
+    if q8:
+        pks, pvs = _q8_pair(k_pool, k_scales, "k")[1], _q8_pair(v_pool, v_scales, "v")[1]
+    kv = SparkPagedKV(pk, pv, pks, pvs, pt, k_pool.shape[2], k_pool.shape[0], block_table.shape[1])
+    kv._keep = (k_pool, v_pool, block_table, k_scales, v_scales)
+    return kv
+
+
+def spark_kv_append_paged(kv: SparkPagedKV, k, v, pos0, cfg: SparkLayerCfg, flags: int = 0, stream=None) -> None:
+    """Append k, v [B, T, 4, 256] at positions pos0[b] + t into a paged pool (quantised if it is 8-bit)."""
+    pk, pv = _dev(k, "k", ndim=4), _dev(v, "v", ndim=4)
+    pp = _dev(pos0, "pos0", torch.int32, 1)
+    _raise(_lib().spark_kv_append_paged(ctypes.byref(kv), pk, pv, k.shape[0], k.shape[1], pp, ctypes.byref(cfg),
+                                        flags, _stream(stream)))
+
+
+def spark_decode_paged_workspace_bytes(B: int, kv: SparkPagedKV, cfg: SparkLayerCfg) -> int:
+    return int(_lib().spark_decode_paged_workspace_bytes(B, ctypes.byref(kv), ctypes.byref(cfg)))
+
+
+def spark_attn_decode_paged(out, q, gate, kv: SparkPagedKV, pos, cfg: SparkLayerCfg, workspace: torch.Tensor,
+                            flags: int = 0, stream=None) -> None:
+    """spark_attn_decode over a paged pool."""
+    po, pq = _dev(out, "out", ndim=3), _dev(q, "q", ndim=3)
+    pg = _dev(gate, "gate", ndim=2)
+    pp = _dev(pos, "pos", torch.int32, 1)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _raise(_lib().spark_attn_decode_paged(po, pq, pg, ctypes.byref(kv), q.shape[0], pp, ctypes.byref(cfg),
+                                          workspace.data_ptr(), ws_bytes, flags, _stream(stream)))
 
 
 def spark_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:

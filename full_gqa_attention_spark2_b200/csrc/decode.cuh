@@ -45,7 +45,36 @@ struct DecodeParams {
   int rope, rot;
   double log2_theta;
   unsigned long long timeout_ns;
+  // paged caches only: pool [n_pages][4][page][256]; logical row r of sequence b
+  // lives in page block_table[b * max_pages + r / page] at row r % page
+  const int* block_table;
+  int max_pages, page_shift, n_pages;
 };
+
+// TMA coordinates of the 64 keys that start at logical row `row0` of
+// (sequence b, KV head g): a dense cache is 3-D (dim, row, b * 4 + g), a paged
+// pool 4-D (dim, row in page, head, page).  `ok` is false for a page index
+// outside the pool.
+struct KvTile {
+  int c1, c2, c3;
+  bool ok;
+};
+
+template <bool kPaged>
+__device__ __forceinline__ KvTile kv_tile(const DecodeParams& P, int b, int g, int row0) {
+  if (!kPaged) return KvTile{row0, b * kNkv + g, 0, true};
+  const int pg = P.block_table[(long long)b * P.max_pages + (row0 >> P.page_shift)];
+  return KvTile{row0 & ((1 << P.page_shift) - 1), g, pg, pg >= 0 && pg < P.n_pages};
+}
+
+template <bool kPaged>
+__device__ __forceinline__ void kv_tile_load(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x,
+                                             const KvTile& t) {
+  if (kPaged)
+    tma_load_4d(dst, map, bar, x, t.c1, t.c2, t.c3);
+  else
+    tma_load_3d(dst, map, bar, x, t.c1, t.c2);
+}
 
 // Factor of the merged numerator: 1 / (softmax denominator) times the
 // sigmoid of the head's gate logit; 0 for a row that saw no key.
@@ -60,6 +89,7 @@ __device__ __forceinline__ uint32_t swz_addr(uint32_t tile, int key, int dim) {
          ((uint32_t)(((dim & 63) >> 3) ^ (key & 7)) << 4);
 }
 
+template <bool kPaged>
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_partial_kernel(const __grid_constant__ CUtensorMap kmap,
                           const __grid_constant__ CUtensorMap vmap, const DecodeParams P) {
@@ -103,21 +133,25 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (lane == 0 && n_tiles > 0) {
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      const int plane = b * kNkv + g;
       int issued = 0;
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % kDecStages;
         if (i >= kDecStages &&
             !mbar_wait(bar_empty + 8 * s, ((i / kDecStages) - 1) & 1, abort_flag, P.timeout_ns, 0x10u))
           break;
+        const KvTile t = kv_tile<kPaged>(P, b, g, key_begin + i * kDecNK);
+        if (!t.ok) {                       // a page index outside the pool: flag it, stop the block
+          raise_error(kErrPosition, 0x600u | (unsigned)b);
+          *abort_flag = 1;
+          break;
+        }
         const uint32_t full = bar_full + 8 * s;
         mbar_arrive_expect_tx(full, kDecStageBytes);
         const uint32_t kt = base + s * kDecStageBytes;
-        const int row0 = key_begin + i * kDecNK;
 #pragma unroll
         for (int d = 0; d < 4; ++d) {
-          tma_load_3d(kt + d * kDecBoxBytes, &kmap, full, d * 64, row0, plane);
-          tma_load_3d(kt + kDecTileBytes + d * kDecBoxBytes, &vmap, full, d * 64, row0, plane);
+          kv_tile_load<kPaged>(kt + d * kDecBoxBytes, &kmap, full, d * 64, t);
+          kv_tile_load<kPaged>(kt + kDecTileBytes + d * kDecBoxBytes, &vmap, full, d * 64, t);
         }
         issued = i + 1;
       }

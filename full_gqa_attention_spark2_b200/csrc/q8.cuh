@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
     uint8_t* __restrict__ k_codes, __half* __restrict__ k_scales, uint8_t* __restrict__ v_codes,
     __half* __restrict__ v_scales, int cap, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, int B, int T, int t_first, const int* __restrict__ pos0, int sliding,
-    int rope, double log2_theta, int rot) {
+    int rope, double log2_theta, int rot, CachePages pages) {
   __shared__ float xs[2][kNkv * kHeadDim + kNkv * kHeadDim / 32];
   const int t = t_first + blockIdx.x;
   const int b = blockIdx.y;
@@ -136,8 +136,12 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
     w[e >> 2] |= u << (8 * (e & 3));
   }
   const int h = hb >> 3, bl = hb & 7;
-  const long long row = sliding ? (pos & (kWindow - 1)) : pos;
-  const long long crow = ((long long)b * kNkv + h) * cap + row;
+  const int row = sliding ? (pos & (kWindow - 1)) : pos;
+  const long long crow = cache_row(pages, b, h, cap, row);
+  if (crow < 0) {                        // a page index outside the pool
+    if (tid == 0) raise_error(kErrPosition, 0x800u | (unsigned)b);
+    return;
+  }
   uint8_t* codes = which ? v_codes : k_codes;
   *reinterpret_cast<uint4*>(codes + crow * kHeadDim + bl * kQ8Block + hf * 16) = make_uint4(w[0], w[1], w[2], w[3]);
   if (hf == 0) (which ? v_scales : k_scales)[crow * 8 + bl] = __float2half_rn(__fdiv_rn(amax, 127.f));
@@ -187,6 +191,7 @@ __device__ __forceinline__ uint32_t q8_pair(uint32_t bytes, uint32_t sel) {
   return hsub2_u32(prmt(bytes, kQ8Magic, sel), kQ8Bias);
 }
 
+template <bool kPaged>
 __global__ void __launch_bounds__(kQ8Threads, 1)
     decode_q8_partial_kernel(const __grid_constant__ CUtensorMap kcmap, const __grid_constant__ CUtensorMap ksmap,
                              const __grid_constant__ CUtensorMap vcmap, const __grid_constant__ CUtensorMap vsmap,
@@ -235,23 +240,27 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       tma_prefetch_desc(&ksmap);
       tma_prefetch_desc(&vcmap);
       tma_prefetch_desc(&vsmap);
-      const int plane = b * kNkv + g;
       int issued = 0;
       for (int i = 0; i < n_tiles; ++i) {
         const int s = i % kQ8Stages;
         if (i >= kQ8Stages &&
             !mbar_wait(bar_empty + 8 * s, ((i / kQ8Stages) - 1) & 1, abort_flag, P.timeout_ns, 0x20u))
           break;
+        const KvTile t = kv_tile<kPaged>(P, b, g, key_begin + i * kQ8NK);
+        if (!t.ok) {                       // a page index outside the pool: flag it, stop the block
+          raise_error(kErrPosition, 0x700u | (unsigned)b);
+          *abort_flag = 1;
+          break;
+        }
         const uint32_t full = bar_full + 8 * s;
         mbar_arrive_expect_tx(full, kQ8StageBytes);
         const uint32_t st = base + s * kQ8StageBytes;
-        const int row0 = key_begin + i * kQ8NK;
-        tma_load_3d(st, &kcmap, full, 0, row0, plane);
-        tma_load_3d(st + kQ8CodeBox, &kcmap, full, 128, row0, plane);
-        tma_load_3d(st + kQ8CodeTile, &vcmap, full, 0, row0, plane);
-        tma_load_3d(st + kQ8CodeTile + kQ8CodeBox, &vcmap, full, 128, row0, plane);
-        tma_load_3d(st + 2 * kQ8CodeTile, &ksmap, full, 0, row0, plane);
-        tma_load_3d(st + 2 * kQ8CodeTile + kQ8ScaleTile, &vsmap, full, 0, row0, plane);
+        kv_tile_load<kPaged>(st, &kcmap, full, 0, t);
+        kv_tile_load<kPaged>(st + kQ8CodeBox, &kcmap, full, 128, t);
+        kv_tile_load<kPaged>(st + kQ8CodeTile, &vcmap, full, 0, t);
+        kv_tile_load<kPaged>(st + kQ8CodeTile + kQ8CodeBox, &vcmap, full, 128, t);
+        kv_tile_load<kPaged>(st + 2 * kQ8CodeTile, &ksmap, full, 0, t);
+        kv_tile_load<kPaged>(st + 2 * kQ8CodeTile + kQ8ScaleTile, &vsmap, full, 0, t);
         issued = i + 1;
       }
       for (int i = max(0, issued - kQ8Stages); i < issued; ++i)

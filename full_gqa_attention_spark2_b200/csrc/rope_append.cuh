@@ -66,13 +66,31 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
   }
 }
 
+// Where a cache row lives.  Dense caches: [B][4][cap][256].  Paged pools:
+// [n_pages][4][page][256], logical row r of sequence b in page
+// table[b * max_pages + r / page] at row r % page (table == nullptr: dense).
+struct CachePages {
+  const int* table;
+  int max_pages, page_shift, n_pages;
+};
+
+// Index of the 256-element row holding (sequence b, KV head h, logical row),
+// or -1 when the page index is outside the pool.
+__device__ __forceinline__ long long cache_row(const CachePages& pg, int b, int h, int cap, int row) {
+  if (pg.table == nullptr) return ((long long)b * kNkv + h) * cap + row;
+  const int page = pg.table[(long long)b * pg.max_pages + (row >> pg.page_shift)];
+  if (page < 0 || page >= pg.n_pages) return -1;
+  return ((long long)page * kNkv + h) * (1 << pg.page_shift) + (row & ((1 << pg.page_shift) - 1));
+}
+
 // Append k/v [B][T][4][256] of T new tokens into caches [B][4][cap][256].
 // One block per written token, thread = (head, 16-byte chunk of 8 dims).
 // Sliding layers (ring of 512 rows) only write the last min(T, 512) tokens.
 __global__ void __launch_bounds__(128) kv_append_kernel(
     __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache, int cap,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int B, int T,
-    int t_first, const int* __restrict__ pos0, int sliding, int rope, double log2_theta, int rot) {
+    int t_first, const int* __restrict__ pos0, int sliding, int rope, double log2_theta, int rot,
+    CachePages pages) {
   const int t = t_first + blockIdx.x;
   const int b = blockIdx.y;
   const int h = threadIdx.x >> 5;
@@ -84,9 +102,14 @@ __global__ void __launch_bounds__(128) kv_append_kernel(
     return;
   }
   const int pos = p0 + t;
-  const long long row = sliding ? (pos & (kWindow - 1)) : pos;
+  const int row = sliding ? (pos & (kWindow - 1)) : pos;
   const long long src = (((long long)b * T + t) * kNkv + h) * kHeadDim;
-  const long long dst = (((long long)b * kNkv + h) * cap + row) * kHeadDim;
+  const long long crow = cache_row(pages, b, h, cap, row);
+  if (crow < 0) {                        // a page index outside the pool
+    if (ch == 0) raise_error(kErrPosition, 0x900u | (unsigned)b);
+    return;
+  }
+  const long long dst = crow * kHeadDim;
 
   const uint4* vs = reinterpret_cast<const uint4*>(v + src);
   reinterpret_cast<uint4*>(v_cache + dst)[ch] = vs[ch];

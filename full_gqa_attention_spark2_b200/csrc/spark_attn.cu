@@ -80,15 +80,21 @@ int device_ready(int* dev_out) {
       return;
     }
     d.sm_count = sms > 0 ? sms : 148;
-    cudaError_t a = cudaFuncSetAttribute(spark::decode_partial_kernel,
+    cudaError_t a = cudaFuncSetAttribute(spark::decode_partial_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          spark::kDecSmemBytes);
+    if (a == cudaSuccess)
+      a = cudaFuncSetAttribute(spark::decode_partial_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               spark::kDecSmemBytes);
     cudaError_t b = cudaFuncSetAttribute(spark::prefill2_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          spark::kP2SmemBytes);
-    cudaError_t c = cudaFuncSetAttribute(spark::decode_q8_partial_kernel,
+    cudaError_t c = cudaFuncSetAttribute(spark::decode_q8_partial_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          spark::kQ8SmemBytes);
+    if (c == cudaSuccess)
+      c = cudaFuncSetAttribute(spark::decode_q8_partial_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               spark::kQ8SmemBytes);
     if (a != cudaSuccess || b != cudaSuccess || c != cudaSuccess) {
       snprintf(d.why, sizeof(d.why), "cudaFuncSetAttribute: %s",
                cudaGetErrorString(a != cudaSuccess ? a : b != cudaSuccess ? b : c));
@@ -215,6 +221,223 @@ DecodePlan decode_q8_plan(int B, int cap, int sliding, int sm_count) {
   return decode_plan(B, cap, sliding, sm_count);
 }
 
+// ------------------------------------------------------------ cache views ----
+// One layer's K/V storage as the kernels address it: dense [B][4][cap][256]
+// or a paged pool [n_pages][4][page][256]; bf16 values, or 8-bit codes with
+// fp16 scales ([...][8] per row) when ks/vs are set.
+struct CacheView {
+  void* k;
+  void* v;
+  void* ks;             // scales of the 8-bit K codes, nullptr for a bf16 cache
+  void* vs;
+  int cap;              // logical rows: dense capacity, 512 for a ring, max_pages * page when paged
+  int page;             // rows per page (paged), 0 for a dense cache
+  int n_pages;
+  int max_pages;
+  const int* table;     // paged: device int32 [B][max_pages]
+  bool q8() const { return ks != nullptr; }
+  bool paged() const { return page != 0; }
+};
+
+int ilog2(int x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return r;
+}
+
+spark::CachePages pages_of(const CacheView& c) {
+  if (!c.paged()) return spark::CachePages{nullptr, 0, 0, 0};
+  return spark::CachePages{c.table, c.max_pages, ilog2(c.page), c.n_pages};
+}
+
+CacheView dense_view(void* k, void* v, void* ks, void* vs, int cap) {
+  return CacheView{k, v, ks, vs, cap, 0, 0, 0, nullptr};
+}
+
+int paged_view(const spark_paged_kv* kv, const spark_layer_cfg* cfg, CacheView* out) {
+  if (!kv) return fail(SPARK_ERR_INVALID_ARG, "kv is NULL");
+  if (!kv->k || !kv->v || !kv->block_table) return fail(SPARK_ERR_INVALID_ARG, "null pointer in spark_paged_kv");
+  if ((kv->k_scales == nullptr) != (kv->v_scales == nullptr))
+    return fail(SPARK_ERR_INVALID_ARG, "pass both scale pools or neither");
+  const int P = kv->page_size;
+  if (P < 64 || P > 512 || (P & (P - 1)))
+    return fail(SPARK_ERR_INVALID_ARG, "page_size %d: a power of two from 64 to 512", P);
+  if (kv->n_pages <= 0 || kv->max_pages <= 0)
+    return fail(SPARK_ERR_INVALID_ARG, "n_pages %d, max_pages %d", kv->n_pages, kv->max_pages);
+  const long long rows = (long long)kv->max_pages * P;
+  int cap;
+  if (cfg->kind == SPARK_SLIDING) {
+    if (rows < SPARK_WINDOW)
+      return fail(SPARK_ERR_INVALID_ARG, "a sliding ring needs 512 rows: max_pages * page_size = %lld", rows);
+    cap = SPARK_WINDOW;
+  } else {
+    cap = (int)(rows < SPARK_MAX_POSITION ? rows : SPARK_MAX_POSITION);
+  }
+  *out = CacheView{kv->k, kv->v, kv->k_scales, kv->v_scales, cap, P, kv->n_pages, kv->max_pages,
+                   kv->block_table};
+  return SPARK_OK;
+}
+
+int check_view(const CacheView& c, const spark_layer_cfg* cfg) {
+  if (!c.k || !c.v) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (c.cap <= 0) return fail(SPARK_ERR_INVALID_ARG, "bad cap %d", c.cap);
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  if (sliding && c.cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
+  if (!sliding && c.cap > SPARK_MAX_POSITION) return fail(SPARK_ERR_INVALID_ARG, "cap above 2^20");
+  if (!aligned16(c.k) || !aligned16(c.v) || (c.q8() && (!aligned16(c.ks) || !aligned16(c.vs))))
+    return fail(SPARK_ERR_INVALID_ARG, "caches must be 16-byte aligned");
+  return SPARK_OK;
+}
+
+int append_impl(const CacheView& c, const void* k, const void* v, int B, int T, const int* pos0,
+                const spark_layer_cfg* cfg, unsigned flags, void* stream) {
+  int rc = check_view(c, cfg);
+  if (rc) return rc;
+  if (!k || !v || !pos0) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B > 65535 || T <= 0 || T > SPARK_MAX_POSITION)
+    return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d", B, T);
+  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (!aligned16(k) || !aligned16(v)) return fail(SPARK_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  const int t_first = sliding && T > SPARK_WINDOW ? T - SPARK_WINDOW : 0;
+  dim3 grid(T - t_first, B);
+  const int rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
+  if (c.q8()) {
+    spark::kv_append_q8_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
+        (uint8_t*)c.k, (__half*)c.ks, (uint8_t*)c.v, (__half*)c.vs, c.cap, (const __nv_bfloat16*)k,
+        (const __nv_bfloat16*)v, B, T, t_first, pos0, sliding, rope, log2(cfg->theta), cfg->rot_dim, pages_of(c));
+  } else {
+    spark::kv_append_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
+        (__nv_bfloat16*)c.k, (__nv_bfloat16*)c.v, c.cap, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, B, T,
+        t_first, pos0, sliding, rope, log2(cfg->theta), cfg->rot_dim, pages_of(c));
+  }
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, c.q8() ? "kv_append_q8_kernel launch" : "kv_append_kernel launch");
+}
+
+int current_sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+DecodePlan plan_for(int B, const CacheView& c, int sliding, int sms) {
+  return c.q8() ? decode_q8_plan(B, c.cap, sliding, sms) : decode_plan(B, c.cap, sliding, sms);
+}
+
+size_t decode_ws_for(int B, const CacheView& c, const spark_layer_cfg* cfg) {
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  return decode_ws_bytes(B, plan_for(B, c, sliding, current_sm_count()));
+}
+
+// Tensor maps of one cache for the decode kernels: K, V (bf16 or codes) and,
+// for 8-bit caches, the two scale arrays.
+int decode_maps(const CacheView& c, int B, CUtensorMap* km, CUtensorMap* vm, CUtensorMap* ksm, CUtensorMap* vsm) {
+  int rc;
+  const cuuint64_t row_bytes = c.q8() ? 256 : 512;
+  const CUtensorMapDataType dt = c.q8() ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const cuuint32_t box_x = c.q8() ? 128 : 64;              // 128 bytes per swizzled box row
+  if (!c.paged()) {
+    const cuuint64_t dims[3] = {256, (cuuint64_t)c.cap, (cuuint64_t)B * 4};
+    const cuuint64_t str[2] = {row_bytes, (cuuint64_t)c.cap * row_bytes};
+    const cuuint32_t box[3] = {box_x, 64, 1};
+    if ((rc = make_map_t(km, dt, CU_TENSOR_MAP_SWIZZLE_128B, c.k, 3, dims, str, box))) return rc;
+    if ((rc = make_map_t(vm, dt, CU_TENSOR_MAP_SWIZZLE_128B, c.v, 3, dims, str, box))) return rc;
+    if (c.q8()) {
+      const cuuint64_t sd[3] = {8, (cuuint64_t)c.cap, (cuuint64_t)B * 4};
+      const cuuint64_t ss[2] = {16, (cuuint64_t)c.cap * 16};
+      const cuuint32_t sb[3] = {8, 64, 1};
+      if ((rc = make_map_t(ksm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE, c.ks, 3, sd, ss, sb)))
+        return rc;
+      if ((rc = make_map_t(vsm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE, c.vs, 3, sd, ss, sb)))
+        return rc;
+    }
+  } else {
+    const cuuint64_t P = (cuuint64_t)c.page;
+    const cuuint64_t dims[4] = {256, P, 4, (cuuint64_t)c.n_pages};
+    const cuuint64_t str[3] = {row_bytes, P * row_bytes, 4 * P * row_bytes};
+    const cuuint32_t box[4] = {box_x, 64, 1, 1};
+    if ((rc = make_map_t(km, dt, CU_TENSOR_MAP_SWIZZLE_128B, c.k, 4, dims, str, box))) return rc;
+    if ((rc = make_map_t(vm, dt, CU_TENSOR_MAP_SWIZZLE_128B, c.v, 4, dims, str, box))) return rc;
+    if (c.q8()) {
+      const cuuint64_t sd[4] = {8, P, 4, (cuuint64_t)c.n_pages};
+      const cuuint64_t ss[3] = {16, P * 16, 4 * P * 16};
+      const cuuint32_t sb[4] = {8, 64, 1, 1};
+      if ((rc = make_map_t(ksm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE, c.ks, 4, sd, ss, sb)))
+        return rc;
+      if ((rc = make_map_t(vsm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE, c.vs, 4, sd, ss, sb)))
+        return rc;
+    }
+  }
+  return SPARK_OK;
+}
+
+int decode_impl(void* out, const void* q, const void* gate, const CacheView& c, int B, const int* pos,
+                const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes, unsigned flags, void* stream) {
+  int rc = check_view(c, cfg);
+  if (rc) return rc;
+  if (!out || !q || !gate || !pos || !workspace) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B > 65535) return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d", B);
+  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (!aligned16(out) || !aligned16(q) || !aligned16(workspace))
+    return fail(SPARK_ERR_INVALID_ARG, "tensors and workspace must be 16-byte aligned");
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  const DecodePlan pl = plan_for(B, c, sliding, g_dev[dev].sm_count);
+  if (ws_bytes < decode_ws_bytes(B, pl))
+    return fail(SPARK_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu needed", ws_bytes,
+                decode_ws_bytes(B, pl));
+  CUtensorMap km, vm, ksm, vsm;
+  if ((rc = decode_maps(c, B, &km, &vm, &ksm, &vsm))) return rc;
+
+  spark::DecodeParams P;
+  P.q = (const __nv_bfloat16*)q;
+  P.pos = pos;
+  P.o_part = (float*)workspace;
+  P.ml_part = (float*)workspace + (size_t)B * spark::kNq * pl.n_splits * spark::kHeadDim;
+  P.out = (__nv_bfloat16*)out;
+  P.gate = (const __nv_bfloat16*)gate;
+  P.B = B;
+  P.cap = c.cap;
+  P.sliding = sliding;
+  P.n_splits = pl.n_splits;
+  P.tiles_per_split = pl.tiles_per_split;
+  P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
+  P.rot = cfg->rot_dim;
+  P.log2_theta = log2(cfg->theta);
+  P.timeout_ns = wait_timeout_ns();
+  P.block_table = c.table;
+  P.max_pages = c.max_pages;
+  P.page_shift = c.paged() ? ilog2(c.page) : 0;
+  P.n_pages = c.n_pages;
+  dim3 grid(pl.n_splits, spark::kNkv, B);
+  cudaStream_t st = (cudaStream_t)stream;
+  const char* what;
+  if (c.q8()) {
+    what = "decode_q8_partial_kernel launch";
+    if (c.paged())
+      spark::decode_q8_partial_kernel<true><<<grid, spark::kQ8Threads, spark::kQ8SmemBytes, st>>>(km, ksm, vm, vsm, P);
+    else
+      spark::decode_q8_partial_kernel<false><<<grid, spark::kQ8Threads, spark::kQ8SmemBytes, st>>>(km, ksm, vm, vsm, P);
+  } else {
+    what = "decode_partial_kernel launch";
+    if (c.paged())
+      spark::decode_partial_kernel<true><<<grid, spark::kDecThreads, spark::kDecSmemBytes, st>>>(km, vm, P);
+    else
+      spark::decode_partial_kernel<false><<<grid, spark::kDecThreads, spark::kDecSmemBytes, st>>>(km, vm, P);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  if (pl.n_splits == 1) return SPARK_OK;      // the split kernel wrote the output itself
+  spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, st>>>(
+      (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_combine_kernel launch");
+}
+
 // ------------------------------------------------- decode without workspace ----
 // Some callers cannot allocate device memory when they run attention: a
 // serving runtime that plans all of its memory at start-up and forbids any
@@ -323,33 +546,12 @@ int spark_kv_append(void* k_cache, void* v_cache, int cap, const void* k, const 
                     void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (!k_cache || !v_cache || !k || !v || !pos0) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
-  if (B <= 0 || B > 65535 || T <= 0 || T > SPARK_MAX_POSITION || cap <= 0)
-    return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d cap=%d", B, T, cap);
-  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
-  const int sliding = cfg->kind == SPARK_SLIDING;
-  if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
-  if (!sliding && cap > SPARK_MAX_POSITION) return fail(SPARK_ERR_INVALID_ARG, "cap above 2^20");
-  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v))
-    return fail(SPARK_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-  int dev;
-  if ((rc = device_ready(&dev))) return rc;
-  const int t_first = sliding && T > SPARK_WINDOW ? T - SPARK_WINDOW : 0;
-  dim3 grid(T - t_first, B);
-  spark::kv_append_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
-      (__nv_bfloat16*)k_cache, (__nv_bfloat16*)v_cache, cap, (const __nv_bfloat16*)k,
-      (const __nv_bfloat16*)v, B, T, t_first, pos0, sliding, (flags & SPARK_ROPE_FUSED) ? 1 : 0,
-      log2(cfg->theta), cfg->rot_dim);
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "kv_append_kernel launch");
+  return append_impl(dense_view(k_cache, v_cache, nullptr, nullptr, cap), k, v, B, T, pos0, cfg, flags, stream);
 }
 
 size_t spark_decode_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg) {
   if (check_cfg(cfg) != SPARK_OK || B <= 0 || cap <= 0) return 0;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int sliding = cfg->kind == SPARK_SLIDING;
-  return decode_ws_bytes(B, decode_plan(B, sliding ? SPARK_WINDOW : cap, sliding, sms > 0 ? sms : 148));
+  return decode_ws_for(B, dense_view((void*)1, (void*)1, nullptr, nullptr, cap), cfg);
 }
 
 int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_cache,
@@ -358,56 +560,8 @@ int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_
                       unsigned flags, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (!out || !q || !gate || !k_cache || !v_cache || !pos || !workspace)
-    return fail(SPARK_ERR_INVALID_ARG, "null pointer");
-  if (B <= 0 || B > 65535 || cap <= 0) return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d cap=%d", B, cap);
-  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
-  const int sliding = cfg->kind == SPARK_SLIDING;
-  if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
-  if (!sliding && cap > SPARK_MAX_POSITION) return fail(SPARK_ERR_INVALID_ARG, "cap above 2^20");
-  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
-      !aligned16(workspace))
-    return fail(SPARK_ERR_INVALID_ARG, "tensors and workspace must be 16-byte aligned");
-  int dev;
-  if ((rc = device_ready(&dev))) return rc;
-  const DecodePlan pl = decode_plan(B, cap, sliding, g_dev[dev].sm_count);
-  if (ws_bytes < decode_ws_bytes(B, pl))
-    return fail(SPARK_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu needed", ws_bytes,
-                decode_ws_bytes(B, pl));
-
-  CUtensorMap km, vm;
-  const cuuint64_t dims[3] = {256, (cuuint64_t)cap, (cuuint64_t)B * 4};
-  const cuuint64_t strides[2] = {512, (cuuint64_t)cap * 512};
-  const cuuint32_t box[3] = {64, (cuuint32_t)spark::kDecNK, 1};
-  if ((rc = make_map(&km, k_cache, 3, dims, strides, box))) return rc;
-  if ((rc = make_map(&vm, v_cache, 3, dims, strides, box))) return rc;
-
-  spark::DecodeParams P;
-  P.q = (const __nv_bfloat16*)q;
-  P.pos = pos;
-  P.o_part = (float*)workspace;
-  P.ml_part = (float*)workspace + (size_t)B * spark::kNq * pl.n_splits * spark::kHeadDim;
-  P.B = B;
-  P.cap = cap;
-  P.sliding = sliding;
-  P.n_splits = pl.n_splits;
-  P.tiles_per_split = pl.tiles_per_split;
-  P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
-  P.rot = cfg->rot_dim;
-  P.log2_theta = log2(cfg->theta);
-  P.timeout_ns = wait_timeout_ns();
-  P.out = (__nv_bfloat16*)out;
-  P.gate = (const __nv_bfloat16*)gate;
-  dim3 grid(pl.n_splits, spark::kNkv, B);
-  spark::decode_partial_kernel<<<grid, spark::kDecThreads, spark::kDecSmemBytes, (cudaStream_t)stream>>>(
-      km, vm, P);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "decode_partial_kernel launch");
-  if (pl.n_splits == 1) return SPARK_OK;      // the partial kernel wrote the output itself
-  spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, (cudaStream_t)stream>>>(
-      (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
-  e = cudaGetLastError();
-  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_combine_kernel launch");
+  return decode_impl(out, q, gate, dense_view((void*)k_cache, (void*)v_cache, nullptr, nullptr, cap), B, pos, cfg,
+                     workspace, ws_bytes, flags, stream);
 }
 
 long long spark_kv_cache_q8_bytes(const spark_layer_cfg* cfg, int B, long long cap) {
@@ -420,35 +574,14 @@ int spark_kv_append_q8(void* k_codes, void* k_scales, void* v_codes, void* v_sca
                        const spark_layer_cfg* cfg, unsigned flags, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (!k_codes || !k_scales || !v_codes || !v_scales || !k || !v || !pos0)
-    return fail(SPARK_ERR_INVALID_ARG, "null pointer");
-  if (B <= 0 || B > 65535 || T <= 0 || T > SPARK_MAX_POSITION || cap <= 0)
-    return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d cap=%d", B, T, cap);
-  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
-  const int sliding = cfg->kind == SPARK_SLIDING;
-  if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
-  if (!sliding && cap > SPARK_MAX_POSITION) return fail(SPARK_ERR_INVALID_ARG, "cap above 2^20");
-  if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(k_scales) || !aligned16(v_scales) ||
-      !aligned16(k) || !aligned16(v))
-    return fail(SPARK_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-  int dev;
-  if ((rc = device_ready(&dev))) return rc;
-  const int t_first = sliding && T > SPARK_WINDOW ? T - SPARK_WINDOW : 0;
-  dim3 grid(T - t_first, B);
-  spark::kv_append_q8_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
-      (uint8_t*)k_codes, (__half*)k_scales, (uint8_t*)v_codes, (__half*)v_scales, cap,
-      (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, B, T, t_first, pos0, sliding,
-      (flags & SPARK_ROPE_FUSED) ? 1 : 0, log2(cfg->theta), cfg->rot_dim);
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "kv_append_q8_kernel launch");
+  if (!k_scales || !v_scales) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  return append_impl(dense_view(k_codes, v_codes, k_scales, v_scales, cap), k, v, B, T, pos0, cfg, flags,
+                     stream);
 }
 
 size_t spark_decode_q8_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg) {
   if (check_cfg(cfg) != SPARK_OK || B <= 0 || cap <= 0) return 0;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int sliding = cfg->kind == SPARK_SLIDING;
-  return decode_ws_bytes(B, decode_q8_plan(B, sliding ? SPARK_WINDOW : cap, sliding, sms > 0 ? sms : 148));
+  return decode_ws_for(B, dense_view((void*)1, (void*)1, (void*)1, (void*)1, cap), cfg);
 }
 
 int spark_attn_decode_q8(void* out, const void* q, const void* gate, const void* k_codes,
@@ -457,70 +590,35 @@ int spark_attn_decode_q8(void* out, const void* q, const void* gate, const void*
                          size_t ws_bytes, unsigned flags, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (!out || !q || !gate || !k_codes || !k_scales || !v_codes || !v_scales || !pos || !workspace)
-    return fail(SPARK_ERR_INVALID_ARG, "null pointer");
-  if (B <= 0 || B > 65535 || cap <= 0) return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d cap=%d", B, cap);
-  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
-  const int sliding = cfg->kind == SPARK_SLIDING;
-  if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
-  if (!sliding && cap > SPARK_MAX_POSITION) return fail(SPARK_ERR_INVALID_ARG, "cap above 2^20");
-  if (!aligned16(out) || !aligned16(q) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(k_scales) ||
-      !aligned16(v_scales) || !aligned16(workspace))
-    return fail(SPARK_ERR_INVALID_ARG, "tensors and workspace must be 16-byte aligned");
-  int dev;
-  if ((rc = device_ready(&dev))) return rc;
-  const DecodePlan pl = decode_q8_plan(B, cap, sliding, g_dev[dev].sm_count);
-  if (ws_bytes < decode_ws_bytes(B, pl))
-    return fail(SPARK_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu needed", ws_bytes,
-                decode_ws_bytes(B, pl));
+  if (!k_scales || !v_scales) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  return decode_impl(out, q, gate,
+                     dense_view((void*)k_codes, (void*)v_codes, (void*)k_scales, (void*)v_scales, cap), B, pos,
+                     cfg, workspace, ws_bytes, flags, stream);
+}
 
-  // codes [B*4][cap][256] u8 in two 128-byte swizzled boxes per row; scales [B*4][cap][8] fp16
-  CUtensorMap kcm, ksm, vcm, vsm;
-  const cuuint64_t cdims[3] = {256, (cuuint64_t)cap, (cuuint64_t)B * 4};
-  const cuuint64_t cstr[2] = {256, (cuuint64_t)cap * 256};
-  const cuuint32_t cbox[3] = {128, (cuuint32_t)spark::kQ8NK, 1};
-  const cuuint64_t sdims[3] = {8, (cuuint64_t)cap, (cuuint64_t)B * 4};
-  const cuuint64_t sstr[2] = {16, (cuuint64_t)cap * 16};
-  const cuuint32_t sbox[3] = {8, (cuuint32_t)spark::kQ8NK, 1};
-  if ((rc = make_map_t(&kcm, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_128B, k_codes, 3, cdims, cstr,
-                       cbox)))
-    return rc;
-  if ((rc = make_map_t(&vcm, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_128B, v_codes, 3, cdims, cstr,
-                       cbox)))
-    return rc;
-  if ((rc = make_map_t(&ksm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE, k_scales, 3, sdims,
-                       sstr, sbox)))
-    return rc;
-  if ((rc = make_map_t(&vsm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_SWIZZLE_NONE, v_scales, 3, sdims,
-                       sstr, sbox)))
-    return rc;
+int spark_kv_append_paged(const spark_paged_kv* kv, const void* k, const void* v, int B, int T,
+                          const int* pos0, const spark_layer_cfg* cfg, unsigned flags, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  CacheView c;
+  if ((rc = paged_view(kv, cfg, &c))) return rc;
+  return append_impl(c, k, v, B, T, pos0, cfg, flags, stream);
+}
 
-  spark::DecodeParams P;
-  P.q = (const __nv_bfloat16*)q;
-  P.pos = pos;
-  P.o_part = (float*)workspace;
-  P.ml_part = (float*)workspace + (size_t)B * spark::kNq * pl.n_splits * spark::kHeadDim;
-  P.B = B;
-  P.cap = cap;
-  P.sliding = sliding;
-  P.n_splits = pl.n_splits;
-  P.tiles_per_split = pl.tiles_per_split;
-  P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
-  P.rot = cfg->rot_dim;
-  P.log2_theta = log2(cfg->theta);
-  P.timeout_ns = wait_timeout_ns();
-  P.out = (__nv_bfloat16*)out;
-  P.gate = (const __nv_bfloat16*)gate;
-  dim3 grid(pl.n_splits, spark::kNkv, B);
-  spark::decode_q8_partial_kernel<<<grid, spark::kQ8Threads, spark::kQ8SmemBytes, (cudaStream_t)stream>>>(
-      kcm, ksm, vcm, vsm, P);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "decode_q8_partial_kernel launch");
-  if (pl.n_splits == 1) return SPARK_OK;      // the partial kernel wrote the output itself
-  spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, (cudaStream_t)stream>>>(
-      (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
-  e = cudaGetLastError();
-  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_combine_kernel launch");
+size_t spark_decode_paged_workspace_bytes(int B, const spark_paged_kv* kv, const spark_layer_cfg* cfg) {
+  CacheView c;
+  if (check_cfg(cfg) != SPARK_OK || B <= 0 || paged_view(kv, cfg, &c) != SPARK_OK) return 0;
+  return decode_ws_for(B, c, cfg);
+}
+
+int spark_attn_decode_paged(void* out, const void* q, const void* gate, const spark_paged_kv* kv, int B,
+                            const int* pos, const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
+                            unsigned flags, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  CacheView c;
+  if ((rc = paged_view(kv, cfg, &c))) return rc;
+  return decode_impl(out, q, gate, c, B, pos, cfg, workspace, ws_bytes, flags, stream);
 }
 
 int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, const void* gate,
@@ -651,7 +749,9 @@ int spark_attn_decode_static(void* out, const void* q, const void* gate, const v
   P.timeout_ns = wait_timeout_ns();
   P.out = (__nv_bfloat16*)out;
   P.gate = (const __nv_bfloat16*)gate;
-  spark::decode_partial_kernel<<<dim3(pl.n_splits, spark::kNkv, B), spark::kDecThreads, spark::kDecSmemBytes,
+  P.block_table = nullptr;
+  P.max_pages = P.page_shift = P.n_pages = 0;
+  spark::decode_partial_kernel<false><<<dim3(pl.n_splits, spark::kNkv, B), spark::kDecThreads, spark::kDecSmemBytes,
                                  (cudaStream_t)stream>>>(km, vm, P);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_partial_kernel launch");

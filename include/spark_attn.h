@@ -222,6 +222,49 @@ int spark_attn_decode_q8(void* out, const void* q, const void* gate, const void*
                          int B, const int* pos, const spark_layer_cfg* cfg, void* workspace,
                          size_t ws_bytes, unsigned flags, void* stream);
 
+/* ---- Paged KV caches (the serving form; "Spark-X2.6-4B-Base" hybrid-attention
+ * page §配套效率设计 serves the model through vLLM with prefix caching, whose
+ * KV lives in fixed-size pages).  One layer's K and V live in pools of pages;
+ * each sequence maps its logical pages to pool pages through a block table,
+ * so sequences may share the pages of a common prefix.
+ *   k, v           pools [n_pages][4][page_size][256]: bf16, or uint8 codes
+ *                  when k_scales/v_scales are set (the q8_0 format above)
+ *   k_scales, ...  NULL for bf16 pools, else fp16 [n_pages][4][page_size][8]
+ *   block_table    device int32 [B][max_pages]; logical row r of sequence b
+ *                  is row r % page_size of pool page block_table[b][r / page_size]
+ *   page_size      64, 128, 256 or 512
+ * Logical rows: full layers, row = position (positions < max_pages *
+ * page_size); sliding layers, row = position mod 512 (a ring over the first
+ * 512 / page_size table entries).  A page index outside [0, n_pages) that a
+ * call needs is a device-side argument error (spark_check: SPARK_ERR_DEVICE_ARG)
+ * and the affected sequence is not written.  Pages shared by several
+ * sequences are only read by decode; appending into a shared page is the
+ * caller's decision (copy it first to keep the other sequences' rows). */
+typedef struct {
+  void* k;
+  void* v;
+  void* k_scales;
+  void* v_scales;
+  const int* block_table;
+  int page_size;
+  int n_pages;
+  int max_pages;
+} spark_paged_kv;
+
+/* spark_kv_append / spark_kv_append_q8 into a paged pool (same arguments,
+ * positions, rotation and checks otherwise). */
+int spark_kv_append_paged(const spark_paged_kv* kv, const void* k, const void* v, int B, int T,
+                          const int* pos0, const spark_layer_cfg* cfg, unsigned flags, void* stream);
+
+/* Workspace bytes spark_attn_decode_paged needs (0 on bad arguments). */
+size_t spark_decode_paged_workspace_bytes(int B, const spark_paged_kv* kv, const spark_layer_cfg* cfg);
+
+/* spark_attn_decode / spark_attn_decode_q8 over a paged pool: same
+ * arguments, positions, visibility and output. */
+int spark_attn_decode_paged(void* out, const void* q, const void* gate, const spark_paged_kv* kv, int B,
+                            const int* pos, const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
+                            unsigned flags, void* stream);
+
 /* Self-test of the failure-detection path: launches one block that waits,
  * with the same bounded wait every kernel of the library uses, on a barrier
  * phase that nothing completes.  The wait runs out after timeout_ns
