@@ -392,19 +392,34 @@ def run_decode(torch, sa, synth, dist, args, peaks, world):
     }
 
 
-def decode_q8_layers(torch, sa, synth, dev, B: int, p: int, layer_ids=range(N_LAYERS), seed: int = DECODE_SEED,
-                     chunk: int = 2048):
-    """8-bit caches holding positions 0..p-1 (quantised by spark_kv_append_q8 from the generator's
-    tokens, keys taken as rotated) and the new token's q/k/v/gate at p, per layer."""
+def decode_append_layers(torch, sa, synth, dev, B: int, p: int, layer_ids=range(N_LAYERS),
+                         seed: int = DECODE_SEED, q8: bool = False, page: int = 0, chunk: int = 2048):
+    """Caches holding positions 0..p-1 written through the library's own append (the generator's
+    tokens, keys taken as rotated) and the new token's q/k/v/gate at p, per layer.  q8: 8-bit
+    caches; page > 0: paged pools of `page`-row pages, each sequence's pages in shuffled order."""
+    import numpy as np
     layers = []
+    rng = np.random.default_rng(11)
     for l in layer_ids:
         kind = FULL if l % 4 == 3 else SLIDING
         cfg = sa.spark_layer_cfg_for_kind(kind)
         cap = WINDOW if kind == SLIDING else p + 1
-        kc = torch.empty(B, HKV, cap, D, dtype=torch.uint8, device=dev)
-        vc = torch.empty_like(kc)
-        ks = torch.empty(B, HKV, cap, D // 32, dtype=torch.float16, device=dev)
-        vs = torch.empty_like(ks)
+        dt = torch.uint8 if q8 else torch.bfloat16
+        L = dict(layer=l, kind=kind, cfg=cfg, cap=cap, q8=q8, page=page)
+        if page:
+            max_pages = -(-cap // page)
+            n_pages = B * max_pages
+            L["table"] = torch.from_numpy(rng.permutation(n_pages).reshape(B, max_pages).astype(np.int32)).to(dev)
+            shape, sshape = (n_pages, HKV, page, D), (n_pages, HKV, page, D // 32)
+        else:
+            shape, sshape = (B, HKV, cap, D), (B, HKV, cap, D // 32)
+        L["kc"] = torch.empty(shape, dtype=dt, device=dev)
+        L["vc"] = torch.empty_like(L["kc"])
+        if q8:
+            L["ks"] = torch.empty(sshape, dtype=torch.float16, device=dev)
+            L["vs"] = torch.empty_like(L["ks"])
+        if page:
+            L["kv"] = sa.paged_kv(L["kc"], L["vc"], L["table"], L.get("ks"), L.get("vs"))
         first = 0 if kind == FULL else max(0, p - WINDOW)
         for c0 in range(first, p, chunk):
             n = min(chunk, p - c0)
@@ -412,7 +427,7 @@ def decode_q8_layers(torch, sa, synth, dev, B: int, p: int, layer_ids=range(N_LA
             vt = torch.empty_like(kt)
             synth.fill_tokens(kt, seed, synth.tensor_id(l, synth.ROLE_K), c0)
             synth.fill_tokens(vt, seed, synth.tensor_id(l, synth.ROLE_V), c0)
-            sa.spark_kv_append_q8(kc, ks, vc, vs, kt, vt, torch.full((B,), c0, dtype=torch.int32, device=dev), cfg)
+            append_layer(sa, L, kt, vt, torch.full((B,), c0, dtype=torch.int32, device=dev), 0)
             del kt, vt
         q = torch.empty(B, 1, HQ, D, dtype=torch.bfloat16, device=dev)
         kn = torch.empty(B, 1, HKV, D, dtype=torch.bfloat16, device=dev)
@@ -422,32 +437,62 @@ def decode_q8_layers(torch, sa, synth, dev, B: int, p: int, layer_ids=range(N_LA
         synth.fill_tokens(kn, seed, synth.tensor_id(l, synth.ROLE_K), p)
         synth.fill_tokens(vn, seed, synth.tensor_id(l, synth.ROLE_V), p)
         synth.fill_tokens(g, seed, synth.tensor_id(l, synth.ROLE_GATE), p)
-        layers.append(dict(layer=l, kind=kind, cfg=cfg, cap=cap, kc=kc, vc=vc, ks=ks, vs=vs, q=q.view(B, HQ, D),
-                           kn=kn, vn=vn, g=g.view(B, HQ),
-                           out=torch.empty(B, HQ, D, dtype=torch.bfloat16, device=dev)))
+        L.update(q=q.view(B, HQ, D), kn=kn, vn=vn, g=g.view(B, HQ),
+                 out=torch.empty(B, HQ, D, dtype=torch.bfloat16, device=dev))
+        layers.append(L)
     sa.spark_check()
     return layers
 
 
-def decode_q8_step(sa, layers, pos, ws):
-    """One decode step over 8-bit caches: per layer, quantise-append the new token (RoPE fused on k),
-    then attend (RoPE fused on q)."""
-    for L in layers:
-        sa.spark_kv_append_q8(L["kc"], L["ks"], L["vc"], L["vs"], L["kn"], L["vn"], pos, L["cfg"],
-                              flags=sa.SPARK_ROPE_FUSED)
+def decode_q8_layers(torch, sa, synth, dev, B: int, p: int, layer_ids=range(N_LAYERS), seed: int = DECODE_SEED):
+    """8-bit dense caches for the decode step (see decode_append_layers)."""
+    return decode_append_layers(torch, sa, synth, dev, B, p, layer_ids, seed, q8=True)
+
+
+def append_layer(sa, L, k, v, pos, flags):
+    if L["page"]:
+        sa.spark_kv_append_paged(L["kv"], k, v, pos, L["cfg"], flags=flags)
+    elif L["q8"]:
+        sa.spark_kv_append_q8(L["kc"], L["ks"], L["vc"], L["vs"], k, v, pos, L["cfg"], flags=flags)
+    else:
+        sa.spark_kv_append(L["kc"], L["vc"], k, v, pos, L["cfg"], flags=flags)
+
+
+def attend_layer(sa, L, pos, ws):
+    f = sa.SPARK_ROPE_FUSED
+    if L["page"]:
+        sa.spark_attn_decode_paged(L["out"], L["q"], L["g"], L["kv"], pos, L["cfg"], ws, flags=f)
+    elif L["q8"]:
         sa.spark_attn_decode_q8(L["out"], L["q"], L["g"], L["kc"], L["ks"], L["vc"], L["vs"], pos, L["cfg"], ws,
-                                flags=sa.SPARK_ROPE_FUSED)
+                                flags=f)
+    else:
+        sa.spark_attn_decode(L["out"], L["q"], L["g"], L["kc"], L["vc"], pos, L["cfg"], ws, flags=f)
 
 
-def run_decode_q8(torch, sa, synth, dist, args, peaks, world):
-    """The decode step of run_decode (36 layers, B=64, 32768 cached tokens, one CUDA graph) over the
-    8-bit KV cache."""
+def layer_ws_bytes(sa, B, L):
+    if L["page"]:
+        return sa.spark_decode_paged_workspace_bytes(B, L["kv"], L["cfg"])
+    if L["q8"]:
+        return sa.spark_decode_q8_workspace_bytes(B, L["cap"], L["cfg"])
+    return sa.spark_decode_workspace_bytes(B, L["cap"], L["cfg"])
+
+
+def decode_q8_step(sa, layers, pos, ws):
+    """One decode step over caches built by decode_append_layers: per layer, append the new token
+    (RoPE fused on k, quantised if the cache is 8-bit), then attend (RoPE fused on q)."""
+    for L in layers:
+        append_layer(sa, L, L["kn"], L["vn"], pos, sa.SPARK_ROPE_FUSED)
+        attend_layer(sa, L, pos, ws)
+
+
+def run_decode_variant(torch, sa, synth, dist, args, peaks, world, q8: bool, page: int):
+    """The decode step of run_decode (36 layers, B=64, 32768 cached tokens, one CUDA graph) over
+    an 8-bit cache (q8) and/or paged pools (page > 0)."""
     dev = torch.device("cuda")
     B, p = DECODE_B, DECODE_CTX
-    layers = decode_q8_layers(torch, sa, synth, dev, B, p)
+    layers = decode_append_layers(torch, sa, synth, dev, B, p, q8=q8, page=page)
     pos = torch.full((B,), p, dtype=torch.int32, device=dev)
-    ws = torch.empty(max(sa.spark_decode_q8_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers),
-                     dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(layer_ws_bytes(sa, B, L) for L in layers), dtype=torch.uint8, device=dev)
     decode_q8_step(sa, layers, pos, ws)
     torch.cuda.synchronize()
     sa.spark_check()
@@ -465,25 +510,32 @@ def run_decode_q8(torch, sa, synth, dist, args, peaks, world):
     reps = 10
     e0.record()
     for _ in range(reps):
-        sa.spark_attn_decode_q8(full["out"], full["q"], full["g"], full["kc"], full["ks"], full["vc"], full["vs"],
-                                pos, full["cfg"], ws, flags=sa.SPARK_ROPE_FUSED)
+        attend_layer(sa, full, pos, ws)
     e1.record()
     torch.cuda.synchronize()
     k_ms = e0.elapsed_time(e1) / reps
-    total_bytes = sum(decode_q8_kv_bytes(B, p, L["kind"]) for L in layers)
-    full_bytes = decode_q8_kv_bytes(B, p, FULL)
-    launches = decode_launches(sa, B, layers, q8=True)
+    per_key = decode_q8_kv_bytes if q8 else decode_kv_bytes
+    total_bytes = sum(per_key(B, p, L["kind"]) for L in layers)
+    full_bytes = per_key(B, p, FULL)
+    launches = sum(2 + (1 if layer_ws_bytes(sa, B, L) // (B * HQ * (D + 2) * 4) > 1 else 0) for L in layers)
     del graph, layers, ws
     torch.cuda.empty_cache()
+    name = ("decode_q8" if q8 else "decode") + (f"_paged{page}" if page else "")
+    kern = ("decode_q8_partial_kernel" if q8 else "decode_partial_kernel") + ("<paged>" if page else "")
     return {
         "value": total_bytes * world / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
         "ms_per_step": ms_step, "steps_per_s": 1e3 / ms_step, "kv_bytes_per_step": total_bytes,
-        "workload": f"decode_q8_b{B}_ctx{p}_36layers", "gpu_launches_per_step": launches,
-        "roofline": {"bound": "hbm", "kernel": "decode_q8_partial_kernel+combine (full layer)",
+        "workload": f"{name}_b{B}_ctx{p}_36layers", "gpu_launches_per_step": launches,
+        "roofline": {"bound": "hbm", "kernel": f"{kern}+combine (full layer)",
                      "achieved": full_bytes / (k_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": full_bytes / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                     "traffic": ncu_traffic("decode_q8_partial_kernel_full")},
+                     "traffic": None if page else ncu_traffic("decode_q8_partial_kernel_full" if q8 else
+                                                              "decode_partial_kernel_full")},
     }
+
+
+def run_decode_q8(torch, sa, synth, dist, args, peaks, world):
+    return run_decode_variant(torch, sa, synth, dist, args, peaks, world, q8=True, page=0)
 
 
 def run_long_prefill(torch, sa, synth, dist, args, peaks, world):
@@ -700,6 +752,8 @@ def main():
     res = run_prefill(torch, sa, synth, dist, args, peaks, world)
     dec = None if args.no_decode else run_decode(torch, sa, synth, dist, args, peaks, world)
     dec_q8 = None if args.no_decode else run_decode_q8(torch, sa, synth, dist, args, peaks, world)
+    dec_paged = None if args.no_decode else run_decode_variant(torch, sa, synth, dist, args, peaks, world,
+                                                               q8=False, page=256)
     long_pf = None if args.no_long else run_long_prefill(torch, sa, synth, dist, args, peaks, world)
     long_dec = None if (args.no_long or args.no_decode) else run_long_decode(torch, sa, synth, dist, args, peaks, world)
     cpu = None
@@ -724,7 +778,8 @@ def main():
         "tflops": res["tflops"], "prefill_full_kernel": res["prefill_full_kernel"],
         "roofline": res["roofline"], "e2e": res["e2e"], "clocks": res["clocks"],
         "gpu_launches": res["gpu_launches"] + (0 if dec is None else 0),
-        "cpu_baseline": cpu, "decode": dec, "decode_q8": dec_q8, "long_prefill": long_pf, "long_decode": long_dec,
+        "cpu_baseline": cpu, "decode": dec, "decode_q8": dec_q8, "decode_paged256": dec_paged,
+        "long_prefill": long_pf, "long_decode": long_dec,
     }
     print(json.dumps(line), flush=True)
 

@@ -82,6 +82,11 @@ def _lib():
         "spark_decode_paged_workspace_bytes": (ctypes.c_size_t, [_I, ctypes.POINTER(SparkPagedKV), cfgp]),
         "spark_attn_decode_paged": (_I, [_P, _P, _P, ctypes.POINTER(SparkPagedKV), _I, _P, cfgp, _P,
                                          ctypes.c_size_t, ctypes.c_uint, _P]),
+        "spark_rope_apply_varlen": (_I, [_P, _I, _P, _I, _P, _I, cfgp, _P]),
+        "spark_kv_append_varlen": (_I, [ctypes.POINTER(SparkPagedKV), _P, _P, _P, _I, _P, _I, cfgp, ctypes.c_uint,
+                                        _P]),
+        "spark_attn_prefill_varlen": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _P, ctypes.POINTER(SparkPagedKV), _I,
+                                           cfgp, ctypes.c_uint, _P]),
         "spark_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
         "spark_check": (_I, [_P]),
         "spark_last_error": (ctypes.c_char_p, []),
@@ -102,7 +107,8 @@ def exported_symbols():
             "spark_decode_workspace_bytes", "spark_attn_decode", "spark_attn_decode_static",
             "spark_kv_cache_q8_bytes", "spark_kv_append_q8", "spark_decode_q8_workspace_bytes",
             "spark_attn_decode_q8", "spark_kv_append_paged", "spark_decode_paged_workspace_bytes",
-            "spark_attn_decode_paged", "spark_selftest_wait_timeout", "spark_check", "spark_last_error",
+            "spark_attn_decode_paged", "spark_rope_apply_varlen", "spark_kv_append_varlen",
+            "spark_attn_prefill_varlen", "spark_selftest_wait_timeout", "spark_check", "spark_last_error",
             "spark_version"]
 
 
@@ -311,6 +317,44 @@ def spark_attn_decode_paged(out, q, gate, kv: SparkPagedKV, pos, cfg: SparkLayer
     ws_bytes = workspace.numel() * workspace.element_size()
     _raise(_lib().spark_attn_decode_paged(po, pq, pg, ctypes.byref(kv), q.shape[0], pp, ctypes.byref(cfg),
                                           workspace.data_ptr(), ws_bytes, flags, _stream(stream)))
+
+
+def _cu(cu_seqlens):
+    pc = _dev(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    return pc, cu_seqlens.shape[0] - 1
+
+
+def spark_rope_apply_varlen(x, cu_seqlens, max_seqlen: int, pos0, cfg: SparkLayerCfg, stream=None) -> None:
+    """Rotate packed x [total, H, 256] in place; sequence b is rows cu_seqlens[b]:cu_seqlens[b+1]."""
+    px = _dev(x, "x", ndim=3)
+    pc, B = _cu(cu_seqlens)
+    pp = _dev(pos0, "pos0", torch.int32, 1)
+    _raise(_lib().spark_rope_apply_varlen(px, x.shape[1], pc, max_seqlen, pp, B, ctypes.byref(cfg),
+                                          _stream(stream)))
+
+
+def spark_kv_append_varlen(kv: SparkPagedKV, k, v, cu_seqlens, max_seqlen: int, pos0, cfg: SparkLayerCfg,
+                           flags: int = 0, stream=None) -> None:
+    """Append packed k, v [total, 4, 256] into a paged pool."""
+    pk, pv = _dev(k, "k", ndim=3), _dev(v, "v", ndim=3)
+    pc, B = _cu(cu_seqlens)
+    pp = _dev(pos0, "pos0", torch.int32, 1)
+    _raise(_lib().spark_kv_append_varlen(ctypes.byref(kv), pk, pv, pc, max_seqlen, pp, B, ctypes.byref(cfg), flags,
+                                         _stream(stream)))
+
+
+def spark_attn_prefill_varlen(out, q, k, v, gate, cu_seqlens, max_seqlen: int, pos0, history, cfg: SparkLayerCfg,
+                              flags: int = 0, stream=None) -> None:
+    """Prefill of a ragged batch: packed out/q [total, 16, 256], k/v [total, 4, 256], gate [total, 16];
+    history: a paged pool (paged_kv) or None."""
+    po, pq = _dev(out, "out", ndim=3), _dev(q, "q", ndim=3)
+    pk, pv = _dev(k, "k", ndim=3), _dev(v, "v", ndim=3)
+    pg = _dev(gate, "gate", ndim=2)
+    pc, B = _cu(cu_seqlens)
+    pp = _dev(pos0, "pos0", torch.int32, 1)
+    hist = ctypes.byref(history) if history is not None else None
+    _raise(_lib().spark_attn_prefill_varlen(po, pq, pk, pv, pg, pc, q.shape[0], max_seqlen, pp, hist, B,
+                                            ctypes.byref(cfg), flags, _stream(stream)))
 
 
 def spark_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:

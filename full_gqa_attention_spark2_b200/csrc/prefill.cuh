@@ -36,20 +36,30 @@ struct PrefillParams {
   int rope, rot;                 // rope: q is raw and is rotated in shared memory
   double log2_theta;
   unsigned long long timeout_ns;
+  // Ragged batches: sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1 of
+  // the packed q, k, v, gate and out (T is then the longest sequence), and its
+  // history comes from a paged pool: logical row r in page
+  // block_table[b * max_pages + r / page] at row r % page (block_table null:
+  // no paged history).
+  const int* cu_seqlens;
+  const int* block_table;
+  int max_pages, page_shift, n_pages;
 };
 
 // Which KV tiles a block visits.  Tile j < n_hist comes from the cache and
 // covers absolute positions [a0 + 128 j, +128); later tiles come from the
 // chunk and cover positions pos0 + 128 (c_lo + j - n_hist) + [0, 128).
 struct PfSchedule {
-  int pos0, qp0, q_last, need_lo, a0, n_hist, c_lo, n_tiles;
+  int pos0, T, qp0, q_last, need_lo, a0, n_hist, c_lo, n_tiles;
 };
 
-__device__ __forceinline__ PfSchedule pf_schedule(const PrefillParams& P, int qt, int pos0) {
+// T: this sequence's chunk length (P.T for a dense batch).
+__device__ __forceinline__ PfSchedule pf_schedule(const PrefillParams& P, int qt, int pos0, int T) {
   PfSchedule S;
   S.pos0 = pos0;
+  S.T = T;
   S.qp0 = pos0 + qt * kPfM;
-  S.q_last = min(pos0 + P.T, S.qp0 + kPfM) - 1;
+  S.q_last = min(pos0 + T, S.qp0 + kPfM) - 1;
   S.need_lo = P.sliding ? max(0, S.qp0 - (kWindow - 1)) : 0;
   S.n_hist = 0;
   S.a0 = 0;
@@ -81,7 +91,10 @@ __device__ __forceinline__ PfTile pf_tile(const PfSchedule& S, const PrefillPara
     // is moved back to end exactly at pos0, and the keys it shares with the
     // tile before it are masked.  Rows before 0 are the TMA's zero fill.  A
     // ring that has wrapped (pos0 >= 512) holds written rows everywhere.
-    if (j == S.n_hist - 1 && t.kt0 + kPfN > S.pos0 && (!P.sliding || S.pos0 < kWindow)) {
+    // Paged history keeps its tiles page-aligned instead (a moved tile would
+    // straddle pages): there the rows of the last page past pos0 must be finite.
+    if (j == S.n_hist - 1 && t.kt0 + kPfN > S.pos0 && (!P.sliding || S.pos0 < kWindow) &&
+        P.block_table == nullptr) {
       t.v_lo = max(S.need_lo, t.kt0);
       t.kt0 = S.pos0 - kPfN;
     }
@@ -92,7 +105,7 @@ __device__ __forceinline__ PfTile pf_tile(const PfSchedule& S, const PrefillPara
     t.kt0 = S.pos0 + c * kPfN;
     t.row = c * kPfN;
     t.v_lo = S.pos0;
-    t.v_hi = S.pos0 + P.T;
+    t.v_hi = S.pos0 + S.T;
   }
   return t;
 }

@@ -38,6 +38,17 @@ constexpr int kP2SmemBytes = 1024 + kPfQBytes + kP2Slots * kP2SlotBytes + 1024;
 constexpr uint32_t kIdescQK2 = umma_idesc_bf16(256, 128, false, false);
 constexpr uint32_t kIdescPV2 = umma_idesc_bf16(256, 256, false, true);
 
+// A history page index of a ragged batch's block table, or -1 outside the pool.
+__device__ __forceinline__ int pf_page(const PrefillParams& P, int b, int row) {
+  const int pg = P.block_table[(long long)b * P.max_pages + (row >> P.page_shift)];
+  return (pg >= 0 && pg < P.n_pages) ? pg : -1;
+}
+
+// kRagged: packed sequences of different lengths (cu_seqlens) with history
+// from a paged pool; q, k, v, gate and out are [total][heads][256] views
+// (4-D maps with a batch extent of 1), the pool maps 4-D (dim, row in page,
+// head, page).  Otherwise a dense batch [B][T] with a dense cache.
+template <bool kRagged>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     prefill2_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kcmap,
@@ -76,11 +87,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int pos0 = P.pos0[b];
-  const bool bad = pos0 < 0 || pos0 > kMaxPos - P.T || (P.has_cache && !P.sliding && pos0 > P.cap);
-  PfSchedule S = pf_schedule(P, qt, bad ? 0 : pos0);
+  // this sequence's first packed row and chunk length
+  const int tok0 = kRagged ? P.cu_seqlens[b] : 0;
+  const int T_b = kRagged ? P.cu_seqlens[b + 1] - tok0 : P.T;
+  const bool bad = pos0 < 0 || T_b < 0 || T_b > P.T || pos0 > kMaxPos - T_b ||
+                   (P.has_cache && !P.sliding && pos0 > P.cap);
+  PfSchedule S = pf_schedule(P, qt, bad ? 0 : pos0, bad ? 0 : T_b);
   if (bad) {
     S.n_tiles = 0;
     if (threadIdx.x == 0 && qt == 0 && h == 0) raise_error(kErrPosition, 0x500u | (unsigned)b);
+  } else if (kRagged && qt * kPfM >= T_b) {
+    S.n_tiles = 0;                    // a shorter sequence: this query tile is past its end
   }
   const int n = S.n_tiles;
 
@@ -122,7 +139,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       // Q lands on this block's own barrier: its softmax warps rotate it (RoPE at load) or
       // just see it arrive, then tell the even block's MMA thread
       mbar_arrive_expect_tx(bar_q, kPfQBytes);
-      for (int d = 0; d < 4; ++d) tma_load_4d(q_s + d * 16384, &qmap, bar_q, d * 64, h, qt * kPfM, b);
+      for (int d = 0; d < 4; ++d) {
+        if (kRagged) tma_load_4d(q_s + d * 16384, &qmap, bar_q, d * 64, h, tok0 + qt * kPfM, 0);
+        else tma_load_4d(q_s + d * 16384, &qmap, bar_q, d * 64, h, qt * kPfM, b);
+      }
       const int plane = b * kNkv + kvh;
       const int key_half = 64 * (int)rank;       // this block's keys of a K tile
       const int dim_half = 128 * (int)rank;      // this block's dims of a V tile
@@ -140,21 +160,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             ok = false;
             break;
           }
+          // paged history: the pages of this block's part of the tile (both blocks of the pair
+          // look up the same table, so both stop at the same tile on a bad index)
+          int pg[4] = {0, 0, 0, 0};
+          if (kRagged && t.hist) {
+            bool good = true;
+            for (int x = 0; x < 4; ++x) {
+              pg[x] = pf_page(P, b, is_k ? t.row + key_half : t.row + 32 * x);
+              good = good && pg[x] >= 0;
+            }
+            if (!good) {
+              if (lane == 0) raise_error(kErrPosition, 0xA00u | (unsigned)b);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+          }
+          const int pmask = (1 << P.page_shift) - 1;
           const uint32_t dst = slots + s * kP2SlotBytes;
           const uint32_t full0 = mapa_shared(bar_slot_full + 8 * s, 0);
           if (leader) mbar_arrive_expect_tx(bar_slot_full + 8 * s, 2 * kP2SlotBytes);
           if (is_k) {          // four 64-dim boxes of this block's 64 keys, 8 KB each
+            const int kr = t.row + key_half;
             for (int x = 0; x < 4; ++x) {
-              if (t.hist) tma2_load_3d(dst + x * 8192, &kcmap, full0, x * 64, t.row + key_half, plane);
-              else tma2_load_4d(dst + x * 8192, &kmap, full0, x * 64, kvh, t.row + key_half, b);
+              if (kRagged) {
+                if (t.hist) tma2_load_4d(dst + x * 8192, &kcmap, full0, x * 64, kr & pmask, kvh, pg[0]);
+                else tma2_load_4d(dst + x * 8192, &kmap, full0, x * 64, kvh, tok0 + kr, 0);
+              } else {
+                if (t.hist) tma2_load_3d(dst + x * 8192, &kcmap, full0, x * 64, kr, plane);
+                else tma2_load_4d(dst + x * 8192, &kmap, full0, x * 64, kvh, kr, b);
+              }
             }
           } else {             // four 32-key sub-tiles x this block's two 64-dim boxes, 4 KB each
             for (int x = 0; x < 4; ++x)
               for (int d = 0; d < 2; ++d) {
                 const int dim = dim_half + 64 * d;
+                const int vr = t.row + 32 * x;
                 const uint32_t o = dst + x * 8192 + d * 4096;
-                if (t.hist) tma2_load_3d(o, &vcmap, full0, dim, t.row + 32 * x, plane);
-                else tma2_load_4d(o, &vmap, full0, dim, kvh, t.row + 32 * x, b);
+                if (kRagged) {
+                  if (t.hist) tma2_load_4d(o, &vcmap, full0, dim, vr & pmask, kvh, pg[x]);
+                  else tma2_load_4d(o, &vmap, full0, dim, kvh, tok0 + vr, 0);
+                } else {
+                  if (t.hist) tma2_load_3d(o, &vcmap, full0, dim, vr, plane);
+                  else tma2_load_4d(o, &vmap, full0, dim, kvh, vr, b);
+                }
               }
           }
           ++li;
@@ -229,7 +278,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t ocol = tmem + lane_base + kOCol;
     const int qp = S.qp0 + r;
-    const bool row_valid = qp < S.pos0 + P.T;
+    const bool row_valid = qp < S.pos0 + S.T;
     const float c_scale = 0.0625f * 1.4426950408889634f;    // 1/sqrt(256) * log2(e)
     const uint32_t p_ready0 = mapa_shared(bar_p, 0);
     bool ok = true;
@@ -373,7 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       // then written with TMA tensor stores (rows past the chunk are clipped)
       float scale = 0.f;
       if (row_valid) {
-        const long long tok = (long long)b * P.T + (qp - S.pos0);
+        const long long tok = kRagged ? (long long)tok0 + (qp - S.pos0) : (long long)b * P.T + (qp - S.pos0);
         const float gl = __bfloat162float(P.gate[tok * kNq + h]);
         scale = (l_run > 0.f ? 1.f / l_run : 0.f) * (1.f / (1.f + expf(-gl)));
       }
@@ -407,10 +456,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         : "=r"(all_ok)
         : "r"((uint32_t)ep_ok)
         : "memory");
-    if (all_ok && threadIdx.x == 128) {
-      for (int d = 0; d < 4; ++d) tma_store_4d(&omap, q_s + d * 16384, d * 64, h, qt * kPfM, b);
+    const bool full_rows = !kRagged || (qt + 1) * kPfM <= S.T;
+    if (all_ok && full_rows && threadIdx.x == 128) {
+      for (int d = 0; d < 4; ++d) {
+        if (kRagged) tma_store_4d(&omap, q_s + d * 16384, d * 64, h, tok0 + qt * kPfM, 0);
+        else tma_store_4d(&omap, q_s + d * 16384, d * 64, h, qt * kPfM, b);
+      }
       bulk_commit_group();
       bulk_wait_group0();
+    }
+    if (kRagged && all_ok && !full_rows && row_valid) {
+      // the sequence ends inside this tile: the rows after it belong to the next sequence, so
+      // each row is stored by its own thread (the box store would cover all 128)
+      const uint8_t* q_gen = gbase;
+      uint4* dst = reinterpret_cast<uint4*>(P.out + ((long long)(tok0 + (qp - S.pos0)) * kNq + h) * kHeadDim);
+#pragma unroll
+      for (int bx = 0; bx < 4; ++bx)
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          dst[bx * 8 + ch] = *reinterpret_cast<const uint4*>(q_gen + bx * 16384 + r * 128 + ((ch ^ (r & 7)) << 4));
     }
     __syncwarp();
   }

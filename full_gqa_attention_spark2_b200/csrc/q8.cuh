@@ -63,19 +63,21 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
     uint8_t* __restrict__ k_codes, __half* __restrict__ k_scales, uint8_t* __restrict__ v_codes,
     __half* __restrict__ v_scales, int cap, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, int B, int T, int t_first, const int* __restrict__ pos0, int sliding,
-    int rope, double log2_theta, int rot, CachePages pages) {
+    int rope, double log2_theta, int rot, CachePages pages, const int* __restrict__ cu) {
   __shared__ float xs[2][kNkv * kHeadDim + kNkv * kHeadDim / 32];
-  const int t = t_first + blockIdx.x;
   const int b = blockIdx.y;
   const int tid = threadIdx.x;
+  const TokenSpan sp = token_span(b, T, t_first, sliding, cu);
+  const int t = sp.t_first + blockIdx.x;
+  if (t >= sp.T) return;
   const int p0 = pos0[b];
-  const bool bad = p0 < 0 || p0 > kMaxPos - T || (!sliding && p0 + T > cap);
+  const bool bad = p0 < 0 || p0 > kMaxPos - sp.T || (!sliding && p0 + sp.T > cap);
   if (bad) {
     if (blockIdx.x == 0 && tid == 0) raise_error(kErrPosition, 0x400u | (unsigned)b);
     return;
   }
   const int pos = p0 + t;
-  const long long src = ((long long)b * T + t) * kNkv * kHeadDim;
+  const long long src = (sp.tok0 + t) * kNkv * kHeadDim;
   // thread = one 16-byte chunk (8 dims) of K and of V: head tid / 32, dims 8 (tid % 32) ..
   {
     const uint4 kr = reinterpret_cast<const uint4*>(k + src)[tid];

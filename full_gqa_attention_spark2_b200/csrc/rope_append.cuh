@@ -29,10 +29,13 @@ __device__ __forceinline__ void rope_angle(int pos, double f, float& c, float& s
   sincosf((float)r, &s, &c);
 }
 
-// x [B][T][H][256], in place.  One thread per (token, two consecutive pairs).
+// x [B][T][H][256] (dense, cu == nullptr) or packed [total][H][256] with
+// sequence b at rows cu[b] .. cu[b+1]-1 (ragged), in place.  One thread per
+// (token, two consecutive pairs).  Dense: a 1-D grid over the B*T tokens.
+// Ragged: grid.y = sequence, grid.x over its tokens (T = the longest).
 __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x, int B, int T,
                                                    int H, const int* __restrict__ pos0,
-                                                   double log2_theta, int rot) {
+                                                   double log2_theta, int rot, const int* __restrict__ cu) {
   __shared__ double freq[128];
   const int half = rot >> 1;
   for (int i = threadIdx.x; i < half; i += blockDim.x)
@@ -42,12 +45,24 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
   const int per_tok = half >> 1;                  // threads per token
   const int tok_per_block = blockDim.x / per_tok;
   const int j = threadIdx.x % per_tok;
-  const long long n = (long long)blockIdx.x * tok_per_block + threadIdx.x / per_tok;
-  if (threadIdx.x / per_tok >= tok_per_block || n >= (long long)B * T) return;
-  const int b = (int)(n / T);
-  const int t = (int)(n % T);
+  if (threadIdx.x / per_tok >= tok_per_block) return;
+  long long n;                                    // packed row of the token
+  int b, t, T_b;
+  if (cu == nullptr) {
+    n = (long long)blockIdx.x * tok_per_block + threadIdx.x / per_tok;
+    if (n >= (long long)B * T) return;
+    b = (int)(n / T);
+    t = (int)(n % T);
+    T_b = T;
+  } else {
+    b = blockIdx.y;
+    t = blockIdx.x * tok_per_block + threadIdx.x / per_tok;
+    T_b = cu[b + 1] - cu[b];
+    if (t >= T_b) return;
+    n = (long long)cu[b] + t;
+  }
   const int p0 = pos0[b];
-  if (p0 < 0 || p0 > kMaxPos - T) {
+  if (p0 < 0 || p0 > kMaxPos - T_b) {
     if (t == 0 && j == 0) raise_error(kErrPosition, 0x100u | (unsigned)b);
     return;
   }
@@ -83,6 +98,20 @@ __device__ __forceinline__ long long cache_row(const CachePages& pg, int b, int 
   return ((long long)page * kNkv + h) * (1 << pg.page_shift) + (row & ((1 << pg.page_shift) - 1));
 }
 
+// The tokens of sequence b an append writes.  Dense batches [B][T]: rows
+// b*T + t, the launch's t_first.  Ragged (cu != nullptr): rows cu[b] + t of a
+// sequence of cu[b+1] - cu[b] tokens; a sliding layer writes its last 512.
+struct TokenSpan {
+  long long tok0;
+  int T, t_first;
+};
+
+__device__ __forceinline__ TokenSpan token_span(int b, int T, int t_first, int sliding, const int* cu) {
+  if (cu == nullptr) return TokenSpan{(long long)b * T, T, t_first};
+  const int T_b = cu[b + 1] - cu[b];
+  return TokenSpan{(long long)cu[b], T_b, (sliding && T_b > kWindow) ? T_b - kWindow : 0};
+}
+
 // Append k/v [B][T][4][256] of T new tokens into caches [B][4][cap][256].
 // One block per written token, thread = (head, 16-byte chunk of 8 dims).
 // Sliding layers (ring of 512 rows) only write the last min(T, 512) tokens.
@@ -90,20 +119,22 @@ __global__ void __launch_bounds__(128) kv_append_kernel(
     __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache, int cap,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int B, int T,
     int t_first, const int* __restrict__ pos0, int sliding, int rope, double log2_theta, int rot,
-    CachePages pages) {
-  const int t = t_first + blockIdx.x;
+    CachePages pages, const int* __restrict__ cu) {
   const int b = blockIdx.y;
   const int h = threadIdx.x >> 5;
   const int ch = threadIdx.x & 31;
+  const TokenSpan sp = token_span(b, T, t_first, sliding, cu);
+  const int t = sp.t_first + blockIdx.x;
+  if (t >= sp.T) return;
   const int p0 = pos0[b];
-  const bool bad = p0 < 0 || p0 > kMaxPos - T || (!sliding && p0 + T > cap);
+  const bool bad = p0 < 0 || p0 > kMaxPos - sp.T || (!sliding && p0 + sp.T > cap);
   if (bad) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(kErrPosition, 0x200u | (unsigned)b);
     return;
   }
   const int pos = p0 + t;
   const int row = sliding ? (pos & (kWindow - 1)) : pos;
-  const long long src = (((long long)b * T + t) * kNkv + h) * kHeadDim;
+  const long long src = ((sp.tok0 + t) * kNkv + h) * kHeadDim;
   const long long crow = cache_row(pages, b, h, cap, row);
   if (crow < 0) {                        // a page index outside the pool
     if (ch == 0) raise_error(kErrPosition, 0x900u | (unsigned)b);

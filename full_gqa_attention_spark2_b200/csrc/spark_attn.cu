@@ -86,9 +86,12 @@ int device_ready(int* dev_out) {
     if (a == cudaSuccess)
       a = cudaFuncSetAttribute(spark::decode_partial_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                spark::kDecSmemBytes);
-    cudaError_t b = cudaFuncSetAttribute(spark::prefill2_kernel,
+    cudaError_t b = cudaFuncSetAttribute(spark::prefill2_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          spark::kP2SmemBytes);
+    if (b == cudaSuccess)
+      b = cudaFuncSetAttribute(spark::prefill2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               spark::kP2SmemBytes);
     cudaError_t c = cudaFuncSetAttribute(spark::decode_q8_partial_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          spark::kQ8SmemBytes);
@@ -289,8 +292,10 @@ int check_view(const CacheView& c, const spark_layer_cfg* cfg) {
   return SPARK_OK;
 }
 
+// cu_seqlens == nullptr: k/v [B][T][4][256].  Otherwise packed [total][4][256]
+// with sequence b at rows cu_seqlens[b] .. cu_seqlens[b+1]-1 and T the longest.
 int append_impl(const CacheView& c, const void* k, const void* v, int B, int T, const int* pos0,
-                const spark_layer_cfg* cfg, unsigned flags, void* stream) {
+                const spark_layer_cfg* cfg, unsigned flags, void* stream, const int* cu_seqlens = nullptr) {
   int rc = check_view(c, cfg);
   if (rc) return rc;
   if (!k || !v || !pos0) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
@@ -307,11 +312,12 @@ int append_impl(const CacheView& c, const void* k, const void* v, int B, int T, 
   if (c.q8()) {
     spark::kv_append_q8_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
         (uint8_t*)c.k, (__half*)c.ks, (uint8_t*)c.v, (__half*)c.vs, c.cap, (const __nv_bfloat16*)k,
-        (const __nv_bfloat16*)v, B, T, t_first, pos0, sliding, rope, log2(cfg->theta), cfg->rot_dim, pages_of(c));
+        (const __nv_bfloat16*)v, B, T, t_first, pos0, sliding, rope, log2(cfg->theta), cfg->rot_dim, pages_of(c),
+        cu_seqlens);
   } else {
     spark::kv_append_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
         (__nv_bfloat16*)c.k, (__nv_bfloat16*)c.v, c.cap, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, B, T,
-        t_first, pos0, sliding, rope, log2(cfg->theta), cfg->rot_dim, pages_of(c));
+        t_first, pos0, sliding, rope, log2(cfg->theta), cfg->rot_dim, pages_of(c), cu_seqlens);
   }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, c.q8() ? "kv_append_q8_kernel launch" : "kv_append_kernel launch");
@@ -536,7 +542,7 @@ int spark_rope_apply(void* x, int B, int T, int H, const int* pos0, const spark_
   const long long grid = (n + tok_per_block - 1) / tok_per_block;
   if (grid > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "too many tokens");
   spark::rope_kernel<<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>(
-      (__nv_bfloat16*)x, B, T, H, pos0, log2(cfg->theta), cfg->rot_dim);
+      (__nv_bfloat16*)x, B, T, H, pos0, log2(cfg->theta), cfg->rot_dim, nullptr);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "rope_kernel launch");
 }
@@ -684,10 +690,119 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   P.rot = cfg->rot_dim;
   P.log2_theta = log2(cfg->theta);
   P.timeout_ns = wait_timeout_ns();
+  P.cu_seqlens = nullptr;
+  P.block_table = nullptr;
+  P.max_pages = P.page_shift = P.n_pages = 0;
   const long long blocks = (long long)B * spark::kNq * P.n_qt;
   if (blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");
   // clusters of two blocks (an SM pair): two query heads of a KV group, same query tile
-  spark::prefill2_kernel<<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
+  spark::prefill2_kernel<false><<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
+      qm, km, vm, kcm, vcm, om, P);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "prefill2_kernel launch");
+}
+
+int spark_rope_apply_varlen(void* x, int H, const int* cu_seqlens, int max_seqlen, const int* pos0, int B,
+                            const spark_layer_cfg* cfg, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!x || !pos0 || !cu_seqlens) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B > 65535 || max_seqlen <= 0 || max_seqlen > SPARK_MAX_POSITION || (H != 16 && H != 4))
+    return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d max_seqlen=%d H=%d", B, max_seqlen, H);
+  if (!aligned16(x)) return fail(SPARK_ERR_INVALID_ARG, "x must be 16-byte aligned");
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  const int tok_per_block = 128 / (cfg->rot_dim / 4);
+  dim3 grid((max_seqlen + tok_per_block - 1) / tok_per_block, B);
+  spark::rope_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>((__nv_bfloat16*)x, B, max_seqlen, H, pos0,
+                                                              log2(cfg->theta), cfg->rot_dim, cu_seqlens);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "rope_kernel launch");
+}
+
+int spark_kv_append_varlen(const spark_paged_kv* kv, const void* k, const void* v, const int* cu_seqlens,
+                           int max_seqlen, const int* pos0, int B, const spark_layer_cfg* cfg, unsigned flags,
+                           void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!cu_seqlens) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  CacheView c;
+  if ((rc = paged_view(kv, cfg, &c))) return rc;
+  return append_impl(c, k, v, B, max_seqlen, pos0, cfg, flags, stream, cu_seqlens);
+}
+
+int spark_attn_prefill_varlen(void* out, const void* q, const void* k, const void* v, const void* gate,
+                              const int* cu_seqlens, int total, int max_seqlen, const int* pos0,
+                              const spark_paged_kv* history, int B, const spark_layer_cfg* cfg, unsigned flags,
+                              void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!out || !q || !k || !v || !gate || !pos0 || !cu_seqlens) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B > 65535 || total <= 0 || max_seqlen <= 0 || max_seqlen > SPARK_MAX_POSITION)
+    return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d total=%d max_seqlen=%d", B, total, max_seqlen);
+  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v))
+    return fail(SPARK_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  CacheView c{};
+  if (history) {
+    if ((rc = paged_view(history, cfg, &c))) return rc;
+    if (c.q8()) return fail(SPARK_ERR_UNSUPPORTED, "prefill reads bf16 history pages only");
+    if ((rc = check_view(c, cfg))) return rc;
+  }
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  const int sliding = cfg->kind == SPARK_SLIDING;
+
+  // packed q, out [total][16][256] and k, v [total][4][256] as 4-D (dim, head, row, 1);
+  // the history pool [n_pages][4][page][256] as 4-D (dim, row in page, head, page)
+  CUtensorMap qm, km, vm, kcm, vcm, om;
+  {
+    const cuuint64_t dq[4] = {256, 16, (cuuint64_t)total, 1};
+    const cuuint64_t sq[3] = {512, 512ull * 16, 512ull * 16 * total};
+    const cuuint32_t bq[4] = {64, 1, (cuuint32_t)spark::kPfM, 1};
+    if ((rc = make_map(&qm, q, 4, dq, sq, bq))) return rc;
+    if ((rc = make_map(&om, out, 4, dq, sq, bq))) return rc;
+    const cuuint64_t dk[4] = {256, 4, (cuuint64_t)total, 1};
+    const cuuint64_t sk[3] = {512, 512ull * 4, 512ull * 4 * total};
+    const cuuint32_t bk[4] = {64, 1, (cuuint32_t)(spark::kPfN / 2), 1};
+    const cuuint32_t bv[4] = {64, 1, 32, 1};
+    if ((rc = make_map(&km, k, 4, dk, sk, bk))) return rc;
+    if ((rc = make_map(&vm, v, 4, dk, sk, bv))) return rc;
+    if (history) {
+      const cuuint64_t Pg = (cuuint64_t)c.page;
+      const cuuint64_t dc[4] = {256, Pg, 4, (cuuint64_t)c.n_pages};
+      const cuuint64_t sc[3] = {512, Pg * 512, 4 * Pg * 512};
+      const cuuint32_t bkc[4] = {64, (cuuint32_t)(spark::kPfN / 2), 1, 1};
+      const cuuint32_t bvc[4] = {64, 32, 1, 1};
+      if ((rc = make_map(&kcm, c.k, 4, dc, sc, bkc))) return rc;
+      if ((rc = make_map(&vcm, c.v, 4, dc, sc, bvc))) return rc;
+    } else {
+      kcm = km;
+      vcm = vm;
+    }
+  }
+  spark::PrefillParams P;
+  P.out = (__nv_bfloat16*)out;
+  P.gate = (const __nv_bfloat16*)gate;
+  P.pos0 = pos0;
+  P.B = B;
+  P.T = max_seqlen;
+  P.cap = history ? c.cap : 0;
+  P.sliding = sliding;
+  P.has_cache = history ? 1 : 0;
+  P.n_qt = (max_seqlen + spark::kPfM - 1) / spark::kPfM;
+  P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
+  P.rot = cfg->rot_dim;
+  P.log2_theta = log2(cfg->theta);
+  P.timeout_ns = wait_timeout_ns();
+  P.cu_seqlens = cu_seqlens;
+  P.block_table = history ? c.table : nullptr;
+  P.max_pages = history ? c.max_pages : 0;
+  P.page_shift = history ? ilog2(c.page) : 0;
+  P.n_pages = history ? c.n_pages : 0;
+  const long long blocks = (long long)B * spark::kNq * P.n_qt;
+  if (blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");
+  spark::prefill2_kernel<true><<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
       qm, km, vm, kcm, vcm, om, P);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "prefill2_kernel launch");

@@ -265,6 +265,36 @@ int spark_attn_decode_paged(void* out, const void* q, const void* gate, const sp
                             const int* pos, const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
                             unsigned flags, void* stream);
 
+/* ---- Ragged batches (packed sequences of different lengths), the serving
+ * form of prefill.  Sequence b's new tokens are rows cu_seqlens[b] ..
+ * cu_seqlens[b+1]-1 (device int32 [B+1], non-decreasing, cu_seqlens[0] = 0)
+ * of packed tensors with `total` rows: q, out [total][16][256], k, v
+ * [total][4][256], gate [total][16]; its first new token is at position
+ * pos0[b].  max_seqlen (host) bounds every cu_seqlens[b+1] - cu_seqlens[b];
+ * a longer sequence is a device-side argument error. */
+
+/* spark_rope_apply on packed rows: x [total][H][256], H = 16 or 4. */
+int spark_rope_apply_varlen(void* x, int H, const int* cu_seqlens, int max_seqlen, const int* pos0, int B,
+                            const spark_layer_cfg* cfg, void* stream);
+
+/* spark_kv_append_paged for packed k, v [total][4][256] (sliding layers write
+ * each sequence's last 512 tokens). */
+int spark_kv_append_varlen(const spark_paged_kv* kv, const void* k, const void* v, const int* cu_seqlens,
+                           int max_seqlen, const int* pos0, int B, const spark_layer_cfg* cfg, unsigned flags,
+                           void* stream);
+
+/* spark_attn_prefill for a ragged batch: each sequence's chunk attends to
+ * itself and to its history in the paged pool `history` (NULL: no history),
+ * which must hold positions [0, pos0[b]) for full layers and the ring of the
+ * last 512 for sliding layers (bf16 pools only; an 8-bit pool is
+ * SPARK_ERR_UNSUPPORTED here).  History tiles stay page-aligned, so the rows
+ * of a sequence's last history page past pos0[b] must hold finite values (a
+ * zero-initialised pool, or rows an earlier append wrote). */
+int spark_attn_prefill_varlen(void* out, const void* q, const void* k, const void* v, const void* gate,
+                              const int* cu_seqlens, int total, int max_seqlen, const int* pos0,
+                              const spark_paged_kv* history, int B, const spark_layer_cfg* cfg, unsigned flags,
+                              void* stream);
+
 /* Self-test of the failure-detection path: launches one block that waits,
  * with the same bounded wait every kernel of the library uses, on a barrier
  * phase that nothing completes.  The wait runs out after timeout_ns
