@@ -538,6 +538,101 @@ def run_decode_q8(torch, sa, synth, dist, args, peaks, world):
     return run_decode_variant(torch, sa, synth, dist, args, peaks, world, q8=True, page=0)
 
 
+RAGGED_B, RAGGED_SEED, RAGGED_PAGE = 16, 6, 256
+
+
+def ragged_workload():
+    """The serving mix: 16 sequences with seeded chunk lengths in [256, 4096] and history lengths in
+    [0, 16384] (positions before the chunk, already in a paged pool of 256-row pages)."""
+    import numpy as np
+    rng = np.random.default_rng(RAGGED_SEED)
+    lens = rng.integers(256, 4097, RAGGED_B).tolist()
+    hist = rng.integers(0, 16385, RAGGED_B).tolist()
+    return lens, hist
+
+
+def run_prefill_ragged(torch, sa, synth, dist, args, peaks, world):
+    """One sliding and one full layer over the ragged batch: RoPE on the packed k, the prefill with
+    paged history (RoPE on q fused at load), the append of the chunk into the pages."""
+    import numpy as np
+    dev = torch.device("cuda")
+    lens, hist = ragged_workload()
+    B, P = RAGGED_B, RAGGED_PAGE
+    total = sum(lens)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+    hcu = torch.tensor(np.concatenate([[0], np.cumsum(hist)]), dtype=torch.int32, device=dev)
+    pos0 = torch.tensor(hist, dtype=torch.int32, device=dev)
+    zeros = torch.zeros(B, dtype=torch.int32, device=dev)
+    max_len = max(lens)
+    L = {}
+    rng = np.random.default_rng(RAGGED_SEED + 1)
+    for kind, layer in ((SLIDING, 0), (FULL, 3)):
+        cfg = sa.spark_layer_cfg_for_kind(kind)
+        max_pages = WINDOW // P if kind == SLIDING else -(-max(h + n for h, n in zip(hist, lens)) // P)
+        n_pages = B * max_pages
+        table = torch.from_numpy(rng.permutation(n_pages).reshape(B, max_pages).astype(np.int32)).to(dev)
+        kp = torch.zeros(n_pages, HKV, P, D, dtype=torch.bfloat16, device=dev)
+        vp = torch.zeros_like(kp)
+        kv = sa.paged_kv(kp, vp, table)
+        # history: each sequence's positions 0..hist-1, generated per sequence and appended raw (RoPE fused)
+        hk = torch.empty(sum(hist), HKV, D, dtype=torch.bfloat16, device=dev)
+        hv = torch.empty_like(hk)
+        for b in range(B):
+            if hist[b]:
+                sl = slice(int(hcu[b]), int(hcu[b + 1]))
+                synth.fill_tokens(hk[sl].view(1, hist[b], HKV, D), RAGGED_SEED, synth.tensor_id(layer, synth.ROLE_K) + 16 * b, 0)
+                synth.fill_tokens(hv[sl].view(1, hist[b], HKV, D), RAGGED_SEED, synth.tensor_id(layer, synth.ROLE_V) + 16 * b, 0)
+        sa.spark_kv_append_varlen(kv, hk, hv, hcu, max(hist), zeros, cfg, flags=sa.SPARK_ROPE_FUSED)
+        del hk, hv
+        q = torch.empty(total, HQ, D, dtype=torch.bfloat16, device=dev)
+        k = torch.empty(total, HKV, D, dtype=torch.bfloat16, device=dev)
+        v = torch.empty_like(k)
+        g = torch.empty(total, HQ, dtype=torch.bfloat16, device=dev)
+        for b in range(B):
+            sl = slice(int(cu[b]), int(cu[b + 1]))
+            for t_, role, H in ((q, synth.ROLE_Q, HQ), (k, synth.ROLE_K, HKV), (v, synth.ROLE_V, HKV)):
+                synth.fill_tokens(t_[sl].view(1, lens[b], H, D), RAGGED_SEED, synth.tensor_id(layer, role) + 16 * b,
+                                  hist[b])
+            synth.fill_tokens(g[sl].view(1, lens[b], HQ), RAGGED_SEED, synth.tensor_id(layer, synth.ROLE_GATE) + 16 * b,
+                              hist[b])
+        L[kind] = dict(cfg=cfg, kv=kv, q=q, k=k, v=v, g=g, out=torch.empty_like(q), keep=(kp, vp, table))
+    sa.spark_check()
+
+    def step(i=0):
+        for kind in (SLIDING, FULL):
+            w = L[kind]
+            sa.spark_rope_apply_varlen(w["k"], cu, max_len, pos0, w["cfg"])
+            sa.spark_attn_prefill_varlen(w["out"], w["q"], w["k"], w["v"], w["g"], cu, max_len, pos0, w["kv"],
+                                         w["cfg"], flags=sa.SPARK_ROPE_FUSED)
+            sa.spark_kv_append_varlen(w["kv"], w["k"], w["v"], cu, max_len, pos0, w["cfg"])
+
+    for _ in range(max(3, min(args.warmup, 5))):
+        step()
+    sa.spark_check()
+    steps = max(3, min(args.steps, 20))
+    ms = timed_region(torch, dist, step, steps) / steps
+    sa.spark_check()
+    flops = sum(prefill_flops(1, n, h, kind, True) for kind in (SLIDING, FULL) for n, h in zip(lens, hist))
+    f_full = sum(prefill_flops(1, n, h, FULL, True) for n, h in zip(lens, hist))
+    # the full layer's prefill alone, for its roofline
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w = L[FULL]
+    e0.record()
+    for _ in range(5):
+        sa.spark_attn_prefill_varlen(w["out"], w["q"], w["k"], w["v"], w["g"], cu, max_len, pos0, w["kv"], w["cfg"],
+                                     flags=sa.SPARK_ROPE_FUSED)
+    e1.record()
+    torch.cuda.synchronize()
+    k_ms = e0.elapsed_time(e1) / 5
+    del L
+    torch.cuda.empty_cache()
+    return {"workload": f"prefill_ragged_b{B}_len256-4096_hist0-16384_page{P}_sliding+full",
+            "lens": lens, "history": hist, "value": total * world / (ms * 1e-3), "unit": "tok/s",
+            "ms_per_step": ms, "tflops": flops * world / (ms * 1e-3) / 1e12, "gpu_launches_per_step": 6,
+            "full_layer_kernel": {"ms": k_ms, "tflops": f_full / (k_ms * 1e-3) / 1e12,
+                                  "frac": f_full / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}}
+
+
 def run_long_prefill(torch, sa, synth, dist, args, peaks, world):
     """B=1, T=131072 in 16 chunks of 8192 over the growing cache, one full and one sliding layer."""
     dev = torch.device("cuda")
@@ -674,7 +769,7 @@ def run_profile_case(torch, sa, synth, which: str):
     prefill_full / prefill_sliding: B=4, T=8192 (q alone 268 MB > L2);
     decode_full: B=16, 32768 cached tokens, one full layer (2.1 GB of KV)."""
     dev = torch.device("cuda")
-    if which.startswith("prefill"):
+    if which in ("prefill_full", "prefill_sliding"):
         kind = FULL if which == "prefill_full" else SLIDING
         W, pos0 = prefill_workload(torch, sa, synth, dev)
         w = W[kind]
@@ -698,6 +793,10 @@ def run_profile_case(torch, sa, synth, which: str):
         ws = torch.empty(sa.spark_decode_workspace_bytes(B, p + 1, cfg), dtype=torch.uint8, device=dev)
         for _ in range(3):
             sa.spark_attn_decode(out, q.view(B, HQ, D), g.view(B, HQ), kc, vc, pos, cfg, ws, flags=sa.SPARK_ROPE_FUSED)
+    elif which == "prefill_ragged_full":
+        # run_prefill_ragged at its smallest: the second prefill2_kernel launch is the full layer's
+        import types
+        run_prefill_ragged(torch, sa, synth, None, types.SimpleNamespace(steps=1, warmup=0), load_peaks(), 1)
     elif which == "decode_q8_full":
         B, p = 16, DECODE_CTX
         L = decode_q8_layers(torch, sa, synth, dev, B, p, layer_ids=(3,))[0]
@@ -721,7 +820,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context prefill and decode workloads")
-    ap.add_argument("--profile", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_q8_full"],
+    ap.add_argument("--profile", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_q8_full",
+                                          "prefill_ragged_full"],
                     default=None,
                     help="run a small case of one kernel for ncu and exit")
     args = ap.parse_args()
@@ -754,6 +854,7 @@ def main():
     dec_q8 = None if args.no_decode else run_decode_q8(torch, sa, synth, dist, args, peaks, world)
     dec_paged = None if args.no_decode else run_decode_variant(torch, sa, synth, dist, args, peaks, world,
                                                                q8=False, page=256)
+    ragged = run_prefill_ragged(torch, sa, synth, dist, args, peaks, world)
     long_pf = None if args.no_long else run_long_prefill(torch, sa, synth, dist, args, peaks, world)
     long_dec = None if (args.no_long or args.no_decode) else run_long_decode(torch, sa, synth, dist, args, peaks, world)
     cpu = None
@@ -778,7 +879,8 @@ def main():
         "tflops": res["tflops"], "prefill_full_kernel": res["prefill_full_kernel"],
         "roofline": res["roofline"], "e2e": res["e2e"], "clocks": res["clocks"],
         "gpu_launches": res["gpu_launches"] + (0 if dec is None else 0),
-        "cpu_baseline": cpu, "decode": dec, "decode_q8": dec_q8, "decode_paged256": dec_paged,
+        "cpu_baseline": cpu, "prefill_ragged": ragged, "decode": dec, "decode_q8": dec_q8,
+        "decode_paged256": dec_paged,
         "long_prefill": long_pf, "long_decode": long_dec,
     }
     print(json.dumps(line), flush=True)

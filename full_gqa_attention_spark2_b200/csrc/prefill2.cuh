@@ -38,11 +38,9 @@ constexpr int kP2SmemBytes = 1024 + kPfQBytes + kP2Slots * kP2SlotBytes + 1024;
 constexpr uint32_t kIdescQK2 = umma_idesc_bf16(256, 128, false, false);
 constexpr uint32_t kIdescPV2 = umma_idesc_bf16(256, 256, false, true);
 
-// A history page index of a ragged batch's block table, or -1 outside the pool.
-__device__ __forceinline__ int pf_page(const PrefillParams& P, int b, int row) {
-  const int pg = P.block_table[(long long)b * P.max_pages + (row >> P.page_shift)];
-  return (pg >= 0 && pg < P.n_pages) ? pg : -1;
-}
+// Page-entry prefetch of a ragged batch: tiles ahead, and ring slots (2 ints each).
+constexpr int kPgAhead = 3;
+constexpr int kPgRing = 8;
 
 // kRagged: packed sequences of different lengths (cu_seqlens) with history
 // from a paged pool; q, k, v, gate and out are [total][heads][256] views
@@ -126,7 +124,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (n > 0 && warp == 0) {
+  if (n > 0 && warp == 0 && !kRagged) {
     // ------------------------------------------------------ producers (both)
     if (lane == 0) {
       tma_prefetch_desc(&qmap);
@@ -139,10 +137,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       // Q lands on this block's own barrier: its softmax warps rotate it (RoPE at load) or
       // just see it arrive, then tell the even block's MMA thread
       mbar_arrive_expect_tx(bar_q, kPfQBytes);
-      for (int d = 0; d < 4; ++d) {
-        if (kRagged) tma_load_4d(q_s + d * 16384, &qmap, bar_q, d * 64, h, tok0 + qt * kPfM, 0);
-        else tma_load_4d(q_s + d * 16384, &qmap, bar_q, d * 64, h, qt * kPfM, b);
-      }
+      for (int d = 0; d < 4; ++d) tma_load_4d(q_s + d * 16384, &qmap, bar_q, d * 64, h, qt * kPfM, b);
       const int plane = b * kNkv + kvh;
       const int key_half = 64 * (int)rank;       // this block's keys of a K tile
       const int dim_half = 128 * (int)rank;      // this block's dims of a V tile
@@ -160,50 +155,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             ok = false;
             break;
           }
-          // paged history: the pages of this block's part of the tile (both blocks of the pair
-          // look up the same table, so both stop at the same tile on a bad index)
-          int pg[4] = {0, 0, 0, 0};
-          if (kRagged && t.hist) {
-            bool good = true;
-            for (int x = 0; x < 4; ++x) {
-              pg[x] = pf_page(P, b, is_k ? t.row + key_half : t.row + 32 * x);
-              good = good && pg[x] >= 0;
-            }
-            if (!good) {
-              if (lane == 0) raise_error(kErrPosition, 0xA00u | (unsigned)b);
-              *abort_flag = 1;
-              ok = false;
-              break;
-            }
-          }
-          const int pmask = (1 << P.page_shift) - 1;
           const uint32_t dst = slots + s * kP2SlotBytes;
           const uint32_t full0 = mapa_shared(bar_slot_full + 8 * s, 0);
           if (leader) mbar_arrive_expect_tx(bar_slot_full + 8 * s, 2 * kP2SlotBytes);
           if (is_k) {          // four 64-dim boxes of this block's 64 keys, 8 KB each
-            const int kr = t.row + key_half;
             for (int x = 0; x < 4; ++x) {
-              if (kRagged) {
-                if (t.hist) tma2_load_4d(dst + x * 8192, &kcmap, full0, x * 64, kr & pmask, kvh, pg[0]);
-                else tma2_load_4d(dst + x * 8192, &kmap, full0, x * 64, kvh, tok0 + kr, 0);
-              } else {
-                if (t.hist) tma2_load_3d(dst + x * 8192, &kcmap, full0, x * 64, kr, plane);
-                else tma2_load_4d(dst + x * 8192, &kmap, full0, x * 64, kvh, kr, b);
-              }
+              if (t.hist) tma2_load_3d(dst + x * 8192, &kcmap, full0, x * 64, t.row + key_half, plane);
+              else tma2_load_4d(dst + x * 8192, &kmap, full0, x * 64, kvh, t.row + key_half, b);
             }
           } else {             // four 32-key sub-tiles x this block's two 64-dim boxes, 4 KB each
             for (int x = 0; x < 4; ++x)
               for (int d = 0; d < 2; ++d) {
                 const int dim = dim_half + 64 * d;
-                const int vr = t.row + 32 * x;
                 const uint32_t o = dst + x * 8192 + d * 4096;
-                if (kRagged) {
-                  if (t.hist) tma2_load_4d(o, &vcmap, full0, dim, vr & pmask, kvh, pg[x]);
-                  else tma2_load_4d(o, &vmap, full0, dim, kvh, tok0 + vr, 0);
-                } else {
-                  if (t.hist) tma2_load_3d(o, &vcmap, full0, dim, vr, plane);
-                  else tma2_load_4d(o, &vmap, full0, dim, kvh, vr, b);
-                }
+                if (t.hist) tma2_load_3d(o, &vcmap, full0, dim, t.row + 32 * x, plane);
+                else tma2_load_4d(o, &vmap, full0, dim, kvh, t.row + 32 * x, b);
               }
           }
           ++li;
@@ -212,6 +178,116 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       const bool q_landed = mbar_drain(bar_q, 0, 200000000ull);
       if (leader) {
         // the even block's slot barriers count both blocks' bytes: wait for all copies in flight
+        if (q_landed) {
+          for (int i = max(0, li - kP2Slots); i < li; ++i)
+            if (!mbar_drain(bar_slot_full + 8 * (i % kP2Slots), (i / kP2Slots) & 1, 200000000ull)) break;
+        }
+      } else if (!ok) {
+        __nanosleep(200000);   // aborted: let this block's last copies land before the pair leaves
+      }
+    }
+    __syncwarp();
+  } else if (n > 0 && warp == 0) {
+    // ------------------------------------------------- producers (both), ragged batch
+    const int key_half = 64 * (int)rank;       // this block's keys of a K tile
+    const int dim_half = 128 * (int)rank;      // this block's dims of a V tile
+    int li = 0;
+    bool ok = true;
+    if (lane == 0) {
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      if (P.has_cache) {
+        tma_prefetch_desc(&kcmap);
+        tma_prefetch_desc(&vcmap);
+      }
+      mbar_arrive_expect_tx(bar_q, kPfQBytes);
+      for (int d = 0; d < 4; ++d) tma_load_4d(q_s + d * 16384, &qmap, bar_q, d * 64, h, tok0 + qt * kPfM, 0);
+    }
+    {
+      // Ragged batch.  A history tile's rows [row, row + 128) lie in at most two pages (pages of
+      // 64 rows or more): those of rows `row` and `row + 64`.  Their table entries are fetched
+      // kPgAhead tiles ahead with 4-byte asynchronous copies into a small ring in shared memory,
+      // one commit group per tile, so the producer never waits on a table load in a register.
+      // Both blocks of the pair read the same table, so both stop at the same tile on a bad index.
+      if (lane == 0) {
+        const uint32_t ring = misc + 192;          // [kPgRing][2] int
+        int* ring_gen = reinterpret_cast<int*>(gmisc + 192);
+        auto fetch = [&](int j) {                  // entries of tile j (nothing for chunk tiles)
+          if (j < n) {
+            const PfTile t = pf_tile(S, P, j);
+            if (t.hist) {
+              // rows row + 64 .. may lie past the table's last page (then they are past the
+              // history and masked): read the first page's entry again instead
+              const int n_lp = P.sliding ? (kWindow >> P.page_shift) : P.max_pages;
+              const int lp_lo = t.row >> P.page_shift;
+              const int lp_hi = (t.row + 64) >> P.page_shift;
+              const int* row_tab = P.block_table + (long long)b * P.max_pages;
+              const int slot = j % kPgRing;
+              cp_async4(ring + 8 * slot, row_tab + lp_lo);
+              cp_async4(ring + 8 * slot + 4, row_tab + (lp_hi < n_lp ? lp_hi : lp_lo));
+            }
+          }
+          cp_async_commit();
+        };
+        for (int j = 0; j < kPgAhead; ++j) fetch(j);
+        const int pmask = (1 << P.page_shift) - 1;
+        for (int step = 0; step <= n && ok; ++step) {
+          if (step < n) {                          // tile `step` is next needed: fetch one more
+            fetch(step + kPgAhead);
+            cp_async_wait<kPgAhead>();             // ... and the groups up to tile `step` are in
+          }
+          for (int part = 0; part < 2 && ok; ++part) {
+            const bool is_k = (part == 0);
+            const int j = is_k ? step : step - 1;
+            if (j < 0 || j >= n) continue;
+            const PfTile t = pf_tile(S, P, j);
+            const int s = li % kP2Slots;
+            int pg_lo = 0, pg_hi = 0;
+            if (t.hist) {
+              pg_lo = ring_gen[2 * (j % kPgRing)];
+              pg_hi = ring_gen[2 * (j % kPgRing) + 1];
+              if (pg_lo < 0 || pg_lo >= P.n_pages || pg_hi < 0 || pg_hi >= P.n_pages) {
+                raise_error(kErrPosition, 0xA00u | (unsigned)b);
+                *abort_flag = 1;
+                ok = false;
+                break;
+              }
+            }
+            if (li >= kP2Slots &&
+                !mbar_wait(bar_slot_empty + 8 * s, ((li / kP2Slots) - 1) & 1, abort_flag, P.timeout_ns, 0x50u)) {
+              ok = false;
+              break;
+            }
+            const uint32_t dst = slots + s * kP2SlotBytes;
+            const uint32_t full0 = mapa_shared(bar_slot_full + 8 * s, 0);
+            if (leader) mbar_arrive_expect_tx(bar_slot_full + 8 * s, 2 * kP2SlotBytes);
+            if (is_k) {
+              const int kr = t.row + key_half;
+              const int pk = key_half ? pg_hi : pg_lo;
+              for (int x = 0; x < 4; ++x) {
+                if (t.hist) tma2_load_4d(dst + x * 8192, &kcmap, full0, x * 64, kr & pmask, kvh, pk);
+                else tma2_load_4d(dst + x * 8192, &kmap, full0, x * 64, kvh, tok0 + kr, 0);
+              }
+            } else {
+              for (int x = 0; x < 4; ++x)
+                for (int d = 0; d < 2; ++d) {
+                  const int dim = dim_half + 64 * d;
+                  const int vr = t.row + 32 * x;
+                  const uint32_t o = dst + x * 8192 + d * 4096;
+                  if (t.hist) tma2_load_4d(o, &vcmap, full0, dim, vr & pmask, kvh, x < 2 ? pg_lo : pg_hi);
+                  else tma2_load_4d(o, &vmap, full0, dim, kvh, tok0 + vr, 0);
+                }
+            }
+            ++li;
+          }
+        }
+        cp_async_wait<0>();                        // no copy into the ring may outlive the block
+      }
+    }
+    if (lane == 0) {
+      const bool q_landed = mbar_drain(bar_q, 0, 200000000ull);
+      if (leader) {
         if (q_landed) {
           for (int i = max(0, li - kP2Slots); i < li; ++i)
             if (!mbar_drain(bar_slot_full + 8 * (i % kP2Slots), (i / kP2Slots) & 1, 200000000ull)) break;

@@ -100,14 +100,15 @@ def test_append_varlen_paged(kind, q8):
                     assert np.array_equal(got, want), (b, t, name)
 
 
-def _prefill_varlen_case(kind, lens, pos0, P=64, seed=13, layer=0, fused_q=True):
+def _prefill_varlen_case(kind, lens, pos0, P=64, seed=13, layer=0, fused_q=True, tight=False):
     """History 0..pos0[b]-1 appended (RoPE fused) into a zero-initialised paged pool; the chunk's k
     rotated by spark_rope_apply_varlen; q raw (RoPE at load) unless fused_q is False."""
     B = len(lens)
     cfg = sa.spark_layer_cfg_for_kind(kind)
     sliding = kind == O.SLIDING
     cu = np.concatenate([[0], np.cumsum(lens)])
-    max_pages = 512 // P if sliding else -(-(max(p + n for p, n in zip(pos0, lens)) + 1) // P)
+    # tight: the table ends with the last page any position needs (a history tile may reach past it)
+    max_pages = 512 // P if sliding else -(-(max(p + n for p, n in zip(pos0, lens)) + (0 if tight else 1)) // P)
     n_pages = B * max_pages + 3
     rng = np.random.default_rng(5)
     table = torch.from_numpy(rng.permutation(n_pages)[:B * max_pages].reshape(B, max_pages).astype(np.int32)).cuda()
@@ -169,6 +170,12 @@ def test_prefill_varlen_no_history(kind, lens):
 ])
 def test_prefill_varlen_paged_history(kind, lens, pos0, P):
     _prefill_varlen_case(kind, lens, pos0, P=P)
+
+
+def test_prefill_varlen_tight_block_table():
+    """pos0 = 900 with 64-row pages and a 15-page table: the last history tile [896, 1024) reaches
+    rows 960.. that no table entry covers (they are past the history and masked)."""
+    _prefill_varlen_case(O.FULL, [1, 30], [900, 100], P=64, tight=True)
 
 
 def test_prefill_varlen_unfused_q():
