@@ -45,6 +45,7 @@ struct DecodeParams {
   int rope, rot;
   double log2_theta;
   unsigned long long timeout_ns;
+  RopeFreq freq;
   // paged caches only: pool [n_pages][4][page][256]; logical row r of sequence b
   // lives in page block_table[b * max_pages + r / page] at row r % page
   const int* block_table;
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const int i = d < half ? d : d - half;
         const float xp = __bfloat162float(qrow[e + (d < half ? half : -half)]);
         float c, s;
-        rope_angle(p, exp2(-(2.0 * i / P.rot) * P.log2_theta), c, s);
+        rope_angle(p, pow_u8(P.freq.f[1], i), c, s);
         // bf16 rounding of the rotated value, as the stand-alone RoPE kernel does
         x = __bfloat162float(__float2bfloat16_rn(d < half ? x * c - xp * s : x * c + xp * s));
       }

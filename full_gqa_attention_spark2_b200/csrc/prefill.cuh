@@ -36,6 +36,7 @@ struct PrefillParams {
   int rope, rot;                 // rope: q is raw and is rotated in shared memory
   double log2_theta;
   unsigned long long timeout_ns;
+  RopeFreq freq;
   // Ragged batches: sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1 of
   // the packed q, k, v, gate and out (T is then the longest sequence), and its
   // history comes from a paged pool: logical row r in page

@@ -42,6 +42,65 @@ constexpr uint32_t kIdescPV2 = umma_idesc_bf16(256, 256, false, true);
 constexpr int kPgAhead = 3;
 constexpr int kPgRing = 8;
 
+// RoPE at load: rotate the block's raw Q tile in shared memory (four 128-byte
+// swizzled [128 x 64] boxes) in place, shared by kRopeThreads threads (warps 2..7).
+// Thread t takes four adjacent pairs (dims 4 qd .. 4 qd + 3 and their partners
+// half later) on every n_grp-th row from row rg: four independent recurrences
+// and 8-byte accesses, two rows loaded before either is stored.  The first
+// row's angles are exact (fp64 product and reduction); the next rows advance by
+// the rotation by n_grp * f_i.
+constexpr int kRopeThreads = 192;
+
+__device__ __forceinline__ void rope_q_tile(uint8_t* qg, const PrefillParams& P, int qp0, int t) {
+  const int half = P.rot >> 1;
+  const int n_qd = half >> 2;                   // quads per row: 32 (sliding) or 8 (full)
+  const int n_grp = kRopeThreads / n_qd;        // row stride: 6 or 24
+  const int qd = t % n_qd;
+  const int rg = t / n_qd;
+  float c[4], sn[4], cf[4], sf[4];
+  const double r1 = P.freq.f[1];                // the same word for every lane
+  double f = pow_u8(r1, 4 * qd);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    rope_angle(qp0 + rg, f, c[e], sn[e]);
+    rope_angle(n_grp, f, cf[e], sf[e]);
+    f *= r1;
+  }
+  const int dlo = 4 * qd, dhi = 4 * qd + half;
+  auto addr = [&](int d, int row) -> uint2* {
+    return reinterpret_cast<uint2*>(qg + (d >> 6) * 16384 + row * 128 + ((((d & 63) >> 3) ^ (row & 7)) << 4) +
+                                    (d & 7) * 2);
+  };
+  auto rotate = [&](const uint2& lo, const uint2& hi, int row) {
+    const float l[4] = {bf16_lo(lo.x), bf16_hi(lo.x), bf16_lo(lo.y), bf16_hi(lo.y)};
+    const float h[4] = {bf16_lo(hi.x), bf16_hi(hi.x), bf16_lo(hi.y), bf16_hi(hi.y)};
+    uint2 ol, oh;
+    ol.x = pack_bf16(l[0] * c[0] - h[0] * sn[0], l[1] * c[1] - h[1] * sn[1]);
+    ol.y = pack_bf16(l[2] * c[2] - h[2] * sn[2], l[3] * c[3] - h[3] * sn[3]);
+    oh.x = pack_bf16(h[0] * c[0] + l[0] * sn[0], h[1] * c[1] + l[1] * sn[1]);
+    oh.y = pack_bf16(h[2] * c[2] + l[2] * sn[2], h[3] * c[3] + l[3] * sn[3]);
+    *addr(dlo, row) = ol;
+    *addr(dhi, row) = oh;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float cn = c[e] * cf[e] - sn[e] * sf[e];
+      sn[e] = sn[e] * cf[e] + c[e] * sf[e];
+      c[e] = cn;
+    }
+  };
+  int row = rg;
+  for (; row + n_grp < kPfM; row += 2 * n_grp) {
+    const uint2 lo0 = *addr(dlo, row), hi0 = *addr(dhi, row);
+    const uint2 lo1 = *addr(dlo, row + n_grp), hi1 = *addr(dhi, row + n_grp);
+    rotate(lo0, hi0, row);
+    rotate(lo1, hi1, row + n_grp);
+  }
+  if (row < kPfM) {
+    const uint2 lo0 = *addr(dlo, row), hi0 = *addr(dhi, row);
+    rotate(lo0, hi0, row);
+  }
+}
+
 // kRagged: packed sequences of different lengths (cu_seqlens) with history
 // from a paged pool; q, k, v, gate and out are [total][heads][256] views
 // (4-D maps with a batch extent of 1), the pool maps 4-D (dim, row in page,
@@ -111,7 +170,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       mbar_init(bar_o + 8 * x, 1);
     }
     mbar_init(bar_done, 1);
-    mbar_init(bar_q_ready, 8);          // 4 softmax warps of each block
+    mbar_init(bar_q_ready, P.rope ? 12 : 8);   // softmax warps (and RoPE helper warps 2, 3) of each block
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -348,6 +407,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       mbar_drain(bar_done, 0, 200000000ull);
     }
     __syncwarp();
+  } else if (n > 0 && warp >= 2 && warp < 4 && P.rope) {
+    // ------------------------------------------- RoPE helpers (both): their share of Q
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort_flag, P.timeout_ns, 0x74u));
+    if (ok) {
+      rope_q_tile(gbase, P, S.qp0, threadIdx.x - 64);
+      fence_proxy_async_smem();
+    }
+    __syncwarp();
+    if (lane == 0 && ok) {
+      if (leader) mbar_arrive(bar_q_ready);
+      else mbar_arrive_remote_cluster(mapa_shared(bar_q_ready, 0));
+    }
   } else if (n > 0 && warp >= 4) {
     // ------------------------------------------------- softmax warps (both)
     const int r = threadIdx.x - 128;
@@ -359,45 +430,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     const uint32_t p_ready0 = mapa_shared(bar_p, 0);
     bool ok = true;
     {
-      // Q: wait for this block's tile, rotate it in place when q is raw, hand it to the MMA
-      // thread.  Thread t rotates pairs (2 pp, 2 pp + 1) over a group of consecutive rows; the
-      // angle of the group's first row is exact (fp64 reduction), the next rows advance by
-      // the rotation by f_i (complex multiplication).
+      // Q: wait for this block's tile, rotate it in place when q is raw (with warps 2 and 3),
+      // hand it to the MMA thread.
       ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort_flag, P.timeout_ns, 0x73u));
       if (ok && P.rope) {
-        const int tq = threadIdx.x - 128;
-        const int half = P.rot >> 1;
-        const int n_pp = half >> 1;                       // pair-pairs: 64 (sliding) or 16 (full)
-        const int pp = tq % n_pp;
-        const int rows_per = 128 / (128 / n_pp);          // rows per thread: n_pp
-        const int r0 = (tq / n_pp) * rows_per;
-        float c[2], sn[2], cf[2], sf[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int i = 2 * pp + e;
-          const double f = exp2(-(2.0 * i / P.rot) * P.log2_theta);
-          rope_angle(S.qp0 + r0, f, c[e], sn[e]);
-          rope_angle(1, f, cf[e], sf[e]);
-        }
-        const int dlo = 2 * pp, dhi = 2 * pp + half;
-        uint8_t* qg = gbase;
-        for (int rr = 0; rr < rows_per; ++rr) {
-          const int row = r0 + rr;
-          uint32_t* plo = reinterpret_cast<uint32_t*>(qg + (dlo >> 6) * 16384 + row * 128 +
-                                                      (((((dlo & 63) >> 3) ^ (row & 7))) << 4) + (dlo & 7) * 2);
-          uint32_t* phi = reinterpret_cast<uint32_t*>(qg + (dhi >> 6) * 16384 + row * 128 +
-                                                      (((((dhi & 63) >> 3) ^ (row & 7))) << 4) + (dhi & 7) * 2);
-          const uint32_t lo = *plo, hi = *phi;
-          const float l0 = bf16_lo(lo), l1 = bf16_hi(lo), h0 = bf16_lo(hi), h1 = bf16_hi(hi);
-          *plo = pack_bf16(l0 * c[0] - h0 * sn[0], l1 * c[1] - h1 * sn[1]);
-          *phi = pack_bf16(h0 * c[0] + l0 * sn[0], h1 * c[1] + l1 * sn[1]);
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float cn = c[e] * cf[e] - sn[e] * sf[e];
-            sn[e] = sn[e] * cf[e] + c[e] * sf[e];
-            c[e] = cn;
-          }
-        }
+        rope_q_tile(gbase, P, S.qp0, threadIdx.x - 64);
         fence_proxy_async_smem();                         // the tensor core reads Q next
       }
       __syncwarp();

@@ -85,12 +85,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uin
 // Bounded wait on phase `parity` of an mbarrier.  Gives up when `*abort` is
 // set by another thread of the block or after `timeout_ns` of global time; on
 // a timeout it raises the device error word and sets `*abort`, so that every
-// role of the block leaves its loop instead of waiting forever.
+// role of the block leaves its loop instead of waiting forever.  A limit under
+// 1 us (tests) expires at the first unsuccessful test: the global timer may
+// advance in steps of a microsecond, too coarse to see such a limit pass.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t timeout_ns, unsigned where) {
   // never sleep inside one test for longer than the whole wait may last
   const uint32_t hint = timeout_ns < 10000000ull ? (uint32_t)timeout_ns : 10000000u;
   if (mbar_try_wait(bar, parity, hint)) return true;
+  if (timeout_ns < 1000ull) {
+    *abort = 1;
+    raise_error(kErrTimeout, where);
+    return false;
+  }
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity, hint)) return true;
@@ -140,6 +147,11 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
                                                   uint64_t timeout_ns, unsigned where) {
   const uint32_t hint = timeout_ns < 10000000ull ? (uint32_t)timeout_ns : 10000000u;
   if (mbar_try_wait_cluster(bar, parity, hint)) return true;
+  if (timeout_ns < 1000ull) {            // as in mbar_wait: sub-microsecond limits expire at once
+    *abort = 1;
+    raise_error(kErrTimeout, where);
+    return false;
+  }
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_cluster(bar, parity, hint)) return true;

@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
     uint8_t* __restrict__ k_codes, __half* __restrict__ k_scales, uint8_t* __restrict__ v_codes,
     __half* __restrict__ v_scales, int cap, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, int B, int T, int t_first, const int* __restrict__ pos0, int sliding,
-    int rope, double log2_theta, int rot, CachePages pages, const int* __restrict__ cu) {
+    int rope, const RopeFreq rf, int rot, CachePages pages, const int* __restrict__ cu) {
   __shared__ float xs[2][kNkv * kHeadDim + kNkv * kHeadDim / 32];
   const int b = blockIdx.y;
   const int tid = threadIdx.x;
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
         const bool lo = d < half;
         const int i = lo ? d : d - half;
         float c, s;
-        rope_angle(pos, exp2(-(2.0 * i / rot) * log2_theta), c, s);
+        rope_angle(pos, rf.f[i], c, s);
         const float xp = xs[0][q8_pad(8 * tid + e + (lo ? half : -half))];
         r[e] = __bfloat162float(__float2bfloat16_rn(lo ? x * c - xp * s : x * c + xp * s));
       }
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
         const int i = d < half ? d : d - half;
         const float xp = __bfloat162float(qrow[e + (d < half ? half : -half)]);
         float c, s;
-        rope_angle(p, exp2(-(2.0 * i / P.rot) * P.log2_theta), c, s);
+        rope_angle(p, pow_u8(P.freq.f[1], i), c, s);
         x = __bfloat162float(__float2bfloat16_rn(d < half ? x * c - xp * s : x * c + xp * s));
       }
       qv[k8] = x * 0.0625f;

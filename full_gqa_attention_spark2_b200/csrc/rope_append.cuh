@@ -19,6 +19,25 @@ constexpr int kNkv = 4;
 constexpr int kWindow = 512;
 constexpr int kMaxPos = 1 << 20;
 
+// Frequencies f_i = theta^(-2i/rot), i < rot/2, of one layer kind, computed
+// once on the host in double precision and passed in the kernel parameters.
+struct RopeFreq {
+  double f[128];
+};
+
+// r^n for 0 <= n < 256 by binary powers (at most 14 fp64 products).  With
+// r = f_1 = theta^(-2/rot), f_i = r^i: every lane of a warp reads the same
+// f_1, where a lane-indexed table read of the parameters would be serialised.
+__device__ __forceinline__ double pow_u8(double r, int n) {
+  double y = 1.0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    if (n & (1 << k)) y *= r;
+    r *= r;
+  }
+  return y;
+}
+
 // cos/sin of pos * f for an integer position, via an fp64 reduction mod 2*pi.
 __device__ __forceinline__ void rope_angle(int pos, double f, float& c, float& s) {
   const double kTwoPi = 6.283185307179586476925286766559;
@@ -31,53 +50,59 @@ __device__ __forceinline__ void rope_angle(int pos, double f, float& c, float& s
 
 // x [B][T][H][256] (dense, cu == nullptr) or packed [total][H][256] with
 // sequence b at rows cu[b] .. cu[b+1]-1 (ragged), in place.  One thread per
-// (token, two consecutive pairs).  Dense: a 1-D grid over the B*T tokens.
-// Ragged: grid.y = sequence, grid.x over its tokens (T = the longest).
+// (token, two consecutive pairs); a block walks kRopeIters groups of tokens,
+// so that its frequency table serves many tokens.  Dense: a 1-D grid over the
+// B*T tokens.  Ragged: grid.y = sequence, grid.x over its tokens (T = the
+// longest).
+constexpr int kRopeIters = 8;
+
 __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x, int B, int T,
                                                    int H, const int* __restrict__ pos0,
-                                                   double log2_theta, int rot, const int* __restrict__ cu) {
+                                                   const RopeFreq rf, int rot, const int* __restrict__ cu) {
   __shared__ double freq[128];
   const int half = rot >> 1;
-  for (int i = threadIdx.x; i < half; i += blockDim.x)
-    freq[i] = exp2(-(2.0 * i / rot) * log2_theta);
+  for (int i = threadIdx.x; i < half; i += blockDim.x) freq[i] = rf.f[i];
   __syncthreads();
 
   const int per_tok = half >> 1;                  // threads per token
   const int tok_per_block = blockDim.x / per_tok;
   const int j = threadIdx.x % per_tok;
   if (threadIdx.x / per_tok >= tok_per_block) return;
-  long long n;                                    // packed row of the token
-  int b, t, T_b;
-  if (cu == nullptr) {
-    n = (long long)blockIdx.x * tok_per_block + threadIdx.x / per_tok;
-    if (n >= (long long)B * T) return;
-    b = (int)(n / T);
-    t = (int)(n % T);
-    T_b = T;
-  } else {
-    b = blockIdx.y;
-    t = blockIdx.x * tok_per_block + threadIdx.x / per_tok;
-    T_b = cu[b + 1] - cu[b];
-    if (t >= T_b) return;
-    n = (long long)cu[b] + t;
-  }
-  const int p0 = pos0[b];
-  if (p0 < 0 || p0 > kMaxPos - T_b) {
-    if (t == 0 && j == 0) raise_error(kErrPosition, 0x100u | (unsigned)b);
-    return;
-  }
-  const int pos = p0 + t;
-  float c0, s0, c1, s1;
-  rope_angle(pos, freq[2 * j], c0, s0);
-  rope_angle(pos, freq[2 * j + 1], c1, s1);
-  __nv_bfloat16* row = x + n * H * kHeadDim;
-  for (int h = 0; h < H; ++h) {
-    uint32_t* lo_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + 2 * j);
-    uint32_t* hi_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + half + 2 * j);
-    uint32_t lo = *lo_p, hi = *hi_p;
-    float l0 = bf16_lo(lo), l1 = bf16_hi(lo), h0 = bf16_lo(hi), h1 = bf16_hi(hi);
-    *lo_p = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
-    *hi_p = pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);
+  for (int it = 0; it < kRopeIters; ++it) {
+    const long long slot = ((long long)blockIdx.x * kRopeIters + it) * tok_per_block + threadIdx.x / per_tok;
+    long long n;                                  // packed row of the token
+    int b, t, T_b;
+    if (cu == nullptr) {
+      n = slot;
+      if (n >= (long long)B * T) return;
+      b = (int)(n / T);
+      t = (int)(n % T);
+      T_b = T;
+    } else {
+      b = blockIdx.y;
+      t = (int)slot;
+      T_b = cu[b + 1] - cu[b];
+      if (t >= T_b) return;
+      n = (long long)cu[b] + t;
+    }
+    const int p0 = pos0[b];
+    if (p0 < 0 || p0 > kMaxPos - T_b) {
+      if (t == 0 && j == 0) raise_error(kErrPosition, 0x100u | (unsigned)b);
+      continue;
+    }
+    const int pos = p0 + t;
+    float c0, s0, c1, s1;
+    rope_angle(pos, freq[2 * j], c0, s0);
+    rope_angle(pos, freq[2 * j + 1], c1, s1);
+    __nv_bfloat16* row = x + n * H * kHeadDim;
+    for (int h = 0; h < H; ++h) {
+      uint32_t* lo_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + 2 * j);
+      uint32_t* hi_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + half + 2 * j);
+      uint32_t lo = *lo_p, hi = *hi_p;
+      float l0 = bf16_lo(lo), l1 = bf16_hi(lo), h0 = bf16_lo(hi), h1 = bf16_hi(hi);
+      *lo_p = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
+      *hi_p = pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);
+    }
   }
 }
 
@@ -118,7 +143,7 @@ __device__ __forceinline__ TokenSpan token_span(int b, int T, int t_first, int s
 __global__ void __launch_bounds__(128) kv_append_kernel(
     __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache, int cap,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int B, int T,
-    int t_first, const int* __restrict__ pos0, int sliding, int rope, double log2_theta, int rot,
+    int t_first, const int* __restrict__ pos0, int sliding, int rope, const RopeFreq rf, int rot,
     CachePages pages, const int* __restrict__ cu) {
   const int b = blockIdx.y;
   const int h = threadIdx.x >> 5;
@@ -161,8 +186,8 @@ __global__ void __launch_bounds__(128) kv_append_kernel(
   for (int e = 0; e < 4; ++e) {
     const int i0 = ch * 8 + 2 * e;
     float c0, s0, c1, s1;
-    rope_angle(pos, exp2(-(2.0 * i0 / rot) * log2_theta), c0, s0);
-    rope_angle(pos, exp2(-(2.0 * (i0 + 1) / rot) * log2_theta), c1, s1);
+    rope_angle(pos, rf.f[i0], c0, s0);
+    rope_angle(pos, rf.f[i0 + 1], c1, s1);
     float l0 = bf16_lo(l[e]), l1 = bf16_hi(l[e]), h0 = bf16_lo(hh[e]), h1 = bf16_hi(hh[e]);
     l[e] = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
     hh[e] = pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);

@@ -163,6 +163,31 @@ int make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, 
                     box);
 }
 
+// -------------------------------------------------------------- RoPE tables ----
+// f_i = theta^(-2i/rot) of the two layer kinds, computed once on the host in
+// double precision and passed in the kernel parameters (no device memory;
+// safe to use while a stream is being captured).
+struct RopeTables {
+  spark::RopeFreq freq[2];
+};
+
+const RopeTables& rope_tables() {
+  static RopeTables t;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    for (int k = 0; k < 2; ++k) {
+      const int rot = k == 0 ? 256 : 64;
+      const double theta = k == 0 ? 1.0e4 : 5.0e6;
+      for (int i = 0; i < 128; ++i) t.freq[k].f[i] = i < rot / 2 ? exp2(-(2.0 * i / rot) * log2(theta)) : 0.0;
+    }
+  });
+  return t;
+}
+
+int kind_index(const spark_layer_cfg* cfg) { return cfg->kind == SPARK_SLIDING ? 0 : 1; }
+
+const spark::RopeFreq& rope_freq(const spark_layer_cfg* cfg) { return rope_tables().freq[kind_index(cfg)]; }
+
 // -------------------------------------------------------------- checks -----
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -312,12 +337,12 @@ int append_impl(const CacheView& c, const void* k, const void* v, int B, int T, 
   if (c.q8()) {
     spark::kv_append_q8_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
         (uint8_t*)c.k, (__half*)c.ks, (uint8_t*)c.v, (__half*)c.vs, c.cap, (const __nv_bfloat16*)k,
-        (const __nv_bfloat16*)v, B, T, t_first, pos0, sliding, rope, log2(cfg->theta), cfg->rot_dim, pages_of(c),
+        (const __nv_bfloat16*)v, B, T, t_first, pos0, sliding, rope, rope_freq(cfg), cfg->rot_dim, pages_of(c),
         cu_seqlens);
   } else {
     spark::kv_append_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
         (__nv_bfloat16*)c.k, (__nv_bfloat16*)c.v, c.cap, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, B, T,
-        t_first, pos0, sliding, rope, log2(cfg->theta), cfg->rot_dim, pages_of(c), cu_seqlens);
+        t_first, pos0, sliding, rope, rope_freq(cfg), cfg->rot_dim, pages_of(c), cu_seqlens);
   }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, c.q8() ? "kv_append_q8_kernel launch" : "kv_append_kernel launch");
@@ -414,6 +439,7 @@ int decode_impl(void* out, const void* q, const void* gate, const CacheView& c, 
   P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
   P.rot = cfg->rot_dim;
   P.log2_theta = log2(cfg->theta);
+  P.freq = rope_freq(cfg);
   P.timeout_ns = wait_timeout_ns();
   P.block_table = c.table;
   P.max_pages = c.max_pages;
@@ -537,12 +563,12 @@ int spark_rope_apply(void* x, int B, int T, int H, const int* pos0, const spark_
   int dev;
   if ((rc = device_ready(&dev))) return rc;
   const int per_tok = cfg->rot_dim / 4;
-  const int tok_per_block = 128 / per_tok;
+  const int tok_per_block = 128 / per_tok * spark::kRopeIters;
   const long long n = (long long)B * T;
   const long long grid = (n + tok_per_block - 1) / tok_per_block;
   if (grid > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "too many tokens");
   spark::rope_kernel<<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>(
-      (__nv_bfloat16*)x, B, T, H, pos0, log2(cfg->theta), cfg->rot_dim, nullptr);
+      (__nv_bfloat16*)x, B, T, H, pos0, rope_freq(cfg), cfg->rot_dim, nullptr);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "rope_kernel launch");
 }
@@ -689,6 +715,7 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
   P.rot = cfg->rot_dim;
   P.log2_theta = log2(cfg->theta);
+  P.freq = rope_freq(cfg);
   P.timeout_ns = wait_timeout_ns();
   P.cu_seqlens = nullptr;
   P.block_table = nullptr;
@@ -712,10 +739,10 @@ int spark_rope_apply_varlen(void* x, int H, const int* cu_seqlens, int max_seqle
   if (!aligned16(x)) return fail(SPARK_ERR_INVALID_ARG, "x must be 16-byte aligned");
   int dev;
   if ((rc = device_ready(&dev))) return rc;
-  const int tok_per_block = 128 / (cfg->rot_dim / 4);
+  const int tok_per_block = 128 / (cfg->rot_dim / 4) * spark::kRopeIters;
   dim3 grid((max_seqlen + tok_per_block - 1) / tok_per_block, B);
   spark::rope_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>((__nv_bfloat16*)x, B, max_seqlen, H, pos0,
-                                                              log2(cfg->theta), cfg->rot_dim, cu_seqlens);
+                                                              rope_freq(cfg), cfg->rot_dim, cu_seqlens);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "rope_kernel launch");
 }
@@ -794,6 +821,7 @@ int spark_attn_prefill_varlen(void* out, const void* q, const void* k, const voi
   P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
   P.rot = cfg->rot_dim;
   P.log2_theta = log2(cfg->theta);
+  P.freq = rope_freq(cfg);
   P.timeout_ns = wait_timeout_ns();
   P.cu_seqlens = cu_seqlens;
   P.block_table = history ? c.table : nullptr;
@@ -861,6 +889,7 @@ int spark_attn_decode_static(void* out, const void* q, const void* gate, const v
   P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
   P.rot = cfg->rot_dim;
   P.log2_theta = log2(cfg->theta);
+  P.freq = rope_freq(cfg);
   P.timeout_ns = wait_timeout_ns();
   P.out = (__nv_bfloat16*)out;
   P.gate = (const __nv_bfloat16*)gate;
