@@ -773,10 +773,10 @@ def run_profile_case(torch, sa, synth, which: str):
         kind = FULL if which == "prefill_full" else SLIDING
         W, pos0 = prefill_workload(torch, sa, synth, dev)
         w = W[kind]
-        sa.spark_rope_apply(w["q"], pos0, w["cfg"])
         sa.spark_rope_apply(w["k"], pos0, w["cfg"])
-        for _ in range(3):
-            sa.spark_attn_prefill(w["out"], w["q"], w["k"], w["v"], w["g"], None, None, pos0, w["cfg"])
+        for _ in range(3):            # as in prefill_step: q raw, rotated at load
+            sa.spark_attn_prefill(w["out"], w["q"], w["k"], w["v"], w["g"], None, None, pos0, w["cfg"],
+                                  flags=sa.SPARK_ROPE_FUSED)
     elif which == "decode_full":
         B, p = 16, DECODE_CTX
         cfg = sa.spark_layer_cfg_for_kind(FULL)
