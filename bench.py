@@ -282,10 +282,10 @@ def run_prefill(torch, sa, synth, dist, args, peaks, world):
         "ms_per_step": ms_step,
         "tflops": (f_full + f_slide) * world / (ms_step * 1e-3) / 1e12,
         "prefill_full_kernel": {"ms": kern_ms, "tflops": achieved, "flops": f_full},
-        "roofline": {"bound": "tensor", "kernel": "prefill2_kernel (full layer, SM pairs)", "achieved": achieved,
+        "roofline": {"bound": "tensor", "kernel": "prefill3_kernel (full layer, persistent SM pairs)", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"bf16_tflops burst, {peaks['source']}",
-                     "traffic": ncu_traffic("prefill2_kernel_full")},
+                     "traffic": ncu_traffic("prefill3_kernel_full")},
         "e2e": {"value": tokens / (ms_e2e / e2e_steps * 1e-3), "unit": "tok/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk,

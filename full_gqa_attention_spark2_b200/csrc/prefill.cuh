@@ -111,4 +111,65 @@ __device__ __forceinline__ PfTile pf_tile(const PfSchedule& S, const PrefillPara
   return t;
 }
 
+// RoPE at load: rotate the block's raw Q tile in shared memory (four 128-byte
+// swizzled [128 x 64] boxes) in place, shared by kRopeThreads threads (warps 2..7).
+// Thread t takes four adjacent pairs (dims 4 qd .. 4 qd + 3 and their partners
+// half later) on every n_grp-th row from row rg: four independent recurrences
+// and 8-byte accesses, two rows loaded before either is stored.  The first
+// row's angles are exact (fp64 product and reduction); the next rows advance by
+// the rotation by n_grp * f_i.
+constexpr int kRopeThreads = 192;
+
+// n_thr: the threads sharing the tile (a multiple of 32 that n_qd divides).
+__device__ __forceinline__ void rope_q_tile(uint8_t* qg, const PrefillParams& P, int qp0, int t,
+                                            int n_thr = kRopeThreads) {
+  const int half = P.rot >> 1;
+  const int n_qd = half >> 2;                   // quads per row: 32 (sliding) or 8 (full)
+  const int n_grp = n_thr / n_qd;               // row stride: 6 or 24 for 192 threads
+  const int qd = t % n_qd;
+  const int rg = t / n_qd;
+  float c[4], sn[4], cf[4], sf[4];
+  const double r1 = P.freq.f[1];                // the same word for every lane
+  double f = pow_u8(r1, 4 * qd);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    rope_angle(qp0 + rg, f, c[e], sn[e]);
+    rope_angle(n_grp, f, cf[e], sf[e]);
+    f *= r1;
+  }
+  const int dlo = 4 * qd, dhi = 4 * qd + half;
+  auto addr = [&](int d, int row) -> uint2* {
+    return reinterpret_cast<uint2*>(qg + (d >> 6) * 16384 + row * 128 + ((((d & 63) >> 3) ^ (row & 7)) << 4) +
+                                    (d & 7) * 2);
+  };
+  auto rotate = [&](const uint2& lo, const uint2& hi, int row) {
+    const float l[4] = {bf16_lo(lo.x), bf16_hi(lo.x), bf16_lo(lo.y), bf16_hi(lo.y)};
+    const float h[4] = {bf16_lo(hi.x), bf16_hi(hi.x), bf16_lo(hi.y), bf16_hi(hi.y)};
+    uint2 ol, oh;
+    ol.x = pack_bf16(l[0] * c[0] - h[0] * sn[0], l[1] * c[1] - h[1] * sn[1]);
+    ol.y = pack_bf16(l[2] * c[2] - h[2] * sn[2], l[3] * c[3] - h[3] * sn[3]);
+    oh.x = pack_bf16(h[0] * c[0] + l[0] * sn[0], h[1] * c[1] + l[1] * sn[1]);
+    oh.y = pack_bf16(h[2] * c[2] + l[2] * sn[2], h[3] * c[3] + l[3] * sn[3]);
+    *addr(dlo, row) = ol;
+    *addr(dhi, row) = oh;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float cn = c[e] * cf[e] - sn[e] * sf[e];
+      sn[e] = sn[e] * cf[e] + c[e] * sf[e];
+      c[e] = cn;
+    }
+  };
+  int row = rg;
+  for (; row + n_grp < kPfM; row += 2 * n_grp) {
+    const uint2 lo0 = *addr(dlo, row), hi0 = *addr(dhi, row);
+    const uint2 lo1 = *addr(dlo, row + n_grp), hi1 = *addr(dhi, row + n_grp);
+    rotate(lo0, hi0, row);
+    rotate(lo1, hi1, row + n_grp);
+  }
+  if (row < kPfM) {
+    const uint2 lo0 = *addr(dlo, row), hi0 = *addr(dhi, row);
+    rotate(lo0, hi0, row);
+  }
+}
+
 }  // namespace spark

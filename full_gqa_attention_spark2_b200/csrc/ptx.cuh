@@ -259,6 +259,10 @@ __device__ __forceinline__ void tma_store_4d(const void* map, uint32_t src, int 
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // wait until this thread's bulk stores have completed
 __device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// the shared-memory sources of every committed bulk store have been read (the writes may still be in flight)
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 
 // 4-byte asynchronous copy global -> shared (completion per thread, by group).
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {

@@ -16,6 +16,7 @@
 #include "decode.cuh"
 #include "prefill.cuh"
 #include "prefill2.cuh"
+#include "prefill3.cuh"
 #include "ptx.cuh"
 #include "q8.cuh"
 #include "rope_append.cuh"
@@ -92,6 +93,9 @@ int device_ready(int* dev_out) {
     if (b == cudaSuccess)
       b = cudaFuncSetAttribute(spark::prefill2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                spark::kP2SmemBytes);
+    if (b == cudaSuccess)
+      b = cudaFuncSetAttribute(spark::prefill3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               spark::kP2SmemBytes);
     cudaError_t c = cudaFuncSetAttribute(spark::decode_q8_partial_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          spark::kQ8SmemBytes);
@@ -162,6 +166,9 @@ int make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, 
   return make_map_t(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_128B, ptr, rank, dims, strides,
                     box);
 }
+
+// Dense prefill without a cache runs the persistent kernel (prefill3).
+constexpr bool kPersistentPrefill = true;
 
 // -------------------------------------------------------------- RoPE tables ----
 // f_i = theta^(-2i/rot) of the two layer kinds, computed once on the host in
@@ -722,6 +729,16 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   P.max_pages = P.page_shift = P.n_pages = 0;
   const long long blocks = (long long)B * spark::kNq * P.n_qt;
   if (blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");
+  if (kPersistentPrefill && !k_cache) {
+    // one resident cluster per SM pair walks the units (two query heads x one 128-query tile)
+    const long long unit_pairs = (long long)B * 8 * ((P.n_qt + 1) / 2);
+    const long long sm_pairs = g_dev[dev].sm_count / 2;
+    const unsigned clusters = (unsigned)(unit_pairs < sm_pairs ? unit_pairs : sm_pairs);
+    spark::prefill3_kernel<<<2 * clusters, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
+        qm, km, vm, om, P);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "prefill3_kernel launch");
+  }
   // clusters of two blocks (an SM pair): two query heads of a KV group, same query tile
   spark::prefill2_kernel<false><<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
       qm, km, vm, kcm, vcm, om, P);
