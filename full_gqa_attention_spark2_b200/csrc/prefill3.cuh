@@ -15,7 +15,14 @@
 //     as soon as O is staged; the next unit's first P.V (which overwrites O)
 //     waits only until the epilogue has read O out of tensor memory (`o_free`);
 //   - the slot ring, the S buffers and all barrier phases continue across units.
-// Units are dealt in pairs of equal total work (see pf_unit).
+// The grid has one cluster per unit, in the order of pf_unit_of (per sequence
+// and KV head, the heaviest query tiles first).  A resident cluster takes more
+// units by cancelling clusters that have not started yet (cluster launch
+// control): the even block's producer asks for the next unit while it loads the
+// current one and hands the answer to every role of both blocks through a small
+// queue in shared memory.  Every unit runs exactly once, either in its own
+// cluster or in the one that cancelled it, and the hardware hands out units in
+// launch order, so the load balances like a non-persistent grid.
 #pragma once
 #include <cuda.h>
 #include "prefill.cuh"
@@ -27,33 +34,22 @@ struct PfUnit {
   int hp, qt, kvh, b;
 };
 
-// The units of one launch come in pairs: for each (sequence, KV head, head
-// pair), query tile n_qt-1-i with tile i, so every pair carries about the same
-// work (causal: n_qt+1 tiles, plus twice the history).  Pairs run in
-// (sequence, KV head) order, so the ~74 pairs in flight at any time read the
-// K/V of about one KV head (it stays in L2), and cluster c takes pairs
-// c, c + C, c + 2C, ...  Unit k of cluster c is member k % 2 of its pair
-// k / 2; returns 0 past the end, -1 for the absent second member of a middle
-// tile (odd n_qt), 1 otherwise.
-__device__ __forceinline__ int pf_unit(const PrefillParams& P, int c, int C, int k, PfUnit& x) {
-  const int pairs_per = (P.n_qt + 1) >> 1;                // per (b, kvh, hp)
-  const int p = c + C * (k >> 1);
-  if (p >= P.B * 8 * pairs_per) return 0;
-  const int g = p / (2 * pairs_per);                      // b * 4 + kvh
-  const int rem = p % (2 * pairs_per);
-  const int i = rem >> 1;
-  const int qt_hi = P.n_qt - 1 - i;
-  x.hp = rem & 1;
-  x.kvh = g & 3;
-  x.b = g >> 2;
-  if (k & 1) {
-    if (i == qt_hi) return -1;
-    x.qt = i;
-  } else {
-    x.qt = qt_hi;
-  }
-  return 1;
+// Unit u (a cluster id): head pair hp of KV head kvh of sequence b over query
+// tile qt, with u = ((b * 4 + kvh) * n_qt + (n_qt - 1 - qt)) * 2 + hp.  The
+// ~74 units in flight at a time read the K/V of about one KV head (it stays in
+// L2), and the long (causal: late) query tiles of each come first.
+__device__ __forceinline__ void pf_unit_of(const PrefillParams& P, int u, PfUnit& x) {
+  x.hp = u & 1;
+  int id = u >> 1;
+  x.qt = P.n_qt - 1 - id % P.n_qt;
+  id /= P.n_qt;
+  x.kvh = id & 3;
+  x.b = id >> 2;
 }
+
+constexpr int kUq = 8;          // unit queue entries
+constexpr int kUqReaders = 14;  // per entry: MMA thread, 2 Q warps, 4 softmax warps (even block);
+                                // producer, 2 Q warps, 4 softmax warps (odd block)
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     prefill3_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
@@ -80,20 +76,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gmisc + 168);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gmisc + 172);
   const uint32_t bar_o_staged = misc + 176;         // this block's output staged (one phase per unit)
+  const uint32_t bar_uq_full = misc + 184;          // [kUq] unit queue entry written (both)
+  const uint32_t bar_uq_empty = misc + 248;         // [kUq] entry read by every role (even block's)
+  const uint32_t bar_clc = misc + 312;              // cancellation answer landed (even block's)
+  volatile int* uq = reinterpret_cast<volatile int*>(gmisc + 320);   // [kUq] unit ids (-1: none left)
+  const uint32_t clc_resp = misc + 352;             // 16-byte cancellation answer
 
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int c = blockIdx.x >> 1;
-  const int C = gridDim.x >> 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Unit k of this cluster and its schedule: returns -2 past the last unit,
-  // else its tile count (0: nothing to do: no such unit, or a bad position,
-  // which is flagged).
-  auto unit_schedule = [&](int k, PfUnit& x, PfSchedule& S) -> int {
-    const int st = pf_unit(P, c, C, k, x);
-    if (st == 0) return -2;
-    if (st < 0) return 0;
+  // Unit u and its schedule: returns its tile count (0: a bad position, which is flagged).
+  auto unit_schedule = [&](int u, PfUnit& x, PfSchedule& S) -> int {
+    pf_unit_of(P, u, x);
     const int pos0 = P.pos0[x.b];
     const bool bad = pos0 < 0 || pos0 > kMaxPos - P.T || (P.has_cache && !P.sliding && pos0 > P.cap);
     S = pf_schedule(P, x.qt, bad ? 0 : pos0, bad ? 0 : P.T);
@@ -102,6 +97,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       if (threadIdx.x == 0 && x.qt == 0 && x.hp == 0 && x.kvh == 0) raise_error(kErrPosition, 0x500u | (unsigned)x.b);
     }
     return S.n_tiles;
+  };
+  // The k-th unit id of this cluster from the queue (every lane of a warp, or one thread), and
+  // the hand-back of its entry (one thread per reader).
+  auto uq_get = [&](int k, int& u, unsigned where) -> bool {
+    if (!mbar_wait_cluster(bar_uq_full + 8 * (k % kUq), (k / kUq) & 1, abort_flag, P.timeout_ns, where)) return false;
+    u = uq[k % kUq];
+    return true;
+  };
+  auto uq_release = [&](int k) {
+    if (leader) mbar_arrive(bar_uq_empty + 8 * (k % kUq));
+    else mbar_arrive_remote_cluster(mapa_shared(bar_uq_empty + 8 * (k % kUq), 0));
   };
 
   if (threadIdx.x == 0) {
@@ -120,6 +126,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     mbar_init(bar_q_free, 1);
     mbar_init(bar_o_free, 8);           // 4 softmax warps of each block
     mbar_init(bar_o_staged, 4);         // this block's 4 softmax warps
+    for (int e = 0; e < kUq; ++e) {
+      mbar_init(bar_uq_full + 8 * e, 1);
+      mbar_init(bar_uq_empty + 8 * e, kUqReaders);
+    }
+    mbar_init(bar_clc, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -142,12 +153,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       const int dim_half = 128 * (int)rank;      // this block's dims of a V tile
       int li = 0, qu = 0;
       bool ok = true;
+      // even block: the scheduler.  Entry k of both blocks' queues gets unit k's id.
+      auto publish = [&](int k, int u) -> bool {
+        const int e = k % kUq;
+        if (k >= kUq &&
+            !mbar_wait_cluster(bar_uq_empty + 8 * e, ((k / kUq) - 1) & 1, abort_flag, P.timeout_ns, 0x8Du))
+          return false;
+        uq[e] = u;
+        mbar_arrive(bar_uq_full + 8 * e);
+        asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(mapa_shared(smem_u32((const void*)(uq + e)), 1)), "r"(u)
+                     : "memory");
+        mbar_arrive_remote_cluster(mapa_shared(bar_uq_full + 8 * e, 1));
+        return true;
+      };
+      int clc_asked = 0, clc_got = 0;        // cancellation requests issued / answered
+      bool clc_more = true;                  // no request has come back empty yet
+      int u_next = (int)(blockIdx.x >> 1);   // this cluster's own unit first
+      if (leader) ok = publish(0, u_next);
       for (int k = 0; ok; ++k) {
+        int u = u_next;
+        if (!leader) {
+          ok = uq_get(k, u, 0x8Eu);
+          if (!ok) break;
+          uq_release(k);
+        }
+        if (u < 0) break;
+        if (leader && clc_more) {
+          // ask now for the unit after this one: a cluster that has not started gives up its own
+          mbar_arrive_expect_tx(bar_clc, 16);
+          asm volatile(
+              "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+                  clc_resp),
+              "r"(bar_clc)
+              : "memory");
+          ++clc_asked;
+        }
         PfUnit x;
         PfSchedule S;
-        const int n = unit_schedule(k, x, S);
-        if (n == -2) break;
-        if (n == 0) continue;
+        const int n = unit_schedule(u, x, S);
         const int h = x.kvh * 4 + x.hp * 2 + (int)rank;
         bool q_issued = false;
         for (int step = 0; step <= n && ok; ++step) {
@@ -189,7 +232,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             ++li;
           }
         }
+        if (leader && ok) {
+          u_next = -1;
+          if (clc_more) {
+            ok = mbar_wait(bar_clc, clc_got & 1, abort_flag, P.timeout_ns, 0x8Fu);
+            if (!ok) break;
+            ++clc_got;
+            uint32_t cx, valid;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+                "ld.shared.b128 r, [%2];\n\t"
+                "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+                "selp.u32 %1, 1, 0, p;\n\t"
+                "mov.u32 %0, 0;\n\t"
+                "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %0, r;\n\t}"
+                : "=r"(cx), "=r"(valid)
+                : "r"(clc_resp)
+                : "memory");
+            fence_proxy_async_smem();      // the next answer overwrites the buffer
+            if (valid) u_next = (int)(cx >> 1);
+            else clc_more = false;
+          }
+          ok = publish(k + 1, u_next);
+        }
       }
+      // an unanswered cancellation request must land before the block leaves
+      if (leader && clc_asked > clc_got) mbar_drain(bar_clc, clc_got & 1, 200000000ull);
       // never leave with copies in flight: this block's last Q, and (even block) every slot's bytes
       const bool q_landed = qu == 0 || mbar_drain(bar_q, (qu - 1) & 1, 200000000ull);
       if (leader) {
@@ -245,10 +313,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         return true;
       };
       for (int k = 0; ok; ++k) {
+        int u;
+        if (!uq_get(k, u, 0x90u)) break;
+        uq_release(k);
+        if (u < 0) break;
         PfUnit x;
         PfSchedule S;
-        const int n = unit_schedule(k, x, S);
-        if (n == -2) break;
+        const int n = unit_schedule(u, x, S);
         if (n == 0) continue;
         li_end = li + 2 * n;
         ok = mbar_wait_cluster(bar_q_ready, qu & 1, abort_flag, P.timeout_ns, 0x85u);
@@ -302,10 +373,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       return __all_sync(0xffffffffu, good);
     };
     for (int k = 0; ok; ++k) {
+      int u;
+      if (!__all_sync(0xffffffffu, uq_get(k, u, 0x91u))) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      if (lane == 0) uq_release(k);
+      if (u < 0) break;
       PfUnit x;
       PfSchedule S;
-      const int n = unit_schedule(k, x, S);
-      if (n == -2) break;
+      const int n = unit_schedule(u, x, S);
       if (n == 0) continue;
       if (!__all_sync(0xffffffffu, mbar_wait(bar_q, qu & 1, abort_flag, P.timeout_ns, 0x87u))) {
         ok = false;
@@ -342,10 +420,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     int jg = 0, qu = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
+      int u;
+      if (!__all_sync(0xffffffffu, uq_get(k, u, 0x91u))) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      if (lane == 0) uq_release(k);
+      if (u < 0) break;
       PfUnit x;
       PfSchedule S;
-      const int n = unit_schedule(k, x, S);
-      if (n == -2) break;
+      const int n = unit_schedule(u, x, S);
       if (n == 0) continue;
       const int h = x.kvh * 4 + x.hp * 2 + (int)rank;
       const int qp = S.qp0 + r;

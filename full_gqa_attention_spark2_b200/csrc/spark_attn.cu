@@ -730,11 +730,9 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   const long long blocks = (long long)B * spark::kNq * P.n_qt;
   if (blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");
   if (kPersistentPrefill && !k_cache) {
-    // one resident cluster per SM pair walks the units (two query heads x one 128-query tile)
-    const long long unit_pairs = (long long)B * 8 * ((P.n_qt + 1) / 2);
-    const long long sm_pairs = g_dev[dev].sm_count / 2;
-    const unsigned clusters = (unsigned)(unit_pairs < sm_pairs ? unit_pairs : sm_pairs);
-    spark::prefill3_kernel<<<2 * clusters, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
+    // one cluster per unit (two query heads x one 128-query tile); resident clusters take the
+    // units of clusters that have not started (cluster launch control)
+    spark::prefill3_kernel<<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
         qm, km, vm, om, P);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "prefill3_kernel launch");
