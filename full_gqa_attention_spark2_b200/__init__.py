@@ -87,6 +87,11 @@ def _lib():
                                         _P]),
         "spark_attn_prefill_varlen": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _P, ctypes.POINTER(SparkPagedKV), _I,
                                            cfgp, ctypes.c_uint, _P]),
+        "spark_decode_cp_record_bytes": (ctypes.c_size_t, [_I]),
+        "spark_kv_append_cp": (_I, [_P, _P, _I, _I, _P, _P, _I, _P, cfgp, ctypes.c_uint, _P]),
+        "spark_attn_decode_cp_partial": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, cfgp, _P, ctypes.c_size_t,
+                                              ctypes.c_uint, _P]),
+        "spark_attn_decode_cp_merge": (_I, [_P, _P, _P, _I, _I, _P]),
         "spark_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
         "spark_check": (_I, [_P]),
         "spark_last_error": (ctypes.c_char_p, []),
@@ -108,8 +113,9 @@ def exported_symbols():
             "spark_kv_cache_q8_bytes", "spark_kv_append_q8", "spark_decode_q8_workspace_bytes",
             "spark_attn_decode_q8", "spark_kv_append_paged", "spark_decode_paged_workspace_bytes",
             "spark_attn_decode_paged", "spark_rope_apply_varlen", "spark_kv_append_varlen",
-            "spark_attn_prefill_varlen", "spark_selftest_wait_timeout", "spark_check", "spark_last_error",
-            "spark_version"]
+            "spark_attn_prefill_varlen", "spark_decode_cp_record_bytes", "spark_kv_append_cp",
+            "spark_attn_decode_cp_partial", "spark_attn_decode_cp_merge", "spark_selftest_wait_timeout",
+            "spark_check", "spark_last_error", "spark_version"]
 
 
 def _raise(rc: int):
@@ -196,6 +202,49 @@ def spark_attn_prefill(out, q, k, v, gate, k_cache, v_cache, pos0, cfg: SparkLay
     B, T = q.shape[0], q.shape[1]
     _raise(_lib().spark_attn_prefill(po, pq, pk, pv, pg, pkc, pvc, cap, B, T, pp, ctypes.byref(cfg), flags,
                                      _stream(stream)))
+
+
+def spark_decode_cp_record_bytes(B: int) -> int:
+    """Bytes of one rank's context-parallel decode record for B sequences."""
+    return int(_lib().spark_decode_cp_record_bytes(B))
+
+
+def spark_kv_append_cp(k_cache, v_cache, key_off: int, k, v, pos, cfg: SparkLayerCfg, flags: int = 0,
+                       stream=None) -> None:
+    """Append k, v [B, 4, 256] at pos[b] into a rank's shard [B, 4, cap, 256] holding positions key_off.. (rows
+    outside the shard are skipped)."""
+    pkc, pvc = _dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4)
+    pk, pv = _dev(k, "k", ndim=3), _dev(v, "v", ndim=3)
+    pp = _dev(pos, "pos", torch.int32, 1)
+    _raise(_lib().spark_kv_append_cp(pkc, pvc, k_cache.shape[2], key_off, pk, pv, k.shape[0], pp, ctypes.byref(cfg),
+                                     flags, _stream(stream)))
+
+
+def spark_attn_decode_cp_partial(record, q, k_cache, v_cache, key_off: int, pos, cfg: SparkLayerCfg,
+                                 workspace: torch.Tensor, flags: int = 0, stream=None) -> None:
+    """A rank's record (fp32, spark_decode_cp_record_bytes(B) bytes) of decode over its shard of a full layer."""
+    pr = _dev(record, "record", torch.float32)
+    if record.numel() * 4 < spark_decode_cp_record_bytes(q.shape[0]):
+        raise ValueError("record is too small")
+    pq = _dev(q, "q", ndim=3)
+    pkc, pvc = _dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4)
+    pp = _dev(pos, "pos", torch.int32, 1)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    _raise(_lib().spark_attn_decode_cp_partial(pr, pq, pkc, pvc, k_cache.shape[2], key_off, q.shape[0], pp,
+                                               ctypes.byref(cfg), workspace.data_ptr(),
+                                               workspace.numel() * workspace.element_size(), flags,
+                                               _stream(stream)))
+
+
+def spark_attn_decode_cp_merge(out, gate, records, stream=None) -> None:
+    """out [B, 16, 256] from the records of G ranks (records: fp32 [G, record floats], rank order)."""
+    po, pg = _dev(out, "out", ndim=3), _dev(gate, "gate", ndim=2)
+    prs = _dev(records, "records", torch.float32, 2)
+    B = out.shape[0]
+    if records.shape[1] * 4 != spark_decode_cp_record_bytes(B):
+        raise ValueError("records must be [G, spark_decode_cp_record_bytes(B) / 4]")
+    _raise(_lib().spark_attn_decode_cp_merge(po, pg, prs, records.shape[0], B, _stream(stream)))
 
 
 def spark_decode_workspace_bytes(B: int, cap: int, cfg: SparkLayerCfg) -> int:

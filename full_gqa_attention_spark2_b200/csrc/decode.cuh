@@ -50,6 +50,11 @@ struct DecodeParams {
   // lives in page block_table[b * max_pages + r / page] at row r % page
   const int* block_table;
   int max_pages, page_shift, n_pages;
+  // context parallelism (full layers): this cache holds positions key_off ..
+  // key_off + cap - 1 of a cache sharded across ranks (row = position -
+  // key_off); a query sees the rows up to its own position, none when it lies
+  // before the shard.  The partials are always left for decode_cp_reduce_kernel.
+  int key_off, shard;
 };
 
 // TMA coordinates of the 64 keys that start at logical row `row0` of
@@ -112,8 +117,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int p = P.pos[b];
-  const bool bad = p < 0 || p >= kMaxPos || (!P.sliding && p >= P.cap);
-  const int n_keys = bad ? 0 : (P.sliding ? min(p + 1, kWindow) : p + 1);
+  const bool bad = p < 0 || p >= kMaxPos || (!P.sliding && !P.shard && p >= P.cap);
+  const int n_keys = bad ? 0 : (P.sliding ? min(p + 1, kWindow) : min(max(p + 1 - P.key_off, 0), P.cap));
   const int key_begin = split * P.tiles_per_split * kDecNK;
   const int key_end = min(n_keys, key_begin + P.tiles_per_split * kDecNK);
   const int n_tiles = key_end > key_begin ? (key_end - key_begin + kDecNK - 1) / kDecNK : 0;
@@ -331,7 +336,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       ls += ew[w] * sm_l[w * 4 + hh];
     }
     const long long row = ((long long)b * kNq + g * 4 + hh) * P.n_splits + split;
-    if (P.n_splits == 1) {
+    if (P.n_splits == 1 && !P.shard) {
       // a single split is the whole answer: normalise, gate and store it here
       const float scale = decode_out_scale(ls, P.gate[(long long)b * kNq + g * 4 + hh]);
       __nv_bfloat16* dst = P.out + ((long long)b * kNq + g * 4 + hh) * kHeadDim;
@@ -384,6 +389,69 @@ __global__ void __launch_bounds__(64) decode_combine_kernel(__nv_bfloat16* __res
   packed.x = pack_bf16(acc.x * scale, acc.y * scale);
   packed.y = pack_bf16(acc.z * scale, acc.w * scale);
   reinterpret_cast<uint2*>(out + ((long long)b * kNq + h) * kHeadDim)[threadIdx.x] = packed;
+}
+
+// ------------------------------------------------- context parallelism ----
+// A rank's record of one layer's decode: for every (sequence b, q head h) its
+// attention output over the keys it holds, normalised, and the log-sum-exp of
+// those keys' logits in base 2 (logits scaled by log2(e)/16, the kernels'
+// exponent domain; -inf when the rank holds none).  Layout: o [B][16][256]
+// then lse [B][16], fp32, cp_record_floats(B) floats.
+__host__ __device__ constexpr long long cp_record_floats(int B) { return (long long)B * kNq * (kHeadDim + 1); }
+
+__global__ void __launch_bounds__(64) decode_cp_reduce_kernel(float* __restrict__ rec, const float* __restrict__ o_part,
+                                                              const float* __restrict__ ml_part, int n_splits, int B) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const long long row0 = ((long long)b * kNq + h) * n_splits;
+  float ms = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) ms = fmaxf(ms, ml_part[(row0 + s) * 2]);
+  float ls = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < n_splits; ++s) {
+    const float m = ml_part[(row0 + s) * 2];
+    const float e = (m == -INFINITY) ? 0.f : fast_exp2(m - ms);
+    ls += e * ml_part[(row0 + s) * 2 + 1];
+    const float4 v = reinterpret_cast<const float4*>(o_part + (row0 + s) * kHeadDim)[threadIdx.x];
+    acc.x += e * v.x;
+    acc.y += e * v.y;
+    acc.z += e * v.z;
+    acc.w += e * v.w;
+  }
+  const float inv = ls > 0.f ? 1.f / ls : 0.f;
+  const long long bh = (long long)b * kNq + h;
+  reinterpret_cast<float4*>(rec + bh * kHeadDim)[threadIdx.x] =
+      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (threadIdx.x == 0) rec[(long long)B * kNq * kHeadDim + bh] = ls > 0.f ? ms + log2f(ls) : -INFINITY;
+}
+
+// out = (sum over ranks of 2^(lse_r - M) o_r) / (sum of 2^(lse_r - M)) * sigmoid(gate), M the
+// largest lse; recs holds G records back to back (rank order, as an all-gather lays them out).
+__global__ void __launch_bounds__(64) decode_cp_merge_kernel(__nv_bfloat16* __restrict__ out,
+                                                             const __nv_bfloat16* __restrict__ gate,
+                                                             const float* __restrict__ recs, int G, int B) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const long long bh = (long long)b * kNq + h;
+  const long long stride = cp_record_floats(B);
+  const long long lse_at = (long long)B * kNq * kHeadDim + bh;
+  float M = -INFINITY;
+  for (int r = 0; r < G; ++r) M = fmaxf(M, recs[r * stride + lse_at]);
+  float W = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int r = 0; r < G; ++r) {
+    const float l = recs[r * stride + lse_at];
+    const float w = (l == -INFINITY) ? 0.f : fast_exp2(l - M);
+    W += w;
+    const float4 v = reinterpret_cast<const float4*>(recs + r * stride + bh * kHeadDim)[threadIdx.x];
+    acc.x += w * v.x;
+    acc.y += w * v.y;
+    acc.z += w * v.z;
+    acc.w += w * v.w;
+  }
+  const float scale = decode_out_scale(W, gate[bh]);
+  uint2 packed;
+  packed.x = pack_bf16(acc.x * scale, acc.y * scale);
+  packed.y = pack_bf16(acc.z * scale, acc.w * scale);
+  reinterpret_cast<uint2*>(out + bh * kHeadDim)[threadIdx.x] = packed;
 }
 
 }  // namespace spark

@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
     uint8_t* __restrict__ k_codes, __half* __restrict__ k_scales, uint8_t* __restrict__ v_codes,
     __half* __restrict__ v_scales, int cap, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, int B, int T, int t_first, const int* __restrict__ pos0, int sliding,
-    int rope, const RopeFreq rf, int rot, CachePages pages, const int* __restrict__ cu) {
+    int rope, const RopeFreq rf, int rot, CachePages pages, const int* __restrict__ cu, int key_off, int shard) {
   __shared__ float xs[2][kNkv * kHeadDim + kNkv * kHeadDim / 32];
   const int b = blockIdx.y;
   const int tid = threadIdx.x;
@@ -71,12 +71,13 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
   const int t = sp.t_first + blockIdx.x;
   if (t >= sp.T) return;
   const int p0 = pos0[b];
-  const bool bad = p0 < 0 || p0 > kMaxPos - sp.T || (!sliding && p0 + sp.T > cap);
+  const bool bad = p0 < 0 || p0 > kMaxPos - sp.T || (!sliding && !shard && p0 + sp.T > cap);
   if (bad) {
     if (blockIdx.x == 0 && tid == 0) raise_error(kErrPosition, 0x400u | (unsigned)b);
     return;
   }
   const int pos = p0 + t;
+  if (shard && (pos - key_off < 0 || pos - key_off >= cap)) return;   // another rank's position
   const long long src = (sp.tok0 + t) * kNkv * kHeadDim;
   // thread = one 16-byte chunk (8 dims) of K and of V: head tid / 32, dims 8 (tid % 32) ..
   {
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
     w[e >> 2] |= u << (8 * (e & 3));
   }
   const int h = hb >> 3, bl = hb & 7;
-  const int row = sliding ? (pos & (kWindow - 1)) : pos;
+  const int row = sliding ? (pos & (kWindow - 1)) : pos - key_off;
   const long long crow = cache_row(pages, b, h, cap, row);
   if (crow < 0) {                        // a page index outside the pool
     if (tid == 0) raise_error(kErrPosition, 0x800u | (unsigned)b);
@@ -217,8 +218,8 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int p = P.pos[b];
-  const bool bad = p < 0 || p >= kMaxPos || (!P.sliding && p >= P.cap);
-  const int n_keys = bad ? 0 : (P.sliding ? min(p + 1, kWindow) : p + 1);
+  const bool bad = p < 0 || p >= kMaxPos || (!P.sliding && !P.shard && p >= P.cap);
+  const int n_keys = bad ? 0 : (P.sliding ? min(p + 1, kWindow) : min(max(p + 1 - P.key_off, 0), P.cap));
   const int key_begin = split * P.tiles_per_split * kQ8NK;
   const int key_end = min(n_keys, key_begin + P.tiles_per_split * kQ8NK);
   const int n_tiles = key_end > key_begin ? (key_end - key_begin + kQ8NK - 1) / kQ8NK : 0;
@@ -483,7 +484,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       ls += ew[w] * sm_l[w * 4 + hh];
     }
     const long long row = ((long long)b * kNq + g * 4 + hh) * P.n_splits + split;
-    if (P.n_splits == 1) {
+    if (P.n_splits == 1 && !P.shard) {
       // a single split is the whole answer: normalise, gate and store it here
       const float scale = decode_out_scale(ls, P.gate[(long long)b * kNq + g * 4 + hh]);
       __nv_bfloat16* dst = P.out + ((long long)b * kNq + g * 4 + hh) * kHeadDim;

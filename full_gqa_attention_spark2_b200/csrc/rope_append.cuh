@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(128) kv_append_kernel(
     __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache, int cap,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int B, int T,
     int t_first, const int* __restrict__ pos0, int sliding, int rope, const RopeFreq rf, int rot,
-    CachePages pages, const int* __restrict__ cu) {
+    CachePages pages, const int* __restrict__ cu, int key_off, int shard) {
   const int b = blockIdx.y;
   const int h = threadIdx.x >> 5;
   const int ch = threadIdx.x & 31;
@@ -152,13 +152,15 @@ __global__ void __launch_bounds__(128) kv_append_kernel(
   const int t = sp.t_first + blockIdx.x;
   if (t >= sp.T) return;
   const int p0 = pos0[b];
-  const bool bad = p0 < 0 || p0 > kMaxPos - sp.T || (!sliding && p0 + sp.T > cap);
+  const bool bad = p0 < 0 || p0 > kMaxPos - sp.T || (!sliding && !shard && p0 + sp.T > cap);
   if (bad) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(kErrPosition, 0x200u | (unsigned)b);
     return;
   }
   const int pos = p0 + t;
-  const int row = sliding ? (pos & (kWindow - 1)) : pos;
+  // full layers: row = position - key_off (0 unless the cache is one rank's shard of positions)
+  const int row = sliding ? (pos & (kWindow - 1)) : pos - key_off;
+  if (shard && (row < 0 || row >= cap)) return;   // another rank's position
   const long long src = ((sp.tok0 + t) * kNkv + h) * kHeadDim;
   const long long crow = cache_row(pages, b, h, cap, row);
   if (crow < 0) {                        // a page index outside the pool

@@ -326,8 +326,11 @@ int check_view(const CacheView& c, const spark_layer_cfg* cfg) {
 
 // cu_seqlens == nullptr: k/v [B][T][4][256].  Otherwise packed [total][4][256]
 // with sequence b at rows cu_seqlens[b] .. cu_seqlens[b+1]-1 and T the longest.
+// key_off / shard: the cache holds positions key_off .. key_off + cap - 1 of a
+// full layer sharded across ranks; tokens outside that range are skipped.
 int append_impl(const CacheView& c, const void* k, const void* v, int B, int T, const int* pos0,
-                const spark_layer_cfg* cfg, unsigned flags, void* stream, const int* cu_seqlens = nullptr) {
+                const spark_layer_cfg* cfg, unsigned flags, void* stream, const int* cu_seqlens = nullptr,
+                int key_off = 0, int shard = 0) {
   int rc = check_view(c, cfg);
   if (rc) return rc;
   if (!k || !v || !pos0) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
@@ -345,11 +348,11 @@ int append_impl(const CacheView& c, const void* k, const void* v, int B, int T, 
     spark::kv_append_q8_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
         (uint8_t*)c.k, (__half*)c.ks, (uint8_t*)c.v, (__half*)c.vs, c.cap, (const __nv_bfloat16*)k,
         (const __nv_bfloat16*)v, B, T, t_first, pos0, sliding, rope, rope_freq(cfg), cfg->rot_dim, pages_of(c),
-        cu_seqlens);
+        cu_seqlens, key_off, shard);
   } else {
     spark::kv_append_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
         (__nv_bfloat16*)c.k, (__nv_bfloat16*)c.v, c.cap, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, B, T,
-        t_first, pos0, sliding, rope, rope_freq(cfg), cfg->rot_dim, pages_of(c), cu_seqlens);
+        t_first, pos0, sliding, rope, rope_freq(cfg), cfg->rot_dim, pages_of(c), cu_seqlens, key_off, shard);
   }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, c.q8() ? "kv_append_q8_kernel launch" : "kv_append_kernel launch");
@@ -412,10 +415,17 @@ int decode_maps(const CacheView& c, int B, CUtensorMap* km, CUtensorMap* vm, CUt
   return SPARK_OK;
 }
 
+// record != nullptr: context parallelism (a full layer's cache is one rank's
+// shard, positions key_off ..): no output, this rank's record is written instead.
 int decode_impl(void* out, const void* q, const void* gate, const CacheView& c, int B, const int* pos,
-                const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes, unsigned flags, void* stream) {
+                const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes, unsigned flags, void* stream,
+                int key_off = 0, float* record = nullptr) {
   int rc = check_view(c, cfg);
   if (rc) return rc;
+  if (record) {
+    out = record;                      // checked below like an output
+    gate = record;
+  }
   if (!out || !q || !gate || !pos || !workspace) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
   if (B <= 0 || B > 65535) return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d", B);
   if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
@@ -452,6 +462,12 @@ int decode_impl(void* out, const void* q, const void* gate, const CacheView& c, 
   P.max_pages = c.max_pages;
   P.page_shift = c.paged() ? ilog2(c.page) : 0;
   P.n_pages = c.n_pages;
+  P.key_off = key_off;
+  P.shard = record ? 1 : 0;
+  if (record) {
+    P.out = nullptr;
+    P.gate = nullptr;
+  }
   dim3 grid(pl.n_splits, spark::kNkv, B);
   cudaStream_t st = (cudaStream_t)stream;
   const char* what;
@@ -470,11 +486,25 @@ int decode_impl(void* out, const void* q, const void* gate, const CacheView& c, 
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, what);
+  if (record) {
+    spark::decode_cp_reduce_kernel<<<dim3(spark::kNq, B), 64, 0, st>>>(record, P.o_part, P.ml_part, pl.n_splits, B);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_cp_reduce_kernel launch");
+  }
   if (pl.n_splits == 1) return SPARK_OK;      // the split kernel wrote the output itself
   spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, st>>>(
       (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
   e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_combine_kernel launch");
+}
+
+// ------------------------------------------------- context parallelism ----
+int check_cp_shard(int cap, int key_off, const spark_layer_cfg* cfg) {
+  if (cfg->kind != SPARK_FULL)
+    return fail(SPARK_ERR_UNSUPPORTED, "context parallelism shards full layers only (sliding layers hold 512 rows)");
+  if (key_off < 0 || key_off >= SPARK_MAX_POSITION || cap <= 0 || cap > SPARK_MAX_POSITION - key_off)
+    return fail(SPARK_ERR_INVALID_ARG, "shard of %d rows at %d outside [0, 2^20)", cap, key_off);
+  return SPARK_OK;
 }
 
 // ------------------------------------------------- decode without workspace ----
@@ -910,6 +940,7 @@ int spark_attn_decode_static(void* out, const void* q, const void* gate, const v
   P.gate = (const __nv_bfloat16*)gate;
   P.block_table = nullptr;
   P.max_pages = P.page_shift = P.n_pages = 0;
+  P.key_off = P.shard = 0;
   spark::decode_partial_kernel<false><<<dim3(pl.n_splits, spark::kNkv, B), spark::kDecThreads, spark::kDecSmemBytes,
                                  (cudaStream_t)stream>>>(km, vm, P);
   cudaError_t e = cudaGetLastError();
@@ -944,6 +975,44 @@ int spark_check(void* stream) {
   if (word & spark::kErrPosition)
     return fail(SPARK_ERR_DEVICE_ARG, "a position failed its device-side check (site 0x%x)", info);
   return SPARK_OK;
+}
+
+// ------------------------------------------------- context parallelism ----
+size_t spark_decode_cp_record_bytes(int B) {
+  if (B <= 0 || B > 65535) return 0;
+  return (size_t)spark::cp_record_floats(B) * sizeof(float);
+}
+
+int spark_kv_append_cp(void* k_cache, void* v_cache, int cap, int key_off, const void* k, const void* v, int B,
+                       const int* pos, const spark_layer_cfg* cfg, unsigned flags, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if ((rc = check_cp_shard(cap, key_off, cfg))) return rc;
+  return append_impl(dense_view(k_cache, v_cache, nullptr, nullptr, cap), k, v, B, 1, pos, cfg, flags, stream,
+                     nullptr, key_off, 1);
+}
+
+int spark_attn_decode_cp_partial(void* record, const void* q, const void* k_cache, const void* v_cache, int cap,
+                                 int key_off, int B, const int* pos, const spark_layer_cfg* cfg, void* workspace,
+                                 size_t ws_bytes, unsigned flags, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if ((rc = check_cp_shard(cap, key_off, cfg))) return rc;
+  if (!record) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  return decode_impl(nullptr, q, nullptr, dense_view((void*)k_cache, (void*)v_cache, nullptr, nullptr, cap), B, pos,
+                     cfg, workspace, ws_bytes, flags, stream, key_off, (float*)record);
+}
+
+int spark_attn_decode_cp_merge(void* out, const void* gate, const void* records, int G, int B, void* stream) {
+  if (!out || !gate || !records) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B > 65535 || G <= 0 || G > 1024) return fail(SPARK_ERR_INVALID_ARG, "bad shape G=%d B=%d", G, B);
+  if (!aligned16(out) || !aligned16(records)) return fail(SPARK_ERR_INVALID_ARG, "out and records must be 16-byte aligned");
+  int rc, dev;
+  if ((rc = device_ready(&dev))) return rc;
+  spark::decode_cp_merge_kernel<<<dim3(spark::kNq, B), 64, 0, (cudaStream_t)stream>>>(
+      (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, (const float*)records, G, B);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_cp_merge_kernel launch");
 }
 
 }  // extern "C"

@@ -295,6 +295,49 @@ int spark_attn_prefill_varlen(void* out, const void* q, const void* k, const voi
                               const spark_paged_kv* history, int B, const spark_layer_cfg* cfg, unsigned flags,
                               void* stream);
 
+/* Context-parallel decode of a full layer (no counterpart on the pages, which
+ * give the 1M-position context, "Spark-X2.6-4B-FP8 W8A8" page §一, and note
+ * that decode is bound by reading the KV cache, "星火 X2.5-4B F16 与 Q4 实测对比"
+ * page §三; splitting one sequence's cache across GPUs is this library's way to
+ * read it with several GPUs' bandwidth).  The cache of a full layer is sharded
+ * by position: a rank's k_cache / v_cache [B][4][cap][256] holds positions
+ * key_off .. key_off + cap - 1 (row = position - key_off).  Sliding layers are
+ * not sharded (SPARK_ERR_UNSUPPORTED): each rank keeps the whole 512-row ring
+ * and runs spark_attn_decode.  One decode step of a full layer on G ranks:
+ *   1. spark_kv_append_cp on every rank (only the rank holding pos[b] writes
+ *      token b; the others skip it);
+ *   2. spark_attn_decode_cp_partial on every rank: its record;
+ *   3. all-gather of the records (rank order, back to back);
+ *   4. spark_attn_decode_cp_merge on every rank (or on the one that needs out).
+ * The result equals spark_attn_decode over the whole cache up to rounding. */
+
+/* Bytes of one rank's record for B sequences: fp32 o [B][16][256] (the rank's
+ * attention output over its keys, normalised) followed by fp32 lse [B][16] (the
+ * log-sum-exp of those keys' logits in base 2, of q.k / 16 * log2(e); -inf when
+ * the rank holds none of a sequence's visible keys).  0 on bad B. */
+size_t spark_decode_cp_record_bytes(int B);
+
+/* spark_kv_append of one token per sequence (k, v [B][4][256], position
+ * pos[b]) into a rank's shard: written at row pos[b] - key_off when that row is
+ * in [0, cap), skipped otherwise.  With SPARK_ROPE_FUSED k is rotated at
+ * pos[b].  0 <= key_off, key_off + cap <= 2^20. */
+int spark_kv_append_cp(void* k_cache, void* v_cache, int cap, int key_off, const void* k, const void* v,
+                       int B, const int* pos, const spark_layer_cfg* cfg, unsigned flags, void* stream);
+
+/* A rank's part of spark_attn_decode: q [B][16][256] (raw with
+ * SPARK_ROPE_FUSED, rotated at pos[b]) against the shard's rows for positions
+ * key_off .. min(pos[b], key_off + cap - 1) (none when pos[b] < key_off);
+ * writes the record (spark_decode_cp_record_bytes(B) bytes, 16-byte aligned).
+ * workspace: at least spark_decode_workspace_bytes(B, cap, cfg) bytes. */
+int spark_attn_decode_cp_partial(void* record, const void* q, const void* k_cache, const void* v_cache,
+                                 int cap, int key_off, int B, const int* pos, const spark_layer_cfg* cfg,
+                                 void* workspace, size_t ws_bytes, unsigned flags, void* stream);
+
+/* Merge the records of G ranks (records: G records back to back, 16-byte
+ * aligned) into out [B][16][256] bf16: the log-sum-exp weighted mean of the
+ * ranks' outputs, times sigmoid(gate [B][16]). */
+int spark_attn_decode_cp_merge(void* out, const void* gate, const void* records, int G, int B, void* stream);
+
 /* Self-test of the failure-detection path: launches one block that waits,
  * with the same bounded wait every kernel of the library uses, on a barrier
  * phase that nothing completes.  The wait runs out after timeout_ns
