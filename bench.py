@@ -251,7 +251,9 @@ def run_prefill(torch, sa, synth, dist, args, peaks, world):
     achieved = f_full / (kern_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
 
-    # end to end: pinned host inputs -> device, the path, outputs -> pinned host
+    # end to end: pinned host inputs -> device, the path, outputs -> pinned host, every step.
+    # Pipelined across steps with two sets of device buffers: the copy-in of step i+1 and the
+    # copy-out of step i-1 run on their own streams while step i computes (PCIe is full duplex).
     host_in = {kind: {n: torch.empty(W[kind][n].shape, dtype=torch.bfloat16, pin_memory=True)
                       for n in ("q", "k", "v", "g")} for kind in W}
     host_out = {kind: torch.empty(W[kind]["out"].shape, dtype=torch.bfloat16, pin_memory=True) for kind in W}
@@ -260,18 +262,51 @@ def run_prefill(torch, sa, synth, dist, args, peaks, world):
             host_in[kind][n].copy_(W[kind][n])
     h2d = sum(t.numel() * 2 for kind in W for t in host_in[kind].values())
     d2h = sum(t.numel() * 2 for t in host_out.values())
+    W2 = {kind: dict(W[kind], **{n: torch.empty_like(W[kind][n]) for n in ("q", "k", "v", "g", "out", "kc", "vc")})
+          for kind in W}
+    bufs = (W, W2)
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-    def e2e_step(i):
-        for kind in W:
-            for n in ("q", "k", "v", "g"):
-                W[kind][n].copy_(host_in[kind][n], non_blocking=True)
-        prefill_step(sa, W, pos0)
-        for kind in W:
-            host_out[kind].copy_(W[kind]["out"], non_blocking=True)
+    def e2e_pipeline(steps):
+        ev_in = [torch.cuda.Event() for _ in range(steps)]
+        ev_cmp = [torch.cuda.Event() for _ in range(steps)]
+        ev_out = [torch.cuda.Event() for _ in range(steps)]
 
+        def step(i):
+            cur = torch.cuda.current_stream()
+            if i == 0:
+                for st in (s_in, s_cmp, s_out):
+                    st.wait_stream(cur)
+            Wi = bufs[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_cmp[i - 2])          # step i-2 has read these inputs
+                for kind in Wi:
+                    for n in ("q", "k", "v", "g"):
+                        Wi[kind][n].copy_(host_in[kind][n], non_blocking=True)
+                ev_in[i].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in[i])
+                if i >= 2:
+                    s_cmp.wait_event(ev_out[i - 2])         # step i-2's output has been copied out
+                prefill_step(sa, Wi, pos0)
+                ev_cmp[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[i])
+                for kind in Wi:
+                    host_out[kind].copy_(Wi[kind]["out"], non_blocking=True)
+                ev_out[i].record(s_out)
+            if i == steps - 1:
+                cur.wait_event(ev_out[i])
+        return step
+
+    warm = e2e_pipeline(2)
+    warm(0)
+    warm(1)
+    torch.cuda.synchronize()
     e2e_steps = max(3, min(args.steps, 10))
-    e2e_step(0)
-    ms_e2e = timed_region(torch, dist, e2e_step, e2e_steps)
+    ms_e2e = timed_region(torch, dist, e2e_pipeline(e2e_steps), e2e_steps)
+    del W2, bufs
     sa.spark_check()
     del W
     torch.cuda.empty_cache()
