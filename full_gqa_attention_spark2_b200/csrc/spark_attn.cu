@@ -167,9 +167,6 @@ int make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, 
                     box);
 }
 
-// Dense prefill without a cache runs the persistent kernel (prefill3).
-constexpr bool kPersistentPrefill = true;
-
 // -------------------------------------------------------------- RoPE tables ----
 // f_i = theta^(-2i/rot) of the two layer kinds, computed once on the host in
 // double precision and passed in the kernel parameters (no device memory;
@@ -759,9 +756,10 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   P.max_pages = P.page_shift = P.n_pages = 0;
   const long long blocks = (long long)B * spark::kNq * P.n_qt;
   if (blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");
-  if (kPersistentPrefill && !k_cache) {
-    // one cluster per unit (two query heads x one 128-query tile); resident clusters take the
-    // units of clusters that have not started (cluster launch control)
+  if (!k_cache) {
+    // no history: the persistent kernel.  One cluster per unit (two query heads x one 128-query
+    // tile); resident clusters take the units of clusters that have not started (cluster launch
+    // control)
     spark::prefill3_kernel<<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
         qm, km, vm, om, P);
     cudaError_t e = cudaGetLastError();
