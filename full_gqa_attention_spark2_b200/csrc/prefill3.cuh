@@ -435,6 +435,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       const int h = x.kvh * 4 + x.hp * 2 + (int)rank;
       const int qp = S.qp0 + r;
       const bool row_valid = qp < S.pos0 + S.T;
+      // the row's gate logit, read now (its latency hides behind the unit) and used at the epilogue
+      const float gl =
+          row_valid ? __bfloat162float(P.gate[((long long)x.b * P.T + (qp - S.pos0)) * kNq + h]) : 0.f;
       float m_ref = -INFINITY, l_run = 0.f;
       for (int j = 0; j < n && ok; ++j) {
         const int jgl = jg + j;
@@ -537,19 +540,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         break;
       }
       tc_fence_after();
-      float scale = 0.f;
-      if (row_valid) {
-        const long long tok = (long long)x.b * P.T + (qp - S.pos0);
-        const float gl = __bfloat162float(P.gate[tok * kNq + h]);
-        scale = (l_run > 0.f ? 1.f / l_run : 0.f) * (1.f / (1.f + expf(-gl)));
-      }
+      const float scale = row_valid ? (l_run > 0.f ? 1.f / l_run : 0.f) * (1.f / (1.f + expf(-gl))) : 0.f;
       const int li_end = 2 * (jg + n);
       uint8_t* const gslots = gbase + kPfQBytes;
-#pragma unroll 1
-      for (int cc = 0; cc < 8; ++cc) {
-        uint32_t ov[32];
-        tmem_ld32(ocol + 32 * cc, ov);
-        tmem_wait_ld();
+      auto stage = [&](const uint32_t* ov, int cc) {
         uint8_t* box = gslots + ((li_end - 2 + (cc >> 2)) % kP2Slots) * kP2SlotBytes + ((cc >> 1) & 1) * 16384 + r * 128;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -561,16 +555,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
           const int chunk = (cc & 1) * 4 + e;     // 16-byte chunk within the 128-byte row of the box
           *reinterpret_cast<uint4*>(box + ((chunk ^ (r & 7)) << 4)) = w;
         }
+      };
+      // two 32-column reads of O in flight: chunk cc+1 loads while chunk cc is staged
+      uint32_t ova[32], ovb[32];
+      tmem_ld32(ocol, ova);
+#pragma unroll 1
+      for (int cc = 0; cc < 8; cc += 2) {
+        tmem_wait_ld();
+        tmem_ld32(ocol + 32 * (cc + 1), ovb);
+        stage(ova, cc);
+        tmem_wait_ld();
+        if (cc + 2 < 8) {
+          tmem_ld32(ocol + 32 * (cc + 2), ova);
+        } else {
+          // every read of O has landed: the next unit's first P.V may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (leader) mbar_arrive(bar_o_free);
+            else mbar_arrive_remote(o_free0);
+          }
+        }
+        stage(ovb, cc + 1);
       }
-      // O has been read: the next unit's first P.V may overwrite it
-      tc_fence_before();
       fence_proxy_async_smem();                   // make the staged rows visible to the TMA store
       __syncwarp();
-      if (lane == 0) {
-        if (leader) mbar_arrive(bar_o_free);
-        else mbar_arrive_remote(o_free0);
-        mbar_arrive(bar_o_staged);
-      }
+      if (lane == 0) mbar_arrive(bar_o_staged);
       jg += n;
       ++qu;
     }
