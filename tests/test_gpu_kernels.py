@@ -288,6 +288,15 @@ def test_prefill_batch_of_two(kind):
     assert_close(got, ref, f"prefill {KIND_NAME[kind]} B=2")
 
 
+@pytest.mark.parametrize("kind", KINDS)
+def test_prefill_more_units_than_resident_clusters(kind):
+    """B=5 x 773 tokens: 5 * 8 * 7 = 280 units (two query heads x one 128-query tile each) for about
+    74 resident SM pairs, so most units run in clusters that took them from clusters that never
+    started; every element is checked, with an odd tile count and a ragged last tile."""
+    got, ref = _prefill_case(kind, 5, 773, [0] * 5, seed=21)
+    assert_close(got, ref, f"prefill {KIND_NAME[kind]} B=5 T=773")
+
+
 @pytest.mark.parametrize("kind,T,pos0", [(O.SLIDING, 256, 512), (O.SLIDING, 200, 700), (O.SLIDING, 130, 1000),
                                          (O.FULL, 256, 512), (O.FULL, 100, 333), (O.FULL, 129, 1)])
 def test_prefill_with_history(kind, T, pos0):

@@ -52,10 +52,15 @@ def test_prefill_b4_t8192_sampled_rows():
                                      rng.integers(0, T, 4)]))
     for kind, layer in ((O.SLIDING, 0), (O.FULL, 3)):
         w = W[kind]
+        w["out"].fill_(float("nan"))
         sa.spark_rope_apply(w["k"], pos0, w["cfg"])                  # as in bench.prefill_step:
         sa.spark_attn_prefill(w["out"], w["q"], w["k"], w["v"], w["g"], None, None, pos0, w["cfg"],
                               flags=sa.SPARK_ROPE_FUSED)              # q raw, rotated at load
         sa.spark_check()
+        # every element written (no unit skipped or stored twice by the dynamic scheduling), and each
+        # output a gated convex combination of v rows: |out| <= max |v|
+        assert bool(torch.isfinite(w["out"]).all()), f"kind={kind}: unwritten or non-finite outputs"
+        assert float(w["out"].abs().max()) <= float(w["v"].abs().max()) * (1 + 2 ** -7)
         for b in (0, 3):
             got = dev_to_f64(w["out"][b, torch.as_tensor(rows, device=dev)])
             for g in range(4):
