@@ -56,6 +56,11 @@ __device__ __forceinline__ void rope_angle(int pos, double f, float& c, float& s
 // longest).
 constexpr int kRopeIters = 8;
 
+// kAllHeads (q, 16 heads): all heads' pairs are loaded before any is stored, so sixteen loads
+// are in flight together (3x faster on full layers than one head at a time).  k's four heads go
+// one at a time: there the separate instantiation keeps fewer registers and more warps resident,
+// which measured faster.
+template <bool kAllHeads>
 __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x, int B, int T,
                                                    int H, const int* __restrict__ pos0,
                                                    const RopeFreq rf, int rot, const int* __restrict__ cu) {
@@ -95,13 +100,29 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
     rope_angle(pos, freq[2 * j], c0, s0);
     rope_angle(pos, freq[2 * j + 1], c1, s1);
     __nv_bfloat16* row = x + n * H * kHeadDim;
-    for (int h = 0; h < H; ++h) {
-      uint32_t* lo_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + 2 * j);
-      uint32_t* hi_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + half + 2 * j);
-      uint32_t lo = *lo_p, hi = *hi_p;
-      float l0 = bf16_lo(lo), l1 = bf16_hi(lo), h0 = bf16_lo(hi), h1 = bf16_hi(hi);
-      *lo_p = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
-      *hi_p = pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);
+    if constexpr (kAllHeads) {
+      uint32_t lo[16], hi[16];
+#pragma unroll
+      for (int h = 0; h < 16; ++h) {
+        lo[h] = *reinterpret_cast<const uint32_t*>(row + h * kHeadDim + 2 * j);
+        hi[h] = *reinterpret_cast<const uint32_t*>(row + h * kHeadDim + half + 2 * j);
+      }
+#pragma unroll
+      for (int h = 0; h < 16; ++h) {
+        const float l0 = bf16_lo(lo[h]), l1 = bf16_hi(lo[h]), h0 = bf16_lo(hi[h]), h1 = bf16_hi(hi[h]);
+        *reinterpret_cast<uint32_t*>(row + h * kHeadDim + 2 * j) = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
+        *reinterpret_cast<uint32_t*>(row + h * kHeadDim + half + 2 * j) =
+            pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);
+      }
+    } else {
+      for (int h = 0; h < H; ++h) {
+        uint32_t* lo_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + 2 * j);
+        uint32_t* hi_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + half + 2 * j);
+        uint32_t lo = *lo_p, hi = *hi_p;
+        float l0 = bf16_lo(lo), l1 = bf16_hi(lo), h0 = bf16_lo(hi), h1 = bf16_hi(hi);
+        *lo_p = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
+        *hi_p = pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);
+      }
     }
   }
 }

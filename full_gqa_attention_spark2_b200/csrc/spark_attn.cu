@@ -601,8 +601,12 @@ int spark_rope_apply(void* x, int B, int T, int H, const int* pos0, const spark_
   const long long n = (long long)B * T;
   const long long grid = (n + tok_per_block - 1) / tok_per_block;
   if (grid > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "too many tokens");
-  spark::rope_kernel<<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>(
-      (__nv_bfloat16*)x, B, T, H, pos0, rope_freq(cfg), cfg->rot_dim, nullptr);
+  if (H == 16)
+    spark::rope_kernel<true><<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>(
+        (__nv_bfloat16*)x, B, T, H, pos0, rope_freq(cfg), cfg->rot_dim, nullptr);
+  else
+    spark::rope_kernel<false><<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>(
+        (__nv_bfloat16*)x, B, T, H, pos0, rope_freq(cfg), cfg->rot_dim, nullptr);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "rope_kernel launch");
 }
@@ -784,8 +788,12 @@ int spark_rope_apply_varlen(void* x, int H, const int* cu_seqlens, int max_seqle
   if ((rc = device_ready(&dev))) return rc;
   const int tok_per_block = 128 / (cfg->rot_dim / 4) * spark::kRopeIters;
   dim3 grid((max_seqlen + tok_per_block - 1) / tok_per_block, B);
-  spark::rope_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>((__nv_bfloat16*)x, B, max_seqlen, H, pos0,
-                                                              rope_freq(cfg), cfg->rot_dim, cu_seqlens);
+  if (H == 16)
+    spark::rope_kernel<true><<<grid, 128, 0, (cudaStream_t)stream>>>((__nv_bfloat16*)x, B, max_seqlen, H, pos0,
+                                                                    rope_freq(cfg), cfg->rot_dim, cu_seqlens);
+  else
+    spark::rope_kernel<false><<<grid, 128, 0, (cudaStream_t)stream>>>((__nv_bfloat16*)x, B, max_seqlen, H, pos0,
+                                                                     rope_freq(cfg), cfg->rot_dim, cu_seqlens);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "rope_kernel launch");
 }
