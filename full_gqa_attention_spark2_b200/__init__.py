@@ -16,6 +16,7 @@ import torch
 SPARK_SLIDING = 0
 SPARK_FULL = 1
 SPARK_ROPE_FUSED = 1
+SPARK_APPEND_FUSED = 2
 N_LAYERS = 36
 N_Q_HEADS = 16
 N_KV_HEADS = 4

@@ -701,7 +701,9 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
     return fail(SPARK_ERR_INVALID_ARG, "pass both caches or neither");
   if (B <= 0 || B > 65535 || T <= 0 || T > SPARK_MAX_POSITION)
     return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d", B, T);
-  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~(SPARK_ROPE_FUSED | SPARK_APPEND_FUSED)) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if ((flags & SPARK_APPEND_FUSED) && !k_cache)
+    return fail(SPARK_ERR_INVALID_ARG, "SPARK_APPEND_FUSED needs the caches to append to");
   const int sliding = cfg->kind == SPARK_SLIDING;
   if (k_cache) {
     if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
@@ -773,7 +775,12 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   spark::prefill2_kernel<false><<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
       qm, km, vm, kcm, vcm, om, P);
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "prefill2_kernel launch");
+  if (e != cudaSuccess) return cuda_fail(e, "prefill2_kernel launch");
+  if (!(flags & SPARK_APPEND_FUSED)) return SPARK_OK;
+  // the chunk's k (rotated) and v into the cache, after the attention on the same stream: a sliding
+  // ring's rows are overwritten only once the attention has read them as history
+  return append_impl(dense_view((void*)k_cache, (void*)v_cache, nullptr, nullptr, cap), k, v, B, T, pos0, cfg, 0,
+                     stream);
 }
 
 int spark_rope_apply_varlen(void* x, int H, const int* cu_seqlens, int max_seqlen, const int* pos0, int B,

@@ -83,6 +83,7 @@ typedef struct {
 
 /* Flags */
 #define SPARK_ROPE_FUSED 1u  /* the call rotates its raw q (prefill, decode) or k (kv_append) itself */
+#define SPARK_APPEND_FUSED 2u  /* spark_attn_prefill also appends the chunk's k and v to the cache */
 
 /* Parameters of 0-based layer `layer` of the 36-layer stack: layer l is full
  * iff l % 4 == 3 ("3 sliding + 1 full", the last layer full).
@@ -129,9 +130,15 @@ int spark_kv_append(void* k_cache, void* v_cache, int cap, const void* k, const 
  *   positions < pos0[b]) come from the cache: full layers read rows
  *   [0, pos0[b]); sliding layers read the ring rows of positions
  *   [max(0, pos0[b] - 511), pos0[b]).  Pass k_cache = v_cache = NULL when no
- *   sequence has history.  The cache is only read: append the chunk after
- *   this call on sliding layers (the ring rows are still needed here), before
- *   or after it on full layers.
+ *   sequence has history.  Without SPARK_APPEND_FUSED the cache is only read:
+ *   append the chunk after this call on sliding layers (the ring rows are
+ *   still needed here), before or after it on full layers.
+ * With SPARK_APPEND_FUSED (caches required) the call also appends the chunk's k
+ * (as passed: rotated) and v to the cache, as spark_kv_append would, after the
+ * attention on the same stream, so a sliding ring is overwritten only once it
+ * has been read as history.  Without caches (no history) the call runs the
+ * persistent kernel, which is faster on sliding layers; a first chunk is
+ * therefore best attended without caches and appended by spark_kv_append.
  * Device requirements: sm_100a, about 225 KB of shared memory per block. */
 int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, const void* gate,
                        const void* k_cache, const void* v_cache, int cap, int B, int T,

@@ -297,6 +297,42 @@ def test_prefill_more_units_than_resident_clusters(kind):
     assert_close(got, ref, f"prefill {KIND_NAME[kind]} B=5 T=773")
 
 
+@pytest.mark.parametrize("kind,T,pos0_list", [(O.SLIDING, 300, [700, 0]), (O.FULL, 200, [333, 0])])
+def test_prefill_append_fused(kind, T, pos0_list):
+    """SPARK_APPEND_FUSED: the same output as without it, and the cache afterwards bit-identical to an
+    explicit spark_kv_append after the call (sliding: ring rows that were history for this chunk get
+    overwritten only after the attention)."""
+    B = len(pos0_list)
+    cfg = _cfg(kind)
+    sliding = kind == O.SLIDING
+    seed, layer = 9, 0
+    pos = np.array([[p0 + t for t in range(T)] for p0 in pos0_list])
+    q = to_dev(synth.token_tensor(seed, tid(layer, synth.ROLE_Q), B, 16, 256, pos))
+    k = to_dev(synth.token_tensor(seed, tid(layer, synth.ROLE_K), B, 4, 256, pos))
+    v = to_dev(synth.token_tensor(seed, tid(layer, synth.ROLE_V), B, 4, 256, pos))
+    g = to_dev(synth.token_tensor(seed, tid(layer, synth.ROLE_GATE), B, 16, 1, pos))
+    p0 = _pos_tensor(pos0_list)
+    sa.spark_rope_apply(k, p0, cfg)
+    cap = 512 if sliding else max(pos0_list) + T + 3
+    kc = torch.empty(B, 4, cap, 256, dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+    synth.fill_cache(kc, seed, tid(layer, synth.ROLE_K), max(pos0_list), sliding)
+    synth.fill_cache(vc, seed, tid(layer, synth.ROLE_V), max(pos0_list), sliding)
+    kc2, vc2 = kc.clone(), vc.clone()
+    out1 = torch.empty(B, T, 16, 256, dtype=torch.bfloat16, device="cuda")
+    out2 = torch.empty_like(out1)
+    sa.spark_attn_prefill(out1, q, k, v, g, kc, vc, p0, cfg, flags=sa.SPARK_ROPE_FUSED)
+    sa.spark_kv_append(kc, vc, k, v, p0, cfg)
+    sa.spark_attn_prefill(out2, q, k, v, g, kc2, vc2, p0, cfg, flags=sa.SPARK_ROPE_FUSED | sa.SPARK_APPEND_FUSED)
+    sa.spark_check()
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    assert torch.equal(kc.view(torch.int16), kc2.view(torch.int16))
+    assert torch.equal(vc.view(torch.int16), vc2.view(torch.int16))
+    with pytest.raises(sa.SparkError) as e:
+        sa.spark_attn_prefill(out2, q, k, v, g, None, None, p0, cfg, flags=sa.SPARK_APPEND_FUSED)
+    assert e.value.status == -1
+
+
 @pytest.mark.parametrize("kind,T,pos0", [(O.SLIDING, 256, 512), (O.SLIDING, 200, 700), (O.SLIDING, 130, 1000),
                                          (O.FULL, 256, 512), (O.FULL, 100, 333), (O.FULL, 129, 1)])
 def test_prefill_with_history(kind, T, pos0):
