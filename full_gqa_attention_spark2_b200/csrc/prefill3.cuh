@@ -53,7 +53,8 @@ constexpr int kUqReaders = 14;  // per entry: MMA thread, 2 Q warps, 4 softmax w
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     prefill3_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap,
+                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kcmap,
+                    const __grid_constant__ CUtensorMap vcmap, const __grid_constant__ CUtensorMap omap,
                     const PrefillParams P) {
   extern __shared__ uint8_t dsmem[];
   const uint32_t raw = smem_u32(dsmem);
@@ -149,6 +150,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
+      if (P.has_cache) {
+        tma_prefetch_desc(&kcmap);
+        tma_prefetch_desc(&vcmap);
+      }
       const int key_half = 64 * (int)rank;       // this block's keys of a K tile
       const int dim_half = 128 * (int)rank;      // this block's dims of a V tile
       int li = 0, qu = 0;
@@ -222,12 +227,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             if (leader) mbar_arrive_expect_tx(bar_slot_full + 8 * s, 2 * kP2SlotBytes);
             if (is_k) {
               for (int xx = 0; xx < 4; ++xx)
-                tma2_load_4d(dst + xx * 8192, &kmap, full0, xx * 64, x.kvh, t.row + key_half, x.b);
+                if (t.hist)
+                  tma2_load_3d(dst + xx * 8192, &kcmap, full0, xx * 64, t.row + key_half, x.b * kNkv + x.kvh);
+                else
+                  tma2_load_4d(dst + xx * 8192, &kmap, full0, xx * 64, x.kvh, t.row + key_half, x.b);
             } else {
               for (int xx = 0; xx < 4; ++xx)
-                for (int d = 0; d < 2; ++d)
-                  tma2_load_4d(dst + xx * 8192 + d * 4096, &vmap, full0, dim_half + 64 * d, x.kvh, t.row + 32 * xx,
-                               x.b);
+                for (int d = 0; d < 2; ++d) {
+                  if (t.hist)
+                    tma2_load_3d(dst + xx * 8192 + d * 4096, &vcmap, full0, dim_half + 64 * d, t.row + 32 * xx,
+                                 x.b * kNkv + x.kvh);
+                  else
+                    tma2_load_4d(dst + xx * 8192 + d * 4096, &vmap, full0, dim_half + 64 * d, x.kvh, t.row + 32 * xx,
+                                 x.b);
+                }
             }
             ++li;
           }

@@ -762,20 +762,22 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   P.max_pages = P.page_shift = P.n_pages = 0;
   const long long blocks = (long long)B * spark::kNq * P.n_qt;
   if (blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");
-  if (!k_cache) {
-    // no history: the persistent kernel.  One cluster per unit (two query heads x one 128-query
-    // tile); resident clusters take the units of clusters that have not started (cluster launch
-    // control)
+  cudaError_t e;
+  if (!k_cache || sliding) {
+    // the persistent kernel: one cluster per unit (two query heads x one 128-query tile); resident
+    // clusters take the units of clusters that have not started (cluster launch control).  Full
+    // layers with a history (units of hundreds of KV tiles) measured 5-8 % faster in prefill2.
     spark::prefill3_kernel<<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
-        qm, km, vm, om, P);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "prefill3_kernel launch");
+        qm, km, vm, kcm, vcm, om, P);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "prefill3_kernel launch");
+  } else {
+    // clusters of two blocks (an SM pair): two query heads of a KV group, same query tile
+    spark::prefill2_kernel<false><<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes,
+                                    (cudaStream_t)stream>>>(qm, km, vm, kcm, vcm, om, P);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "prefill2_kernel launch");
   }
-  // clusters of two blocks (an SM pair): two query heads of a KV group, same query tile
-  spark::prefill2_kernel<false><<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
-      qm, km, vm, kcm, vcm, om, P);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "prefill2_kernel launch");
   if (!(flags & SPARK_APPEND_FUSED)) return SPARK_OK;
   // the chunk's k (rotated) and v into the cache, after the attention on the same stream: a sliding
   // ring's rows are overwritten only once the attention has read them as history
