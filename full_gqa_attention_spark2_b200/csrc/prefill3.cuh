@@ -15,6 +15,8 @@
 //     as soon as O is staged; the next unit's first P.V (which overwrites O)
 //     waits only until the epilogue has read O out of tensor memory (`o_free`);
 //   - the slot ring, the S buffers and all barrier phases continue across units.
+// History tiles (the chunk's earlier keys in a sliding ring or a full cache)
+// load through the cache's tensor maps, as in prefill2_kernel.
 // The grid has one cluster per unit, in the order of pf_unit_of (per sequence
 // and KV head, the heaviest query tiles first).  A resident cluster takes more
 // units by cancelling clusters that have not started yet (cluster launch
