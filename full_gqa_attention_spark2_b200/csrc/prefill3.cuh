@@ -53,6 +53,9 @@ constexpr int kUq = 8;          // unit queue entries
 constexpr int kUqReaders = 14;  // per entry: MMA thread, 2 Q warps, 4 softmax warps (even block);
                                 // producer, 2 Q warps, 4 softmax warps (odd block)
 
+// kHist: history tiles from the cache (sliding layers with a ring); a separate instantiation, so
+// the kernel without one keeps its smaller code (it is sensitive to instruction-fetch stalls).
+template <bool kHist>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     prefill3_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kcmap,
@@ -152,7 +155,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      if (P.has_cache) {
+      if constexpr (kHist) {
         tma_prefetch_desc(&kcmap);
         tma_prefetch_desc(&vcmap);
       }
@@ -229,14 +232,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             if (leader) mbar_arrive_expect_tx(bar_slot_full + 8 * s, 2 * kP2SlotBytes);
             if (is_k) {
               for (int xx = 0; xx < 4; ++xx)
-                if (t.hist)
+                if (kHist && t.hist)
                   tma2_load_3d(dst + xx * 8192, &kcmap, full0, xx * 64, t.row + key_half, x.b * kNkv + x.kvh);
                 else
                   tma2_load_4d(dst + xx * 8192, &kmap, full0, xx * 64, x.kvh, t.row + key_half, x.b);
             } else {
               for (int xx = 0; xx < 4; ++xx)
                 for (int d = 0; d < 2; ++d) {
-                  if (t.hist)
+                  if (kHist && t.hist)
                     tma2_load_3d(dst + xx * 8192 + d * 4096, &vcmap, full0, dim_half + 64 * d, t.row + 32 * xx,
                                  x.b * kNkv + x.kvh);
                   else

@@ -94,7 +94,10 @@ int device_ready(int* dev_out) {
       b = cudaFuncSetAttribute(spark::prefill2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                spark::kP2SmemBytes);
     if (b == cudaSuccess)
-      b = cudaFuncSetAttribute(spark::prefill3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      b = cudaFuncSetAttribute(spark::prefill3_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               spark::kP2SmemBytes);
+    if (b == cudaSuccess)
+      b = cudaFuncSetAttribute(spark::prefill3_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                spark::kP2SmemBytes);
     cudaError_t c = cudaFuncSetAttribute(spark::decode_q8_partial_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -767,8 +770,12 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
     // the persistent kernel: one cluster per unit (two query heads x one 128-query tile); resident
     // clusters take the units of clusters that have not started (cluster launch control).  Full
     // layers with a history (units of hundreds of KV tiles) measured 5-8 % faster in prefill2.
-    spark::prefill3_kernel<<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes, (cudaStream_t)stream>>>(
-        qm, km, vm, kcm, vcm, om, P);
+    if (k_cache)
+      spark::prefill3_kernel<true><<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes,
+                                     (cudaStream_t)stream>>>(qm, km, vm, kcm, vcm, om, P);
+    else
+      spark::prefill3_kernel<false><<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes,
+                                      (cudaStream_t)stream>>>(qm, km, vm, kcm, vcm, om, P);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prefill3_kernel launch");
   } else {
