@@ -57,6 +57,17 @@ def prefill_flops(B: int, T: int, pos0: int, kind: int, with_history: bool = Tru
     return B * visible_pairs(T, pos0, kind, with_history) * HQ * 4 * D
 
 
+def prefill_tile_flops(B: int, T: int, kind: int) -> int:
+    """FLOPs the prefill kernels execute for a chunk without history: every 128-query tile against
+    every 128-key tile it touches (diagonal and window-edge tiles in full, masked or not)."""
+    n_qt = (T + 127) // 128
+    tiles = 0
+    for qt in range(n_qt):
+        first = max(0, qt * 128 - (WINDOW - 1)) // 128 if kind == SLIDING else 0
+        tiles += qt - first + 1
+    return B * HQ * tiles * 128 * 128 * 4 * D
+
+
 def decode_kv_bytes(B: int, p: int, kind: int) -> int:
     """Algorithmic KV bytes a decode step reads: visible keys x 4 heads x (K+V) x 256 x 2 B."""
     keys = p + 1 if kind == FULL else min(p + 1, WINDOW)
@@ -185,16 +196,17 @@ def prefill_workload(torch, sa, synth, dev):
 
 def prefill_step(sa, W, pos0, events=None):
     """One pass of the hot path over the batch, for both layer kinds: RoPE on k, the prefill
-    (which rotates its raw q at load), the KV append."""
+    (which rotates its raw q at load), the KV append.  events: {kind: (start, end)} recorded
+    around each kind's prefill launch."""
     for kind in (SLIDING, FULL):
         w = W[kind]
         sa.spark_rope_apply(w["k"], pos0, w["cfg"])
-        if events is not None and kind == FULL:
-            events[0].record()
+        if events is not None:
+            events[kind][0].record()
         sa.spark_attn_prefill(w["out"], w["q"], w["k"], w["v"], w["g"], None, None, pos0, w["cfg"],
                               flags=sa.SPARK_ROPE_FUSED)
-        if events is not None and kind == FULL:
-            events[1].record()
+        if events is not None:
+            events[kind][1].record()
         sa.spark_kv_append(w["kc"], w["vc"], w["k"], w["v"], pos0, w["cfg"])
 
 
@@ -236,13 +248,15 @@ def run_prefill(torch, sa, synth, dist, args, peaks, world):
         prefill_step(sa, W, pos0)
     sa.spark_check()
     # per-launch duration of the full-layer prefill kernel, on its stream
-    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    pairs = [{kind: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for kind in (SLIDING, FULL)} for _ in range(args.steps)]
     clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
     clocks.start()
     ms = timed_region(torch, dist, lambda i: prefill_step(sa, W, pos0, pairs[i]), args.steps)
     clk = clocks.stop()
     sa.spark_check()
-    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+    kern_ms = statistics.mean(ev[FULL][0].elapsed_time(ev[FULL][1]) for ev in pairs)
+    slide_ms = statistics.mean(ev[SLIDING][0].elapsed_time(ev[SLIDING][1]) for ev in pairs)
     B, T = PREFILL_B, PREFILL_T
     f_full = prefill_flops(B, T, 0, FULL, False)
     f_slide = prefill_flops(B, T, 0, SLIDING, False)
@@ -317,6 +331,14 @@ def run_prefill(torch, sa, synth, dist, args, peaks, world):
         "ms_per_step": ms_step,
         "tflops": (f_full + f_slide) * world / (ms_step * 1e-3) / 1e12,
         "prefill_full_kernel": {"ms": kern_ms, "tflops": achieved, "flops": f_full},
+        "per_layer_kind": {
+            name: {"kernel_us": ms * 1e3, "tok_s": B * T / (ms * 1e-3),
+                   "tflops": f / (ms * 1e-3) / 1e12, "algorithmic_flops": f,
+                   "tile_flops": prefill_tile_flops(B, T, kind)}
+            for name, kind, ms, f in (("sliding", SLIDING, slide_ms, f_slide), ("full", FULL, kern_ms, f_full))},
+        "stack36_derived": {"ms": 27 * slide_ms + 9 * kern_ms,
+                            "tok_s": B * T / ((27 * slide_ms + 9 * kern_ms) * 1e-3),
+                            "note": "derived, not measured: 27 sliding + 9 full layer kernels of this step"},
         "roofline": {"bound": "tensor", "kernel": "prefill3_kernel (full layer, persistent SM pairs)", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"bf16_tflops burst, {peaks['source']}",
@@ -912,6 +934,7 @@ def main():
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (q alone is 268 MB per layer); no flush"},
         "tflops": res["tflops"], "prefill_full_kernel": res["prefill_full_kernel"],
+        "per_layer_kind": res["per_layer_kind"], "stack36_derived": res["stack36_derived"],
         "roofline": res["roofline"], "e2e": res["e2e"], "clocks": res["clocks"],
         "gpu_launches": res["gpu_launches"] + (0 if dec is None else 0),
         "cpu_baseline": cpu, "prefill_ragged": ragged, "decode": dec, "decode_q8": dec_q8,
