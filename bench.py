@@ -766,6 +766,67 @@ def run_long_decode(torch, sa, synth, dist, args, peaks, world):
     return out
 
 
+def run_cp_decode(torch, sa, synth, dist, args, peaks, world):
+    """Context-parallel decode, B=1 at 2^20: each full layer's cache split by position over the
+    ranks (append to the owning shard, each rank's record, one all-gather, the merge); the sliding
+    layers replicated on every rank.  The same sequence for every N (strong scaling).  Eager
+    launches: between ranks the exchange is an NCCL all-gather."""
+    from full_gqa_attention_spark2_b200.context_parallel import FullLayerShard
+    dev = torch.device("cuda")
+    B, ctx = 1, 1 << 20
+    p = ctx - 1
+    seed = 5
+    layers = []
+    for l in range(N_LAYERS):
+        kind = FULL if l % 4 == 3 else SLIDING
+        cfg = sa.spark_layer_cfg_for_kind(kind)
+        toks = {}
+        for name, role, H in (("q", synth.ROLE_Q, HQ), ("kn", synth.ROLE_K, HKV), ("vn", synth.ROLE_V, HKV),
+                              ("g", synth.ROLE_GATE, HQ)):
+            t = torch.empty(B, 1, H, *(() if name == "g" else (D,)), dtype=torch.bfloat16, device=dev)
+            synth.fill_tokens(t, seed, synth.tensor_id(l, role), p)
+            toks[name] = t
+        L = dict(kind=kind, cfg=cfg, q=toks["q"].view(B, HQ, D), kn=toks["kn"], vn=toks["vn"],
+                 g=toks["g"].view(B, HQ), out=torch.empty(B, HQ, D, dtype=torch.bfloat16, device=dev))
+        if kind == FULL:
+            L["shard"] = FullLayerShard(B, ctx, cfg, device=dev)
+        else:
+            kc = torch.empty(B, HKV, WINDOW, D, dtype=torch.bfloat16, device=dev)
+            vc = torch.empty_like(kc)
+            synth.fill_cache(kc, seed, synth.tensor_id(l, synth.ROLE_K), p, True)
+            synth.fill_cache(vc, seed, synth.tensor_id(l, synth.ROLE_V), p, True)
+            L.update(kc=kc, vc=vc)
+        layers.append(L)
+    pos = torch.full((B,), p, dtype=torch.int32, device=dev)
+    cfg_s = sa.spark_layer_cfg_for_kind(SLIDING)
+    ws = torch.empty(sa.spark_decode_workspace_bytes(B, WINDOW, cfg_s), dtype=torch.uint8, device=dev)
+    fused = sa.SPARK_ROPE_FUSED
+
+    def step(i=0):
+        for L in layers:
+            if L["kind"] == FULL:
+                L["shard"].append(L["kn"].view(B, HKV, D), L["vn"].view(B, HKV, D), pos, flags=fused)
+                L["shard"].attend(L["out"], L["q"], L["g"], pos, flags=fused)
+            else:
+                sa.spark_kv_append(L["kc"], L["vc"], L["kn"], L["vn"], pos, L["cfg"], flags=fused)
+                sa.spark_attn_decode(L["out"], L["q"], L["g"], L["kc"], L["vc"], pos, L["cfg"], ws, flags=fused)
+
+    for _ in range(3):
+        step()
+    sa.spark_check()
+    steps = max(5, min(args.steps, 20))
+    ms = timed_region(torch, dist, step, steps) / steps
+    sa.spark_check()
+    total = sum(decode_kv_bytes(B, p, L["kind"]) for L in layers)
+    res = {"b1_ctx1048576": {"value": total / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+                             "steps_per_s": 1e3 / ms, "kv_bytes_per_step": total, "ranks": world,
+                             "scaling": "strong", "record_bytes_per_rank": sa.spark_decode_cp_record_bytes(B),
+                             "frac_of_hbm_x_ranks": total / (ms * 1e-3) / 1e9 / (peaks["hbm_gbs"] * world)}}
+    del layers, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------- oracle timing -------
 
 def oracle_prefill_rate(budget_s: float = 15.0):
@@ -877,6 +938,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context prefill and decode workloads")
+    ap.add_argument("--cp-decode", action="store_true",
+                    help="also run context-parallel decode (B=1 at 2^20, full-layer caches split over the ranks)")
     ap.add_argument("--profile", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_q8_full",
                                           "prefill_ragged_full"],
                     default=None,
@@ -914,6 +977,7 @@ def main():
     ragged = run_prefill_ragged(torch, sa, synth, dist, args, peaks, world)
     long_pf = None if args.no_long else run_long_prefill(torch, sa, synth, dist, args, peaks, world)
     long_dec = None if (args.no_long or args.no_decode) else run_long_decode(torch, sa, synth, dist, args, peaks, world)
+    cp_dec = run_cp_decode(torch, sa, synth, dist, args, peaks, world) if args.cp_decode else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, threads, sample = oracle_prefill_rate()
@@ -940,6 +1004,7 @@ def main():
         "cpu_baseline": cpu, "prefill_ragged": ragged, "decode": dec, "decode_q8": dec_q8,
         "decode_paged256": dec_paged,
         "long_prefill": long_pf, "long_decode": long_dec,
+        "long_decode_cp": cp_dec,
     }
     print(json.dumps(line), flush=True)
 
