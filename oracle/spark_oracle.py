@@ -17,7 +17,7 @@ reordering.  Page citations use the page's title and section:
 * [HYBRID] "Spark-X2.6-4B-Base" hybrid attention (eliteato.com/news/34565)
 * [GGUF]   "Sharp-Spark-X2.5-4B-GGUF" on a 6 GB card (mpbf.cn/news/67460)
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 RoPE pairs dim i with dim i + rot/2 (the rotate-half convention of a
 transformers modeling file); the partial-rotary inverse frequencies use the
 rotated width as denominator, f_i = theta^(-2i/rot); the window of 512 counts
