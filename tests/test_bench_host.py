@@ -25,3 +25,19 @@ def test_headline_work_numbers():
     tot = sum(bench.decode_kv_bytes(64, 32768, O.layer_kind(l)) for l in range(36))
     assert abs(tot / 1e9 - 80.93) < 0.05
     assert bench.decode_kv_bytes(1, 1 << 20 - 0, O.FULL) >= 4 * 2 ** 30
+
+
+@pytest.mark.parametrize("kind", [O.SLIDING, O.FULL])
+@pytest.mark.parametrize("T", [1, 128, 129, 700, 8192])
+def test_tile_flops_count_touched_tiles(kind, T):
+    """Tile-executed FLOPs: every (128-query tile, 128-key tile) pair that holds a visible pair,
+    counted by brute force over the oracle's mask, times 128 x 128 pairs x 4 x 256 FLOP x 16 heads."""
+    n_qt = (T + 127) // 128
+    touched = 0
+    for qt in range(n_qt):
+        q = np.arange(qt * 128, min(T, qt * 128 + 128))
+        for kt in range(n_qt):
+            k = np.arange(kt * 128, min(T, kt * 128 + 128))
+            touched += bool(O.visible(q, k, kind).any())
+    assert bench.prefill_tile_flops(2, T, kind) == 2 * 16 * touched * 128 * 128 * 4 * 256
+    assert bench.prefill_tile_flops(2, T, kind) >= bench.prefill_flops(2, T, 0, kind, False)
