@@ -172,4 +172,120 @@ __device__ __forceinline__ void rope_q_tile(uint8_t* qg, const PrefillParams& P,
   }
 }
 
+
+// One KV tile of the online softmax for this thread's query row (its tensor-memory lane), shared by
+// the two prefill kernels.  The tile's scores are read from tensor memory (scol) and masked on a
+// boundary tile (keys outside [v_lo, v_hi), after the query, or out of its window).  The running
+// max and sum are updated.  The reference max moves only when the max grows by more than 2^8; then
+// O in tensor memory (ocol) is rescaled once the previous P.V has completed (barrier o_bar,
+// parity o_parity).  P = 2^(s log2(e) / 16 - m) is written back over the scores as bf16 pairs.
+// kPacked: the elementwise work in sm_100 packed fp32 pairs and the three-input max.  Returns
+// false when a wait ran out.
+template <bool kPacked>
+__device__ __forceinline__ bool pf_softmax_tile(uint32_t scol, uint32_t ocol, const PfTile& t, const PfSchedule& S,
+                                                const PrefillParams& P, int qp, float& m_ref, float& l_run,
+                                                uint32_t o_bar, uint32_t o_parity, volatile int* abort_flag,
+                                                unsigned where) {
+  const float c_scale = 0.0625f * 1.4426950408889634f;    // 1/sqrt(256) * log2(e)
+  uint32_t sv[128];
+  tmem_ld32(scol, sv);
+  tmem_ld32(scol + 32, sv + 32);
+  tmem_ld32(scol + 64, sv + 64);
+  tmem_ld32(scol + 96, sv + 96);
+  tmem_wait_ld();
+
+  const bool full_tile = t.kt0 >= t.v_lo && t.kt0 + kPfN <= t.v_hi && t.kt0 + kPfN - 1 <= S.qp0 &&
+                         (!P.sliding || t.kt0 > S.qp0 + kPfM - 1 - kWindow);
+  // row max over the raw scores in four independent chains (scale applied after: c_scale > 0)
+  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  if (full_tile) {
+    if constexpr (!kPacked) {
+#pragma unroll
+      for (int i = 0; i < 128; ++i) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(sv[i]));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 128; i += 2)
+        m4[(i >> 1) & 3] = fmax3(m4[(i >> 1) & 3], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+    }
+  } else {
+    const int lo = max(t.v_lo, P.sliding ? qp - (kWindow - 1) : t.v_lo) - t.kt0;
+    const int hi = min(t.v_hi - 1, qp) - t.kt0;
+    if constexpr (!kPacked) {
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        const float x = (i >= lo && i <= hi) ? __uint_as_float(sv[i]) : -INFINITY;
+        sv[i] = __float_as_uint(x);
+        m4[i & 3] = fmaxf(m4[i & 3], x);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 128; i += 2) {
+        const float x0 = (i >= lo && i <= hi) ? __uint_as_float(sv[i]) : -INFINITY;
+        const float x1 = (i + 1 >= lo && i + 1 <= hi) ? __uint_as_float(sv[i + 1]) : -INFINITY;
+        sv[i] = __float_as_uint(x0);
+        sv[i + 1] = __float_as_uint(x1);
+        m4[(i >> 1) & 3] = fmax3(m4[(i >> 1) & 3], x0, x1);
+      }
+    }
+  }
+  const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c_scale;
+  float factor = 1.f;
+  const bool resc = mx > m_ref + 8.f;
+  if (resc) {
+    factor = fast_exp2(m_ref - mx);
+    m_ref = mx;
+  }
+  const bool need_o = resc && l_run > 0.f;
+  if (__any_sync(0xffffffffu, need_o)) {
+    if (!__all_sync(0xffffffffu, mbar_wait(o_bar, o_parity, abort_flag, P.timeout_ns, where))) return false;
+    tc_fence_after();
+    const float f = need_o ? factor : 1.f;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      uint32_t ov[32];
+      tmem_ld32(ocol + 32 * c, ov);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+      tmem_st32(ocol + 32 * c, ov);
+    }
+    tmem_wait_st();
+  }
+  l_run *= factor;
+  const float nmr = (m_ref == -INFINITY) ? 0.f : -m_ref;
+  uint32_t pk[64];
+  if constexpr (!kPacked) {
+    float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * i]), c_scale, nmr));
+      const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * i + 1]), c_scale, nmr));
+      l4[i & 3] += p0 + p1;
+      pk[i] = pack_bf16(p0, p1);
+    }
+    l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+  } else {
+    // p = 2^(s c - m) for pairs of columns with packed FMAs; row sums in two packed accumulators
+    const unsigned long long c2 = f2_pack(c_scale, c_scale), n2 = f2_pack(nmr, nmr);
+    unsigned long long l2[2] = {0ull, 0ull};
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      float x0, x1;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2, n2), x0, x1);
+      const float p0 = fast_exp2(x0);
+      const float p1 = fast_exp2(x1);
+      l2[i & 1] = f2_add(l2[i & 1], f2_pack(p0, p1));
+      pk[i] = pack_bf16(p0, p1);
+    }
+    float la, lb, lc, ld;
+    f2_unpack(l2[0], la, lb);
+    f2_unpack(l2[1], lc, ld);
+    l_run += (la + lb) + (lc + ld);
+  }
+  tmem_st32(scol, pk);
+  tmem_st32(scol + 32, pk + 32);
+  tmem_wait_st();
+  return true;
+}
+
 }  // namespace spark

@@ -432,7 +432,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     const int r = threadIdx.x - 128;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t ocol = tmem + lane_base + kOCol;
-    const float c_scale = 0.0625f * 1.4426950408889634f;    // 1/sqrt(256) * log2(e)
     const uint32_t p_ready0 = mapa_shared(bar_p, 0);
     const uint32_t o_free0 = mapa_shared(bar_o_free, 0);
     int jg = 0, qu = 0;
@@ -466,81 +465,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         }
         tc_fence_after();
         const uint32_t scol = tmem + lane_base + kSCol + 128u * (jgl & 1);
-        uint32_t sv[128];
-        tmem_ld32(scol, sv);
-        tmem_ld32(scol + 32, sv + 32);
-        tmem_ld32(scol + 64, sv + 64);
-        tmem_ld32(scol + 96, sv + 96);
-        tmem_wait_ld();
-
         const PfTile t = pf_tile(S, P, j);
-        const bool full_tile = t.kt0 >= t.v_lo && t.kt0 + kPfN <= t.v_hi && t.kt0 + kPfN - 1 <= S.qp0 &&
-                               (!P.sliding || t.kt0 > S.qp0 + kPfM - 1 - kWindow);
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (full_tile) {
-#pragma unroll
-          for (int i = 0; i < 128; i += 2)
-            m4[(i >> 1) & 3] = fmax3(m4[(i >> 1) & 3], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
-        } else {
-          const int lo = max(t.v_lo, P.sliding ? qp - (kWindow - 1) : t.v_lo) - t.kt0;
-          const int hi = min(t.v_hi - 1, qp) - t.kt0;
-#pragma unroll
-          for (int i = 0; i < 128; i += 2) {
-            const float x0 = (i >= lo && i <= hi) ? __uint_as_float(sv[i]) : -INFINITY;
-            const float x1 = (i + 1 >= lo && i + 1 <= hi) ? __uint_as_float(sv[i + 1]) : -INFINITY;
-            sv[i] = __float_as_uint(x0);
-            sv[i + 1] = __float_as_uint(x1);
-            m4[(i >> 1) & 3] = fmax3(m4[(i >> 1) & 3], x0, x1);
-          }
+        // the previous P.V (tile j-1) must be complete before O is rescaled
+        if (!pf_softmax_tile<true>(scol, ocol, t, S, P, qp, m_ref, l_run, bar_o + 8 * ((jgl - 1) & 1),
+                                 ((jgl - 1) >> 1) & 1, abort_flag, 0x8Au)) {
+          ok = false;
+          break;
         }
-        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c_scale;
-        float factor = 1.f;
-        const bool resc = mx > m_ref + 8.f;
-        if (resc) {
-          factor = fast_exp2(m_ref - mx);
-          m_ref = mx;
-        }
-        const bool need_o = resc && l_run > 0.f;
-        if (__any_sync(0xffffffffu, need_o)) {
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_o + 8 * ((jgl - 1) & 1), ((jgl - 1) >> 1) & 1, abort_flag,
-                                                 P.timeout_ns, 0x8Au))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          for (int cc = 0; cc < 8; ++cc) {
-            uint32_t ov[32];
-            tmem_ld32(ocol + 32 * cc, ov);
-            tmem_wait_ld();
-            const float f = need_o ? factor : 1.f;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-            tmem_st32(ocol + 32 * cc, ov);
-          }
-          tmem_wait_st();
-        }
-        l_run *= factor;
-        const float nmr = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        // p = 2^(s c - m) for pairs of columns with packed FMAs; row sums in two packed accumulators
-        const unsigned long long c2 = f2_pack(c_scale, c_scale), n2 = f2_pack(nmr, nmr);
-        unsigned long long l2[2] = {0ull, 0ull};
-        uint32_t pk[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2, n2), x0, x1);
-          const float p0 = fast_exp2(x0);
-          const float p1 = fast_exp2(x1);
-          l2[i & 1] = f2_add(l2[i & 1], f2_pack(p0, p1));
-          pk[i] = pack_bf16(p0, p1);
-        }
-        float la, lb, lc, ld;
-        f2_unpack(l2[0], la, lb);
-        f2_unpack(l2[1], lc, ld);
-        l_run += (la + lb) + (lc + ld);
-        tmem_st32(scol, pk);
-        tmem_st32(scol + 32, pk + 32);
-        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
