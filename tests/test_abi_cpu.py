@@ -66,3 +66,32 @@ def test_calls_fail_loudly_without_a_device(lib):
     x = torch.zeros(1, 1, 16, 256, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         sa.spark_rope_apply(x, torch.zeros(1, dtype=torch.int32), cfg)
+
+
+def test_host_argument_checks_run_before_the_device(lib):
+    """Host-side validation of the C entry points returns its status before any device call, so it
+    is checked here without a GPU (fake, never dereferenced pointers)."""
+    import full_gqa_attention_spark2_b200 as sa
+    L = sa._lib()
+    full = sa.spark_layer_cfg_for_kind(sa.SPARK_FULL)
+    sliding = sa.spark_layer_cfg_for_kind(sa.SPARK_SLIDING)
+    fake = ctypes.c_void_p(1 << 20)          # 16-byte aligned, never dereferenced on these paths
+    # context parallelism: full layers only; shards inside [0, 2^20)
+    assert L.spark_kv_append_cp(fake, fake, 64, 0, fake, fake, 1, fake, ctypes.byref(sliding), 0, None) == -2
+    assert L.spark_kv_append_cp(fake, fake, 64, -1, fake, fake, 1, fake, ctypes.byref(full), 0, None) == -1
+    assert L.spark_kv_append_cp(fake, fake, 64, (1 << 20) - 10, fake, fake, 1, fake, ctypes.byref(full), 0,
+                                None) == -1
+    assert L.spark_attn_decode_cp_partial(fake, fake, fake, fake, 64, 0, 1, fake, ctypes.byref(sliding), fake, 1 << 20,
+                                          0, None) == -2
+    assert L.spark_attn_decode_cp_partial(None, fake, fake, fake, 64, 0, 1, fake, ctypes.byref(full), fake, 1 << 20,
+                                          0, None) == -1
+    assert L.spark_attn_decode_cp_merge(fake, fake, fake, 0, 1, None) == -1
+    assert L.spark_attn_decode_cp_merge(fake, fake, fake, 2, 0, None) == -1
+    assert L.spark_attn_decode_cp_merge(None, fake, fake, 2, 1, None) == -1
+    assert L.spark_decode_cp_record_bytes(3) == 3 * 16 * 257 * 4
+    assert L.spark_decode_cp_record_bytes(0) == 0
+    # prefill: SPARK_APPEND_FUSED needs the caches; unknown flags are refused
+    args = (fake, fake, fake, fake, fake, None, None, 0, 1, 128, fake, ctypes.byref(full))
+    assert L.spark_attn_prefill(*args, sa.SPARK_APPEND_FUSED, None) == -1
+    assert L.spark_attn_prefill(*args, 0x80, None) == -1
+    assert "SPARK_APPEND_FUSED" in sa.spark_last_error() or "flags" in sa.spark_last_error()
