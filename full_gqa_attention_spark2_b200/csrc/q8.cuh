@@ -134,8 +134,8 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     const float y = __fmul_rn(x[e], inv);
-    const int c = (int)floorf(__fadd_rn(fabsf(y), 0.5f));
-    const uint32_t u = (uint32_t)((y < 0.f ? -c : c) + 128);
+    const int c = (int)roundf(y);          // round half away from zero, exact
+    const uint32_t u = (uint32_t)(c + 128);
     w[e >> 2] |= u << (8 * (e & 3));
   }
   const int h = hb >> 3, bl = hb & 7;

@@ -324,9 +324,10 @@ def quantize_q8(x):
     carry one scale each, cutting 36 KB per token to 19 KB.  The pages give the
     format's name and byte count only; the reading taken here: per block,
     amax = max |x|, scale d = fp16(amax / 127), code c = round-half-away-from-
-    zero(x * (127 / amax)) in [-127, 127], stored offset by 128 as a byte.  All
-    arithmetic before the rounding is float32 (the same operations the device
-    performs), so the codes are exact integers both sides agree on.  A block
+    zero(x * (127 / amax)) in [-127, 127], stored offset by 128 as a byte.  The
+    division and the product are float32 (the same operations the device
+    performs); the rounding of the float32 product y is exact: it is done in
+    float64, where |y| + 1/2 carries no rounding error.  A block
     whose 127 / amax is not a finite float32 (amax below ~3.7e-37, so its fp16
     scale is 0 anyway) gets code 0 throughout, like an all-zero block.
     Returns (u8 codes [..., 256], fp16 scales [..., 8]).
@@ -337,8 +338,8 @@ def quantize_q8(x):
     with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
         inv = (np.float32(127.0) / amax).astype(np.float32)
         inv = np.where((amax > 0) & np.isfinite(inv), inv, np.float32(0.0)).astype(np.float32)
-    y = (blocks * inv).astype(np.float32)
-    c = np.sign(y) * np.floor(np.abs(y) + np.float32(0.5))
+    y = (blocks * inv).astype(np.float32).astype(np.float64)
+    c = np.sign(y) * np.floor(np.abs(y) + 0.5)
     codes = (c + 128).astype(np.uint8).reshape(x.shape)
     scales = (amax[..., 0] / np.float32(127.0)).astype(np.float32).astype(np.float16)
     return codes, scales

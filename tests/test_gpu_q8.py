@@ -94,6 +94,27 @@ def test_kv_append_q8_zero_and_extreme_blocks():
     assert (_host(kc)[0, :, 12:] == 7).all()                    # rows past the tokens untouched
 
 
+def test_kv_append_q8_rounding_ties():
+    """Exact halves round away from zero on the device as in the oracle: a block whose largest value
+    is 127 (factor 127 / amax = 1) holding +-0.5, +-2.5, +-126.5 and the bf16 values next to 1/2."""
+    B, T = 1, 1
+    vals = np.zeros((B, T, 4, 256), np.float32)
+    vals[0, 0, 1, 32:43] = [127.0, 0.5, -0.5, 2.5, -2.5, 126.5, -126.5, 0.498046875, -0.498046875,
+                            0.50390625, 1.5]
+    kb = (vals.view(np.uint32) >> 16).astype(np.uint16)      # all exact in bf16
+    assert np.array_equal(f64(kb), vals.astype(np.float64))
+    kc, ks = _q8_cache(B, 16)
+    vc, vs = _q8_cache(B, 16)
+    cfg = sa.spark_layer_cfg_for_kind(O.FULL)
+    sa.spark_kv_append_q8(kc, ks, vc, vs, to_dev(kb), to_dev(kb), _pos_tensor([3]), cfg)
+    sa.spark_check()
+    codes, scales = O.quantize_q8(vals)
+    assert list(codes[0, 0, 1, 32:43].astype(int) - 128) == [127, 1, -1, 3, -3, 127, -127, 0, 0, 1, 2]
+    for c, sc in ((kc, ks), (vc, vs)):
+        np.testing.assert_array_equal(_host(c)[0, :, 3], codes[0, 0])
+        np.testing.assert_array_equal(_host(sc)[0, :, 3].view(np.uint16), scales[0, 0].view(np.uint16))
+
+
 @pytest.mark.parametrize("kind", [O.SLIDING, O.FULL])
 def test_kv_append_q8_fused_rope(kind):
     B, T = 2, 200

@@ -353,6 +353,37 @@ def test_q8_worked_example():
     assert np.all(scales[1:] == 0) and np.all(codes[32:] == 128)        # all-zero blocks
 
 
+def test_q8_rounding_is_exact_half_away():
+    """Codes are the float32 product y rounded half away from zero, exactly: with amax 127 the
+    factor 127 / amax is 1, so y = x.  0.49999997f (the float just below 1/2) must give 0 even though
+    0.49999997f + 0.5f rounds to 1.0f in float32; exact halves go away from zero."""
+    x = np.zeros(256, dtype=np.float32)
+    below_half = np.nextafter(np.float32(0.5), np.float32(0.0))
+    assert below_half + np.float32(0.5) == np.float32(1.0)          # the float32 shortcut would give 1
+    x[:9] = [127.0, below_half, -below_half, 0.5, -0.5, 2.5, -2.5, 126.5, -126.5]
+    codes, scales = O.quantize_q8(x)
+    assert list(codes[:9].astype(int) - 128) == [127, 0, 0, 1, -1, 3, -3, 127, -127]
+    assert scales[0] == np.float16(1.0)
+
+
+def test_q8_rounding_edge_unreachable_from_bf16():
+    """The one float32 product where floor(|y| + 0.5f) in float32 differs from exact rounding,
+    y = 0.5 - 2^-25, arises from no bf16 value x and bf16 block maximum amax >= |x| (the cache's
+    inputs are bf16): for every amax, only the bf16 neighbours of y / (127 / amax) can round to y."""
+    bits = np.arange(0x0080, 0x7F80, dtype=np.uint32)           # every positive normal bf16
+    amax = (bits << 16).view(np.float32)
+    with np.errstate(over="ignore"):
+        inv = (np.float32(127.0) / amax).astype(np.float32)
+    target = np.nextafter(np.float32(0.5), np.float32(0.0))
+    x_near = ((target / inv.astype(np.float64)).astype(np.float32).view(np.uint32) >> 16).astype(np.int64)
+    for d in range(-2, 3):
+        cand = np.clip(x_near + d, 0x0080, 0x7F7F).astype(np.uint32)
+        x = (cand << 16).view(np.float32)
+        with np.errstate(over="ignore", invalid="ignore"):
+            y = (x * inv).astype(np.float32)
+        assert not np.any((y == target) & (x <= amax))
+
+
 def test_q8_tiny_block_quantises_to_zero():
     """127 / amax overflows float32 for a block of denormal values: codes 0, scale 0 (no inf or NaN)."""
     x = np.zeros(256, dtype=np.float32)
