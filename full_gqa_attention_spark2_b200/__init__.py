@@ -17,6 +17,7 @@ SPARK_SLIDING = 0
 SPARK_FULL = 1
 SPARK_ROPE_FUSED = 1
 SPARK_APPEND_FUSED = 2
+SPARK_STATIC_SCRATCH_BYTES = 16 << 20
 N_LAYERS = 36
 N_Q_HEADS = 16
 N_KV_HEADS = 4
@@ -74,6 +75,7 @@ def _lib():
         "spark_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
         "spark_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, cfgp, _P, ctypes.c_size_t, ctypes.c_uint, _P]),
         "spark_attn_decode_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
+        "spark_decode_static_plan": (ctypes.c_size_t, [_I, _I, cfgp, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
         "spark_kv_cache_q8_bytes": (ctypes.c_longlong, [cfgp, _I, ctypes.c_longlong]),
         "spark_kv_append_q8": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
         "spark_decode_q8_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
@@ -110,7 +112,7 @@ def exported_symbols():
     """Names of the C entry points this binding expects the library to export."""
     return ["spark_layer_cfg_for_layer", "spark_layer_cfg_for_kind", "spark_kv_cache_bytes",
             "spark_stack_kv_bytes", "spark_rope_apply", "spark_kv_append", "spark_attn_prefill",
-            "spark_decode_workspace_bytes", "spark_attn_decode", "spark_attn_decode_static",
+            "spark_decode_workspace_bytes", "spark_attn_decode", "spark_attn_decode_static", "spark_decode_static_plan",
             "spark_kv_cache_q8_bytes", "spark_kv_append_q8", "spark_decode_q8_workspace_bytes",
             "spark_attn_decode_q8", "spark_kv_append_paged", "spark_decode_paged_workspace_bytes",
             "spark_attn_decode_paged", "spark_rope_apply_varlen", "spark_kv_append_varlen",
@@ -280,6 +282,14 @@ def spark_attn_decode_static(out, q, gate, k_cache, v_cache, pos, cfg: SparkLaye
     pp = _dev(pos, "pos", torch.int32, 1)
     _raise(_lib().spark_attn_decode_static(po, pq, pg, pkc, pvc, k_cache.shape[2], q.shape[0], pp,
                                            ctypes.byref(cfg), flags, _stream(stream)))
+
+
+def spark_decode_static_plan(B: int, cap: int, cfg: SparkLayerCfg, sm_count: int = 148):
+    """(n_splits, tiles_per_split, bytes) of spark_attn_decode_static's split plan; bytes is 0 on bad
+    arguments or a batch above the scratch array's limit."""
+    ns, tps = _I(0), _I(0)
+    nbytes = _lib().spark_decode_static_plan(B, cap, ctypes.byref(cfg), sm_count, ctypes.byref(ns), ctypes.byref(tps))
+    return ns.value, tps.value, int(nbytes)
 
 
 def spark_kv_cache_q8_bytes(cfg: SparkLayerCfg, B: int, cap: int) -> int:

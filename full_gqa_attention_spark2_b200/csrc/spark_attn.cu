@@ -415,11 +415,23 @@ int decode_maps(const CacheView& c, int B, CUtensorMap* km, CUtensorMap* vm, CUt
   return SPARK_OK;
 }
 
+// The usual plan with fewer, longer splits when its partials would exceed
+// max_bytes (at least one split's partials must fit: checked by the caller).
+DecodePlan fit_plan(DecodePlan pl, int B, int tiles, size_t max_bytes) {
+  if (decode_ws_bytes(B, pl) <= max_bytes) return pl;
+  const size_t per_split = decode_ws_bytes(B, DecodePlan{1, tiles});
+  const int s_fit = (int)(max_bytes / per_split);
+  pl.tiles_per_split = (tiles + s_fit - 1) / s_fit;
+  pl.n_splits = (tiles + pl.tiles_per_split - 1) / pl.tiles_per_split;
+  return pl;
+}
+
 // record != nullptr: context parallelism (a full layer's cache is one rank's
 // shard, positions key_off ..): no output, this rank's record is written instead.
+// fit_ws: the workspace is a fixed array of ws_bytes; the plan is fitted to it.
 int decode_impl(void* out, const void* q, const void* gate, const CacheView& c, int B, const int* pos,
                 const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes, unsigned flags, void* stream,
-                int key_off = 0, float* record = nullptr) {
+                int key_off = 0, float* record = nullptr, bool fit_ws = false) {
   int rc = check_view(c, cfg);
   if (rc) return rc;
   if (record) {
@@ -434,7 +446,8 @@ int decode_impl(void* out, const void* q, const void* gate, const CacheView& c, 
   int dev;
   if ((rc = device_ready(&dev))) return rc;
   const int sliding = cfg->kind == SPARK_SLIDING;
-  const DecodePlan pl = plan_for(B, c, sliding, g_dev[dev].sm_count);
+  DecodePlan pl = plan_for(B, c, sliding, g_dev[dev].sm_count);
+  if (fit_ws) pl = fit_plan(pl, B, ((sliding ? SPARK_WINDOW : c.cap) + spark::kDecNK - 1) / spark::kDecNK, ws_bytes);
   if (ws_bytes < decode_ws_bytes(B, pl))
     return fail(SPARK_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu needed", ws_bytes,
                 decode_ws_bytes(B, pl));
@@ -519,22 +532,31 @@ int check_cp_shard(int cap, int key_off, const spark_layer_cfg* cfg) {
 constexpr size_t kStaticScratchBytes = (size_t)SPARK_STATIC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
-struct StaticScratch {
-  std::once_flag once;
-  void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
-};
-StaticScratch g_scratch[kMaxDevices];
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is asked of the
-// runtime once per device, with that device current.
-int static_scratch(int dev, void** out) {
-  StaticScratch& s = g_scratch[dev];
-  std::call_once(s.once, [&]() { s.err = cudaGetSymbolAddress(&s.ptr, g_decode_scratch); });
-  if (s.err != cudaSuccess || s.ptr == nullptr)
-    return cuda_fail(s.err != cudaSuccess ? s.err : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
-  *out = s.ptr;
+// runtime once per device, with that device current; only a successful answer
+// is kept (a failed lookup is retried by the next call).  The lookup is refused
+// while `stream` is being captured into a graph: the first call on a device
+// must come before any capture.
+int static_scratch(int dev, cudaStream_t stream, void** out) {
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(stream, &cs);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    if (cs != cudaStreamCaptureStatusNone)
+      return fail(SPARK_ERR_INVALID_ARG,
+                  "the first spark_attn_decode_static call on a device must come before any stream capture");
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    if (p == nullptr) return fail(SPARK_ERR_CUDA, "cudaGetSymbolAddress(scratch) returned NULL");
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
   return SPARK_OK;
 }
 
@@ -908,14 +930,7 @@ int spark_attn_decode_static(void* out, const void* q, const void* gate, const v
                              const spark_layer_cfg* cfg, unsigned flags, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (!out || !q || !gate || !k_cache || !v_cache || !pos) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
-  if (B <= 0 || B > 65535 || cap <= 0) return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d cap=%d", B, cap);
-  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
-  const int sliding = cfg->kind == SPARK_SLIDING;
-  if (sliding && cap != SPARK_WINDOW) return fail(SPARK_ERR_INVALID_ARG, "sliding caches hold 512 rows");
-  if (!sliding && cap > SPARK_MAX_POSITION) return fail(SPARK_ERR_INVALID_ARG, "cap above 2^20");
-  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-    return fail(SPARK_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (B <= 0 || B > 65535) return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d", B);
   // one split needs a partial row (256 + 2 floats) per sequence and query head
   const size_t per_split = (size_t)B * spark::kNq * (spark::kHeadDim + 2) * sizeof(float);
   if (per_split > kStaticScratchBytes)
@@ -926,52 +941,25 @@ int spark_attn_decode_static(void* out, const void* q, const void* gate, const v
   int dev;
   if ((rc = device_ready(&dev))) return rc;
   void* scratch = nullptr;
-  if ((rc = static_scratch(dev, &scratch))) return rc;
-  // the usual split plan, with fewer splits when its partials would not fit
-  DecodePlan pl = decode_plan(B, cap, sliding, g_dev[dev].sm_count);
-  if (decode_ws_bytes(B, pl) > kStaticScratchBytes) {
-    const int tiles = ((sliding ? SPARK_WINDOW : cap) + spark::kDecNK - 1) / spark::kDecNK;
-    const int s_fit = (int)(kStaticScratchBytes / per_split);
-    pl.tiles_per_split = (tiles + s_fit - 1) / s_fit;
-    pl.n_splits = (tiles + pl.tiles_per_split - 1) / pl.tiles_per_split;
-  }
+  if ((rc = static_scratch(dev, (cudaStream_t)stream, &scratch))) return rc;
+  // the usual split plan, with fewer splits when its partials would not fit the array
+  return decode_impl(out, q, gate, dense_view((void*)k_cache, (void*)v_cache, nullptr, nullptr, cap), B, pos, cfg,
+                     scratch, kStaticScratchBytes, flags, stream, 0, nullptr, true);
+}
 
-  CUtensorMap km, vm;
-  const cuuint64_t dims[3] = {256, (cuuint64_t)cap, (cuuint64_t)B * 4};
-  const cuuint64_t strides[2] = {512, (cuuint64_t)cap * 512};
-  const cuuint32_t box[3] = {64, (cuuint32_t)spark::kDecNK, 1};
-  if ((rc = make_map(&km, k_cache, 3, dims, strides, box))) return rc;
-  if ((rc = make_map(&vm, v_cache, 3, dims, strides, box))) return rc;
-
-  spark::DecodeParams P;
-  P.q = (const __nv_bfloat16*)q;
-  P.pos = pos;
-  P.o_part = (float*)scratch;
-  P.ml_part = (float*)scratch + (size_t)B * spark::kNq * pl.n_splits * spark::kHeadDim;
-  P.B = B;
-  P.cap = cap;
-  P.sliding = sliding;
-  P.n_splits = pl.n_splits;
-  P.tiles_per_split = pl.tiles_per_split;
-  P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
-  P.rot = cfg->rot_dim;
-  P.log2_theta = log2(cfg->theta);
-  P.freq = rope_freq(cfg);
-  P.timeout_ns = wait_timeout_ns();
-  P.out = (__nv_bfloat16*)out;
-  P.gate = (const __nv_bfloat16*)gate;
-  P.block_table = nullptr;
-  P.max_pages = P.page_shift = P.n_pages = 0;
-  P.key_off = P.shard = 0;
-  spark::decode_partial_kernel<false><<<dim3(pl.n_splits, spark::kNkv, B), spark::kDecThreads, spark::kDecSmemBytes,
-                                 (cudaStream_t)stream>>>(km, vm, P);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "decode_partial_kernel launch");
-  if (pl.n_splits == 1) return SPARK_OK;      // the partial kernel wrote the output itself
-  spark::decode_combine_kernel<<<dim3(spark::kNq, B), 64, 0, (cudaStream_t)stream>>>(
-      (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
-  e = cudaGetLastError();
-  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_combine_kernel launch");
+// Split plan of spark_attn_decode_static (host only, for tests): writes n_splits and
+// tiles_per_split for `sm_count` SMs; returns the partials' bytes, 0 on bad arguments.
+size_t spark_decode_static_plan(int B, int cap, const spark_layer_cfg* cfg, int sm_count, int* n_splits,
+                                int* tiles_per_split) {
+  if (check_cfg(cfg) != SPARK_OK || B <= 0 || B > 65535 || cap <= 0 || sm_count <= 0) return 0;
+  const size_t per_split = (size_t)B * spark::kNq * (spark::kHeadDim + 2) * sizeof(float);
+  if (per_split > kStaticScratchBytes) return 0;
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  const int tiles = ((sliding ? SPARK_WINDOW : cap) + spark::kDecNK - 1) / spark::kDecNK;
+  const DecodePlan pl = fit_plan(decode_plan(B, cap, sliding, sm_count), B, tiles, kStaticScratchBytes);
+  if (n_splits) *n_splits = pl.n_splits;
+  if (tiles_per_split) *tiles_per_split = pl.tiles_per_split;
+  return decode_ws_bytes(B, pl);
 }
 
 int spark_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {

@@ -180,7 +180,10 @@ int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_
  * allocating routine.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, once per device, with that device current); make
- *     that first call before any stream capture.
+ *     that first call before any stream capture.  A first call made while
+ *     `stream` is being captured is refused with SPARK_ERR_INVALID_ARG and
+ *     nothing is launched; a failed lookup is not remembered, the next call
+ *     tries again.
  *   - One split needs B * 16 * 258 * 4 bytes, so B may be at most 1016; larger
  *     batches are rejected with SPARK_ERR_INVALID_ARG.  When the usual split
  *     plan does not fit, fewer splits are used.
@@ -191,6 +194,14 @@ int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_
 int spark_attn_decode_static(void* out, const void* q, const void* gate, const void* k_cache,
                              const void* v_cache, int cap, int B, const int* pos,
                              const spark_layer_cfg* cfg, unsigned flags, void* stream);
+
+/* Split plan spark_attn_decode_static uses on a device of sm_count SMs (host
+ * only, no device access): *n_splits key splits of *tiles_per_split 64-key
+ * tiles per (sequence, KV head).  Returns the bytes of the array the partials
+ * occupy (<= SPARK_STATIC_SCRATCH_BYTES), 0 on bad arguments or when B is above
+ * the limit.  n_splits, tiles_per_split may be NULL. */
+size_t spark_decode_static_plan(int B, int cap, const spark_layer_cfg* cfg, int sm_count, int* n_splits,
+                                int* tiles_per_split);
 
 /* ---- 8-bit block-quantised KV cache ("Sharp-Spark-X2.5-4B-GGUF" page §四:
  * the K/V cache stored as q8_0, 36 -> 19 KB per token).  The block format is

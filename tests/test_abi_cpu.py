@@ -95,3 +95,23 @@ def test_host_argument_checks_run_before_the_device(lib):
     assert L.spark_attn_prefill(*args, sa.SPARK_APPEND_FUSED, None) == -1
     assert L.spark_attn_prefill(*args, 0x80, None) == -1
     assert "SPARK_APPEND_FUSED" in sa.spark_last_error() or "flags" in sa.spark_last_error()
+
+
+def test_static_decode_plan_fits_and_covers_every_tile(lib):
+    """spark_attn_decode_static's plan: partials within the fixed array, splits that cover every
+    64-key tile exactly once; fewer splits than the usual plan where that plan would not fit."""
+    import full_gqa_attention_spark2_b200 as sa
+    for kind in (sa.SPARK_SLIDING, sa.SPARK_FULL):
+        cfg = sa.spark_layer_cfg_for_kind(kind)
+        for B in (1, 3, 64, 300, 600, 1016):
+            for cap in ((512,) if kind == sa.SPARK_SLIDING else (1, 100, 8192, 16384, 131072, 1 << 20)):
+                ns, tps, nbytes = sa.spark_decode_static_plan(B, cap, cfg, 148)
+                tiles = -(-min(cap, 512 if kind == sa.SPARK_SLIDING else cap) // 64)
+                assert 0 < nbytes <= sa.SPARK_STATIC_SCRATCH_BYTES, (kind, B, cap)
+                assert nbytes == B * 16 * ns * 258 * 4
+                assert (ns - 1) * tps < tiles <= ns * tps, (kind, B, cap, ns, tps)
+                if sa.spark_decode_workspace_bytes(B, cap, cfg) <= sa.SPARK_STATIC_SCRATCH_BYTES:
+                    assert nbytes == sa.spark_decode_workspace_bytes(B, cap, cfg)      # the usual plan
+    full = sa.spark_layer_cfg_for_kind(sa.SPARK_FULL)
+    assert sa.spark_decode_workspace_bytes(300, 16384, full) > sa.SPARK_STATIC_SCRATCH_BYTES
+    assert sa.spark_decode_static_plan(1017, 512, full, 148)[2] == 0
