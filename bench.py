@@ -97,6 +97,18 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def hbm_roofline(kernel: str, achieved_gbs: float, peaks, traffic=None):
+    """Roofline entry of a kernel that only reads HBM (the decode kernels read the KV cache and write
+    a few KB): held to the measured read-only ceiling; the copy figure of MEASURED_PEAKS.json (read +
+    write bytes of a device copy) is kept beside it for reference."""
+    read = peaks.get("hbm_read_gbs")
+    peak, src = (read, "read-only stream over 8 GiB, measured in this run") if read else \
+        (peaks["hbm_gbs"], f"hbm_gbs copy, {peaks['source']} (no read probe in this run)")
+    return {"bound": "hbm", "kernel": kernel, "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
+            "frac": achieved_gbs / peak, "peak_source": src, "copy_peak_gbs": peaks["hbm_gbs"],
+            "frac_of_copy": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic}
+
+
 def kernel_source_sha():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "full_gqa_attention_spark2_b200", "csrc")
@@ -172,9 +184,9 @@ class ClockSampler:
 
 # ------------------------------------------------------------ our arm -------
 
-def prefill_workload(torch, sa, synth, dev):
-    """Device buffers of the headline workload for both layer kinds."""
-    B, T = PREFILL_B, PREFILL_T
+def prefill_workload(torch, sa, synth, dev, B=PREFILL_B, T=PREFILL_T, seed=PREFILL_SEED, k_sigma=0.5,
+                     g_sigma=2.0):
+    """Device buffers of a prefill workload for both layer kinds (default: the headline workload)."""
     W = {}
     for kind, layer in ((SLIDING, 0), (FULL, 3)):
         cfg = sa.spark_layer_cfg_for_kind(kind)
@@ -182,10 +194,10 @@ def prefill_workload(torch, sa, synth, dev):
         k = torch.empty(B, T, HKV, D, dtype=torch.bfloat16, device=dev)
         v = torch.empty_like(k)
         g = torch.empty(B, T, HQ, dtype=torch.bfloat16, device=dev)
-        synth.fill_tokens(q, PREFILL_SEED, synth.tensor_id(layer, synth.ROLE_Q), 0)
-        synth.fill_tokens(k, PREFILL_SEED, synth.tensor_id(layer, synth.ROLE_K), 0, sigma=0.5)
-        synth.fill_tokens(v, PREFILL_SEED, synth.tensor_id(layer, synth.ROLE_V), 0)
-        synth.fill_tokens(g, PREFILL_SEED, synth.tensor_id(layer, synth.ROLE_GATE), 0, sigma=2.0)
+        synth.fill_tokens(q, seed, synth.tensor_id(layer, synth.ROLE_Q), 0)
+        synth.fill_tokens(k, seed, synth.tensor_id(layer, synth.ROLE_K), 0, sigma=k_sigma)
+        synth.fill_tokens(v, seed, synth.tensor_id(layer, synth.ROLE_V), 0)
+        synth.fill_tokens(g, seed, synth.tensor_id(layer, synth.ROLE_GATE), 0, sigma=g_sigma)
         cap = WINDOW if kind == SLIDING else T
         kc = torch.empty(B, HKV, cap, D, dtype=torch.bfloat16, device=dev)
         vc = torch.empty_like(kc)
@@ -350,6 +362,38 @@ def run_prefill(torch, sa, synth, dist, args, peaks, world):
     }
 
 
+TINY_B, TINY_T, TINY_SEED = 1, 1024, 0
+
+
+def run_prefill_tiny(torch, sa, synth, dist, args, peaks, world):
+    """The small prefill workload: B=1, T=1024, seed 0, q/k/v/gate ~N(0,1), one sliding and one full
+    layer, the same step as the headline (RoPE on k, prefill with q rotated at load, the append)."""
+    dev = torch.device("cuda")
+    B, T = TINY_B, TINY_T
+    W, pos0 = prefill_workload(torch, sa, synth, dev, B, T, TINY_SEED, 1.0, 1.0)
+    for _ in range(max(3, args.warmup)):
+        prefill_step(sa, W, pos0)
+    sa.spark_check()
+    steps = max(20, min(args.steps, 200))
+    pairs = [{kind: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for kind in (SLIDING, FULL)} for _ in range(steps)]
+    ms = timed_region(torch, dist, lambda i: prefill_step(sa, W, pos0, pairs[i]), steps) / steps
+    sa.spark_check()
+    per = {}
+    for name, kind in (("sliding", SLIDING), ("full", FULL)):
+        k_ms = statistics.mean(ev[kind][0].elapsed_time(ev[kind][1]) for ev in pairs)
+        f = prefill_flops(B, T, 0, kind, False)
+        per[name] = {"kernel_us": k_ms * 1e3, "tok_s": B * T / (k_ms * 1e-3), "tflops": f / (k_ms * 1e-3) / 1e12,
+                     "algorithmic_flops": f, "tile_flops": prefill_tile_flops(B, T, kind)}
+    f_all = prefill_flops(B, T, 0, SLIDING, False) + prefill_flops(B, T, 0, FULL, False)
+    del W
+    return {"workload": f"prefill_tiny_b{B}_t{T}_sliding+full", "value": B * T * world / (ms * 1e-3),
+            "unit": "tok/s", "ms_per_step": ms, "tflops": f_all * world / (ms * 1e-3) / 1e12,
+            "per_layer_kind": per, "gpu_launches_per_step": 6,
+            "note": "8 query tiles x 4 KV heads x 2 head pairs = 64 units on 74 SM pairs: launch- and "
+                    "latency-bound, not a roofline case"}
+
+
 def decode_layers(torch, sa, synth, dev, B: int, p: int, layer_ids=range(N_LAYERS), seed: int = DECODE_SEED):
     """Caches holding positions 0..p-1 and the new token's q/k/v/gate at p, per layer."""
     layers = []
@@ -442,10 +486,8 @@ def run_decode(torch, sa, synth, dist, args, peaks, world):
         "value": total_bytes * world / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
         "ms_per_step": ms_step, "steps_per_s": 1e3 / ms_step, "kv_bytes_per_step": total_bytes,
         "workload": f"decode_b{B}_ctx{p}_36layers", "gpu_launches_per_step": launches,
-        "roofline": {"bound": "hbm", "kernel": "decode_partial_kernel+combine (full layer)",
-                     "achieved": full_bytes / (k_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": full_bytes / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                     "traffic": ncu_traffic("decode_partial_kernel_full")},
+        "roofline": hbm_roofline("decode_partial_kernel+combine (full layer)", full_bytes / (k_ms * 1e-3) / 1e9,
+                                 peaks, ncu_traffic("decode_partial_kernel_full")),
     }
 
 
@@ -583,11 +625,9 @@ def run_decode_variant(torch, sa, synth, dist, args, peaks, world, q8: bool, pag
         "value": total_bytes * world / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
         "ms_per_step": ms_step, "steps_per_s": 1e3 / ms_step, "kv_bytes_per_step": total_bytes,
         "workload": f"{name}_b{B}_ctx{p}_36layers", "gpu_launches_per_step": launches,
-        "roofline": {"bound": "hbm", "kernel": f"{kern}+combine (full layer)",
-                     "achieved": full_bytes / (k_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": full_bytes / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                     "traffic": None if page else ncu_traffic("decode_q8_partial_kernel_full" if q8 else
-                                                              "decode_partial_kernel_full")},
+        "roofline": hbm_roofline(f"{kern}+combine (full layer)", full_bytes / (k_ms * 1e-3) / 1e9, peaks,
+                                 None if page else ncu_traffic("decode_q8_partial_kernel_full" if q8 else
+                                                               "decode_partial_kernel_full")),
     }
 
 
@@ -760,7 +800,8 @@ def run_long_decode(torch, sa, synth, dist, args, peaks, world):
         total = sum(decode_kv_bytes(B, p, L["kind"]) for L in layers)
         out[f"b{B}_ctx{ctx}"] = {"value": total * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
                                  "steps_per_s": 1e3 / ms, "kv_bytes_per_step": total,
-                                 "frac_of_hbm": total / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+                                 "frac_of_hbm": total / (ms * 1e-3) / 1e9 / (peaks.get("hbm_read_gbs") or
+                                                                             peaks["hbm_gbs"])}
         del graph, layers, ws
         torch.cuda.empty_cache()
     return out
@@ -821,7 +862,8 @@ def run_cp_decode(torch, sa, synth, dist, args, peaks, world):
     res = {"b1_ctx1048576": {"value": total / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
                              "steps_per_s": 1e3 / ms, "kv_bytes_per_step": total, "ranks": world,
                              "scaling": "strong", "record_bytes_per_rank": sa.spark_decode_cp_record_bytes(B),
-                             "frac_of_hbm_x_ranks": total / (ms * 1e-3) / 1e9 / (peaks["hbm_gbs"] * world)}}
+                             "frac_of_hbm_x_ranks": total / (ms * 1e-3) / 1e9 / ((peaks.get("hbm_read_gbs") or
+                                                                                     peaks["hbm_gbs"]) * world)}}
     del layers, ws
     torch.cuda.empty_cache()
     return res
@@ -829,50 +871,91 @@ def run_cp_decode(torch, sa, synth, dist, args, peaks, world):
 
 # ------------------------------------------------------- oracle timing -------
 
-def oracle_prefill_rate(budget_s: float = 15.0):
-    """The fp64 oracle on a bounded sample of the headline workload: query rows of
-    sequence 0 through both layers (all 16 heads); returns (tok/s, threads, description)."""
-    import synth
-    from oracle import spark_oracle as O
-    T = PREFILL_T
-    pos = np.arange(T)
-    layer_of = {SLIDING: 0, FULL: 3}
+class OracleSampler:
+    """The fp64 oracle on the headline workload, one bounded sample at a time: `rows` random query
+    rows of sequence 0 (all 16 heads) through both layers, against all of that sequence's keys."""
 
-    def get(kind, role, H, Dd, p, sig=1.0):
-        return synth.bf16_bits_to_f64(
-            synth.token_tensor(PREFILL_SEED, synth.tensor_id(layer_of[kind], role), 1, H, Dd, p, sig)[0])
+    def __init__(self, rows_per_sample: int = 4, seed: int = 0):
+        import synth
+        from oracle import spark_oracle as O
+        self.O, self.synth = O, synth
+        self.R = rows_per_sample
+        self.pos = np.arange(PREFILL_T)
+        self.layer_of = {SLIDING: 0, FULL: 3}
+        self.kv = {kind: (self._get(kind, synth.ROLE_K, HKV, D, self.pos, 0.5),
+                          self._get(kind, synth.ROLE_V, HKV, D, self.pos)) for kind in self.layer_of}
+        self.rng = np.random.default_rng(seed)
 
-    kv = {kind: (get(kind, synth.ROLE_K, HKV, D, pos, 0.5), get(kind, synth.ROLE_V, HKV, D, pos)) for kind in layer_of}
-    rng = np.random.default_rng(0)
-    done, t_used = 0, 0.0
-    while t_used < budget_s or done < 2:
-        rows = np.sort(rng.integers(0, T, size=2))
+    def _get(self, kind, role, H, Dd, p, sig=1.0):
+        s = self.synth
+        return s.bf16_bits_to_f64(s.token_tensor(PREFILL_SEED, s.tensor_id(self.layer_of[kind], role), 1, H, Dd, p,
+                                                 sig)[0])
+
+    def sample(self) -> float:
+        """Runs one sample; returns the seconds the oracle took (input regeneration excluded)."""
+        rows = np.sort(self.rng.integers(0, PREFILL_T, size=self.R))
+        t_used = 0.0
         for kind in (SLIDING, FULL):
-            q_rows = get(kind, synth.ROLE_Q, HQ, D, rows)
-            g_rows = get(kind, synth.ROLE_GATE, HQ, 1, rows, 2.0)
+            q_rows = self._get(kind, self.synth.ROLE_Q, HQ, D, rows)
+            g_rows = self._get(kind, self.synth.ROLE_GATE, HQ, 1, rows, 2.0)
             t0 = time.perf_counter()
-            O.layer_prefill_rows(q_rows, kv[kind][0], kv[kind][1], g_rows, pos, kind, rows)
+            self.O.layer_prefill_rows(q_rows, self.kv[kind][0], self.kv[kind][1], g_rows, self.pos, kind, rows)
             t_used += time.perf_counter() - t0
-        done += len(rows)
-    threads = None
+        return t_used
+
+
+def oracle_threads():
     try:
         from threadpoolctl import threadpool_info
-        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
     except Exception:
-        threads = os.cpu_count()
-    return done / t_used, threads, f"{done} random query rows of sequence 0 through both layers, {t_used:.1f} s"
+        return os.cpu_count()
+
+
+def oracle_prefill_rate(budget_s: float = 15.0):
+    """The oracle's rate (query rows per second through both layers) over samples run until about
+    budget_s seconds of oracle time; returns (tok/s, threads, description)."""
+    sampler = OracleSampler()
+    done, t_used = 0, 0.0
+    while t_used < budget_s or done < 2 * sampler.R:
+        t_used += sampler.sample()
+        done += sampler.R
+    return done / t_used, oracle_threads(), \
+        f"{done} random query rows of sequence 0 through both layers (all 16 heads, all 8192 keys), {t_used:.1f} s"
+
+
+def main_config(world: int) -> dict:
+    """The headline line's config (both arms)."""
+    return {"workload": "prefill_b4_t8192_sliding+full", "B": PREFILL_B, "T": PREFILL_T,
+            "layers": ["sliding (window 512, rope theta 1e4, 256 dims)", "full (rope theta 5e6, first 64 dims)"],
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (q alone is 268 MB per layer); no flush"}
 
 
 def run_reference(args, rank):
+    """The oracle arm: W untimed and K timed steps, each step one bounded sample of the headline
+    workload (4 random query rows of sequence 0 through both layers, fp64, all host threads).  The
+    line reports what was measured: rows per second and the measured seconds per sampled step."""
     if rank != 0:
         return
-    rate, threads, sample = oracle_prefill_rate(budget_s=max(5.0, min(60.0, 3.0 * args.steps)))
+    sampler = OracleSampler(rows_per_sample=4)
+    for _ in range(args.warmup):
+        sampler.sample()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        sampler.sample()
+    wall = time.perf_counter() - t0
+    rows = args.steps * sampler.R
+    rate = rows / wall
+    threads = oracle_threads()
+    sample = (f"{args.steps} timed steps of {sampler.R} random query rows of sequence 0 through both layers "
+              f"(all 16 heads, all 8192 keys), {wall:.1f} s measured; {args.warmup} untimed steps before")
     line = {
         "impl": "reference", "metric": "prefill attn tok/s & TFLOP/s; decode KV-read GB/s (36-layer stack); % roofline",
         "value": rate, "unit": "tok/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": PREFILL_B * PREFILL_T / rate * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "prefill_b4_t8192_sliding+full", "B": PREFILL_B, "T": PREFILL_T},
+        "ms_per_step": wall / args.steps * 1e3, "tokens_per_step": sampler.R, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded counter generator)",
+        "config": main_config(args.gpus),
         "cpu_baseline": {"value": rate, "unit": "tok/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": rate, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -970,6 +1053,9 @@ def main():
         return
 
     res = run_prefill(torch, sa, synth, dist, args, peaks, world)
+    tiny = run_prefill_tiny(torch, sa, synth, dist, args, peaks, world)
+    if not args.no_decode:
+        peaks["hbm_read_gbs"] = synth.read_probe_gbs()
     dec = None if args.no_decode else run_decode(torch, sa, synth, dist, args, peaks, world)
     dec_q8 = None if args.no_decode else run_decode_q8(torch, sa, synth, dist, args, peaks, world)
     dec_paged = None if args.no_decode else run_decode_variant(torch, sa, synth, dist, args, peaks, world,
@@ -992,16 +1078,13 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded counter generator, shapes of the pages' workloads)",
-        "config": {"workload": "prefill_b4_t8192_sliding+full", "B": PREFILL_B, "T": PREFILL_T,
-                   "layers": ["sliding (window 512, rope theta 1e4, 256 dims)",
-                              "full (rope theta 5e6, first 64 dims)"],
-                   "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (q alone is 268 MB per layer); no flush"},
+        "config": main_config(world),
         "tflops": res["tflops"], "prefill_full_kernel": res["prefill_full_kernel"],
         "per_layer_kind": res["per_layer_kind"], "stack36_derived": res["stack36_derived"],
         "roofline": res["roofline"], "e2e": res["e2e"], "clocks": res["clocks"],
         "gpu_launches": res["gpu_launches"] + (0 if dec is None else 0),
-        "cpu_baseline": cpu, "prefill_ragged": ragged, "decode": dec, "decode_q8": dec_q8,
+        "cpu_baseline": cpu, "prefill_tiny": tiny, "hbm_read_gbs": peaks.get("hbm_read_gbs"),
+        "prefill_ragged": ragged, "decode": dec, "decode_q8": dec_q8,
         "decode_paged256": dec_paged,
         "long_prefill": long_pf, "long_decode": long_dec,
         "long_decode_cp": cp_dec,

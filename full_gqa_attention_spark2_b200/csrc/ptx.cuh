@@ -1,6 +1,8 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers with bounded waits, TMA
 // tensor loads, ldmatrix / mma.sync, and the tcgen05 (UMMA + TMEM) family.
-// Written from the PTX ISA; no multicast forms are used anywhere.
+// Written from the PTX ISA.  No copy uses a multicast form: the one
+// `.multicast::cluster` qualifier is on tcgen05.commit (umma2_commit_mc), an
+// mbarrier arrive delivered to the two CTAs of an SM pair, not a load.
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>

@@ -20,7 +20,8 @@ Logical indexing (independent of any cache layout): the element of a
 per-token tensor at (batch b, head h, absolute position p, dim d) has index
 ((b * H + h) * 2^20 + p) * D + d, with D = 1 for the gate logits.
 
-The device implementation is ``synth/synth.cu`` (``libspark_synth.so``).
+The device implementation is ``synth/synth.cu`` (``libspark_synth.so``), which also holds a
+read-only bandwidth probe for the bench (``read_probe_gbs``), no part of the generator.
 """
 from __future__ import annotations
 
@@ -158,8 +159,41 @@ def load_lib():
             ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_longlong, ctypes.c_int, ctypes.c_ulonglong, ctypes.c_ulonglong, ctypes.c_float,
             ctypes.c_void_p]
+        lib.spark_synth_read_probe.restype = ctypes.c_int
+        lib.spark_synth_read_probe.argtypes = [ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p, ctypes.c_int,
+                                               ctypes.c_void_p]
         _LIB = lib
     return _LIB
+
+
+def read_probe_gbs(n_bytes: int = 8 << 30, reps: int = 10, warmup: int = 3) -> float:
+    """Read-only HBM bandwidth (GB/s, 1e9 B/s) of one stream over a device buffer of n_bytes (far
+    larger than L2), best of `reps` launches timed with CUDA events on the current stream.  Bench
+    infrastructure: the ceiling its HBM-bound kernels, which only read the KV cache, are held to."""
+    import torch
+    buf = torch.ones(n_bytes, dtype=torch.uint8, device="cuda")
+    sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    lib = load_lib()
+    st = _stream_ptr(None)
+
+    def launch():
+        if lib.spark_synth_read_probe(buf.data_ptr(), n_bytes, sink.data_ptr(), sms, st) != 0:
+            raise RuntimeError("spark_synth_read_probe failed")
+
+    for _ in range(warmup):
+        launch()
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        launch()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del buf
+    torch.cuda.empty_cache()
+    return n_bytes / (best * 1e-3) / 1e9
 
 
 def _stream_ptr(stream) -> int:

@@ -1,5 +1,6 @@
 // Device side of the seeded synthetic-input generator (test and bench
-// infrastructure, not part of the attention library).  The definition is the
+// infrastructure, not part of the attention library), and a read-only
+// bandwidth probe the bench uses as the ceiling of its HBM-bound kernels.  The definition is the
 // one in synth/__init__.py: SplitMix64 output function (Steele, Lea, Flood,
 // OOPSLA 2014) over a counter stream, twelve 16-bit uniforms summed and
 // centred (Irwin-Hall), times 2^-16 * sigma (sigma a power of two, so exact),
@@ -94,9 +95,44 @@ int grid_for(long long n) {
   return (int)g;
 }
 
+// Read-only stream over n16 16-byte words: every word is loaded once (non-coherent
+// path, no L1 allocation), four independent loads in flight per thread per step.
+// The xor of everything read goes to *sink only if it equals a value no input
+// here produces, which keeps the loads without writing anything in practice.
+__global__ void __launch_bounds__(512) read_probe_kernel(const uint4* __restrict__ p, long long n16,
+                                                         unsigned* __restrict__ sink) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  unsigned acc = 0;
+  for (; i + 3 * stride < n16; i += 4 * stride) {
+    uint4 w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(w[u].x), "=r"(w[u].y), "=r"(w[u].z), "=r"(w[u].w)
+                   : "l"(p + i + u * stride));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc ^= w[u].x ^ w[u].y ^ w[u].z ^ w[u].w;
+  }
+  for (; i < n16; i += stride) {
+    const uint4 w = p[i];
+    acc ^= w.x ^ w.y ^ w.z ^ w.w;
+  }
+  if (acc == 0x9E3779B9u) sink[0] = acc;
+}
+
 }  // namespace
 
 extern "C" {
+
+// One launch of the read probe over `bytes` (a multiple of 16, 16-byte aligned
+// buffer) on `stream`: 4 blocks of 512 threads per SM.  sink: one device word.
+int spark_synth_read_probe(const void* buf, long long bytes, void* sink, int sm_count, void* stream) {
+  if (!buf || !sink || bytes <= 0 || (bytes & 15) || ((uintptr_t)buf & 15) || sm_count <= 0) return -1;
+  read_probe_kernel<<<sm_count * 4, 512, 0, (cudaStream_t)stream>>>((const uint4*)buf, bytes / 16,
+                                                                    (unsigned*)sink);
+  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
 
 int spark_synth_fill_tokens(void* out, int B, int T, int H, int D, long long pos0,
                             unsigned long long seed, unsigned long long tid, float sigma, void* stream) {
