@@ -431,63 +431,94 @@ def decode_launches(sa, B: int, layers, q8: bool = False) -> int:
 
 
 def decode_step(sa, layers, pos, ws):
-    """One decode step: per layer, append the new token (RoPE fused on k), then attend (RoPE fused on q)."""
+    """One decode step in two calls per layer: append the new token (RoPE fused on k), then attend
+    (RoPE fused on q)."""
     for L in layers:
         sa.spark_kv_append(L["kc"], L["vc"], L["kn"], L["vn"], pos, L["cfg"], flags=sa.SPARK_ROPE_FUSED)
         sa.spark_attn_decode(L["out"], L["q"], L["g"], L["kc"], L["vc"], pos, L["cfg"], ws,
                              flags=sa.SPARK_ROPE_FUSED)
 
 
+def decode_fused_step(sa, layers, pos, wsf):
+    """One decode step in one launch per layer: append, attention and combine fused (RoPE on q and k)."""
+    for L in layers:
+        sa.spark_attn_decode_fused(L["out"], L["q"], L["kn"], L["vn"], L["g"], L["kc"], L["vc"], pos, L["cfg"], wsf,
+                                   flags=sa.SPARK_ROPE_FUSED)
+
+
+def graph_of(torch, fn):
+    """fn() captured in a CUDA graph (after one eager run on a side stream)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def event_ms(torch, fn, reps: int = 10) -> float:
+    """Mean device time of fn() over reps back-to-back calls on the current stream (CUDA events)."""
+    fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
 def run_decode(torch, sa, synth, dist, args, peaks, world):
-    """One decode step of the 36-layer stack, B=64, 32768 cached tokens, in one CUDA graph."""
+    """One decode step of the 36-layer stack, B=64, 32768 cached tokens, in one CUDA graph: one
+    fused launch per layer (the headline decode figure), and the two-call path on the same caches."""
     dev = torch.device("cuda")
     B, p = DECODE_B, DECODE_CTX
     layers = decode_layers(torch, sa, synth, dev, B, p)
     pos = torch.full((B,), p, dtype=torch.int32, device=dev)
-    ws_bytes = max(sa.spark_decode_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-
-    def step():
-        decode_step(sa, layers, pos, ws)
-
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        step()
-    torch.cuda.current_stream().wait_stream(s)
-    sa.spark_check()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        step()
-    for _ in range(args.warmup):
-        graph.replay()
-    torch.cuda.synchronize()
+    ws = torch.empty(max(sa.spark_decode_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers),
+                     dtype=torch.uint8, device=dev)
+    wsf = torch.zeros(max(sa.spark_decode_fused_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers),
+                      dtype=torch.uint8, device=dev)
     dsteps = max(5, min(args.steps, 30))
-    ms = timed_region(torch, dist, lambda i: graph.replay(), dsteps)
+    res = {}
+    for name, step in (("two_call", lambda: decode_step(sa, layers, pos, ws)),
+                       ("fused", lambda: decode_fused_step(sa, layers, pos, wsf))):
+        graph = graph_of(torch, step)
+        sa.spark_check()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        res[name] = timed_region(torch, dist, lambda i: graph.replay(), dsteps) / dsteps
+        sa.spark_check()
+        del graph
+    ms_step = res["fused"]
+    # one layer of each kind alone, eager, for the rooflines
+    per_kind = {}
+    for name, L in (("sliding", layers[0]), ("full", layers[3])):
+        k_ms = event_ms(torch, lambda: sa.spark_attn_decode_fused(
+            L["out"], L["q"], L["kn"], L["vn"], L["g"], L["kc"], L["vc"], pos, L["cfg"], wsf,
+            flags=sa.SPARK_ROPE_FUSED))
+        nbytes = decode_kv_bytes(B, p, L["kind"])
+        per_kind[name] = {"kernel_us": k_ms * 1e3, "kv_bytes": nbytes,
+                          "roofline": hbm_roofline(f"decode_fused_kernel ({name} layer)", nbytes / (k_ms * 1e-3) / 1e9,
+                                                   peaks, ncu_traffic(f"decode_fused_kernel_{name}"))}
     sa.spark_check()
-    ms_step = ms / dsteps
-    # one full layer's decode alone (append + partial + combine), eager, for the roofline
-    full = layers[3]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = 10
-    e0.record()
-    for _ in range(reps):
-        sa.spark_attn_decode(full["out"], full["q"], full["g"], full["kc"], full["vc"], pos, full["cfg"], ws,
-                             flags=sa.SPARK_ROPE_FUSED)
-    e1.record()
-    torch.cuda.synchronize()
-    k_ms = e0.elapsed_time(e1) / reps
     total_bytes = sum(decode_kv_bytes(B, p, L["kind"]) for L in layers)
-    full_bytes = decode_kv_bytes(B, p, FULL)
     launches = decode_launches(sa, B, layers)
-    del graph, layers, ws
+    del layers, ws, wsf
     torch.cuda.empty_cache()
     return {
         "value": total_bytes * world / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
         "ms_per_step": ms_step, "steps_per_s": 1e3 / ms_step, "kv_bytes_per_step": total_bytes,
-        "workload": f"decode_b{B}_ctx{p}_36layers", "gpu_launches_per_step": launches,
-        "roofline": hbm_roofline("decode_partial_kernel+combine (full layer)", full_bytes / (k_ms * 1e-3) / 1e9,
-                                 peaks, ncu_traffic("decode_partial_kernel_full")),
+        "workload": f"decode_b{B}_ctx{p}_36layers", "gpu_launches_per_step": N_LAYERS,
+        "two_call": {"ms_per_step": res["two_call"], "gpu_launches_per_step": launches,
+                     "value": total_bytes * world / (res["two_call"] * 1e-3) / 1e9},
+        "per_layer_kind": per_kind,
+        "roofline": per_kind["full"]["roofline"],
     }
 
 
@@ -787,22 +818,26 @@ def run_long_decode(torch, sa, synth, dist, args, peaks, world):
         pos = torch.full((B,), p, dtype=torch.int32, device=dev)
         ws = torch.empty(max(sa.spark_decode_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers),
                          dtype=torch.uint8, device=dev)
-        graph = torch.cuda.CUDAGraph()
-        decode_step(sa, layers, pos, ws)
-        torch.cuda.synchronize()
-        with torch.cuda.graph(graph):
-            decode_step(sa, layers, pos, ws)
-        for _ in range(3):
-            graph.replay()
+        wsf = torch.zeros(max(sa.spark_decode_fused_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers),
+                          dtype=torch.uint8, device=dev)
         steps = max(5, min(args.steps, 20))
-        ms = timed_region(torch, dist, lambda i: graph.replay(), steps) / steps
-        sa.spark_check()
+        ms = {}
+        for name, step in (("two_call", lambda: decode_step(sa, layers, pos, ws)),
+                           ("fused", lambda: decode_fused_step(sa, layers, pos, wsf))):
+            graph = graph_of(torch, step)
+            for _ in range(3):
+                graph.replay()
+            ms[name] = timed_region(torch, dist, lambda i: graph.replay(), steps) / steps
+            sa.spark_check()
+            del graph
         total = sum(decode_kv_bytes(B, p, L["kind"]) for L in layers)
-        out[f"b{B}_ctx{ctx}"] = {"value": total * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
-                                 "steps_per_s": 1e3 / ms, "kv_bytes_per_step": total,
-                                 "frac_of_hbm": total / (ms * 1e-3) / 1e9 / (peaks.get("hbm_read_gbs") or
-                                                                             peaks["hbm_gbs"])}
-        del graph, layers, ws
+        m = ms["fused"]
+        out[f"b{B}_ctx{ctx}"] = {"value": total * world / (m * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": m,
+                                 "steps_per_s": 1e3 / m, "kv_bytes_per_step": total,
+                                 "frac_of_hbm": total / (m * 1e-3) / 1e9 / (peaks.get("hbm_read_gbs") or
+                                                                            peaks["hbm_gbs"]),
+                                 "two_call_ms_per_step": ms["two_call"], "gpu_launches_per_step": N_LAYERS}
+        del layers, ws, wsf
         torch.cuda.empty_cache()
     return out
 

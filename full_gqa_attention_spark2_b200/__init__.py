@@ -43,6 +43,7 @@ class SparkLayerCfg(ctypes.Structure):
 _LIB = None
 _P = ctypes.c_void_p
 _I = ctypes.c_int
+_LL = ctypes.c_longlong
 
 
 class SparkPagedKV(ctypes.Structure):
@@ -69,12 +70,17 @@ def _lib():
         "spark_layer_cfg_for_kind": (_I, [_I, cfgp]),
         "spark_kv_cache_bytes": (ctypes.c_longlong, [cfgp, _I, ctypes.c_longlong]),
         "spark_stack_kv_bytes": (ctypes.c_longlong, [_I, ctypes.c_longlong]),
-        "spark_rope_apply": (_I, [_P, _I, _I, _I, _P, cfgp, _P]),
-        "spark_kv_append": (_I, [_P, _P, _I, _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
-        "spark_attn_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
+        "spark_rope_apply": (_I, [_P, _I, _I, _I, _LL, _LL, _P, cfgp, _P]),
+        "spark_kv_append": (_I, [_P, _P, _I, _P, _P, _I, _I, _LL, _LL, _P, cfgp, ctypes.c_uint, _P]),
+        "spark_attn_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _LL, _LL, _LL, _LL, _P, cfgp,
+                                    ctypes.c_uint, _P]),
         "spark_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
-        "spark_attn_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, cfgp, _P, ctypes.c_size_t, ctypes.c_uint, _P]),
+        "spark_attn_decode": (_I, [_P, _P, _LL, _P, _P, _P, _I, _I, _P, cfgp, _P, ctypes.c_size_t, ctypes.c_uint,
+                                   _P]),
         "spark_attn_decode_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
+        "spark_decode_fused_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
+        "spark_attn_decode_fused": (_I, [_P, _P, _LL, _P, _P, _LL, _P, _P, _P, _I, _I, _P, cfgp, _P,
+                                         ctypes.c_size_t, ctypes.c_uint, _P]),
         "spark_decode_static_plan": (ctypes.c_size_t, [_I, _I, cfgp, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
         "spark_kv_cache_q8_bytes": (ctypes.c_longlong, [cfgp, _I, ctypes.c_longlong]),
         "spark_kv_append_q8": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
@@ -113,6 +119,7 @@ def exported_symbols():
     return ["spark_layer_cfg_for_layer", "spark_layer_cfg_for_kind", "spark_kv_cache_bytes",
             "spark_stack_kv_bytes", "spark_rope_apply", "spark_kv_append", "spark_attn_prefill",
             "spark_decode_workspace_bytes", "spark_attn_decode", "spark_attn_decode_static", "spark_decode_static_plan",
+            "spark_decode_fused_workspace_bytes", "spark_attn_decode_fused",
             "spark_kv_cache_q8_bytes", "spark_kv_append_q8", "spark_decode_q8_workspace_bytes",
             "spark_attn_decode_q8", "spark_kv_append_paged", "spark_decode_paged_workspace_bytes",
             "spark_attn_decode_paged", "spark_rope_apply_varlen", "spark_kv_append_varlen",
@@ -171,29 +178,55 @@ def _dev(t: torch.Tensor, name: str, dtype=torch.bfloat16, ndim=None):
     return t.data_ptr()
 
 
+def _tokens(t: torch.Tensor, name: str, heads: int, ndim: int = 4):
+    """Pointer and (sequence, token) element strides of a bf16 token tensor [B, T, heads, 256] (ndim 4)
+    or [B, heads, 256] (ndim 3, token stride 0) whose heads are contiguous rows of 256: a view of a
+    wider projection output is accepted."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be torch.bfloat16, got {t.dtype}")
+    if t.dim() != ndim or t.shape[-1] != 256 or t.shape[-2] != heads:
+        raise ValueError(f"{name} must be [{'B, T, ' if ndim == 4 else 'B, '}{heads}, 256], got {tuple(t.shape)}")
+    if t.stride(-1) != 1 or (heads > 1 and t.stride(-2) != 256):
+        raise ValueError(f"{name}: heads must be contiguous rows of 256 elements")
+    return t.data_ptr(), t.stride(0), (t.stride(1) if ndim == 4 else 0)
+
+
 def spark_rope_apply(x: torch.Tensor, pos0: torch.Tensor, cfg: SparkLayerCfg, stream=None) -> None:
-    """Rotate x [B, T, H, 256] bf16 in place; token t of sequence b is at pos0[b] + t."""
-    px = _dev(x, "x", ndim=4)
+    """Rotate x [B, T, H, 256] bf16 in place (a strided view is allowed); token t of sequence b is at
+    pos0[b] + t."""
+    B, T, H = x.shape[0], x.shape[1], x.shape[2] if x.dim() == 4 else 0
+    px, sB, sT = _tokens(x, "x", H)
     pp = _dev(pos0, "pos0", torch.int32, 1)
-    B, T, H, D = x.shape
-    _raise(_lib().spark_rope_apply(px, B, T, H, pp, ctypes.byref(cfg), _stream(stream)))
+    _raise(_lib().spark_rope_apply(px, B, T, H, sB, sT, pp, ctypes.byref(cfg), _stream(stream)))
 
 
 def spark_kv_append(k_cache, v_cache, k, v, pos0, cfg: SparkLayerCfg, flags: int = 0, stream=None) -> None:
-    """Append k, v [B, T, 4, 256] at positions pos0[b] + t into caches [B, 4, cap, 256]."""
+    """Append k, v [B, T, 4, 256] (views with the same strides allowed) at positions pos0[b] + t into
+    caches [B, 4, cap, 256]."""
     pkc, pvc = _dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4)
-    pk, pv = _dev(k, "k", ndim=4), _dev(v, "v", ndim=4)
+    pk, sB, sT = _tokens(k, "k", 4)
+    pv, vB, vT = _tokens(v, "v", 4)
+    if (vB, vT) != (sB, sT) or k.shape != v.shape:
+        raise ValueError("k and v must have the same shape and strides")
     pp = _dev(pos0, "pos0", torch.int32, 1)
     B, T = k.shape[0], k.shape[1]
     cap = k_cache.shape[2]
-    _raise(_lib().spark_kv_append(pkc, pvc, cap, pk, pv, B, T, pp, ctypes.byref(cfg), flags, _stream(stream)))
+    _raise(_lib().spark_kv_append(pkc, pvc, cap, pk, pv, B, T, sB, sT, pp, ctypes.byref(cfg), flags,
+                                  _stream(stream)))
 
 
 def spark_attn_prefill(out, q, k, v, gate, k_cache, v_cache, pos0, cfg: SparkLayerCfg, flags: int = 0,
                        stream=None) -> None:
-    """Gated GQA attention of a chunk of T queries per sequence (see include/spark_attn.h)."""
+    """Gated GQA attention of a chunk of T queries per sequence (see include/spark_attn.h).  q, k, v may
+    be strided views (e.g. slices of one fused projection output); out and gate are dense."""
     po = _dev(out, "out", ndim=4)
-    pq, pk, pv = _dev(q, "q", ndim=4), _dev(k, "k", ndim=4), _dev(v, "v", ndim=4)
+    pq, q_sB, q_sT = _tokens(q, "q", 16)
+    pk, kv_sB, kv_sT = _tokens(k, "k", 4)
+    pv, vB, vT = _tokens(v, "v", 4)
+    if (vB, vT) != (kv_sB, kv_sT) or k.shape != v.shape or tuple(q.shape[:2]) != tuple(k.shape[:2]):
+        raise ValueError("k and v must have the same shape and strides, and q the same [B, T]")
     pg = _dev(gate, "gate", ndim=3)
     pp = _dev(pos0, "pos0", torch.int32, 1)
     if k_cache is None:
@@ -203,8 +236,8 @@ def spark_attn_prefill(out, q, k, v, gate, k_cache, v_cache, pos0, cfg: SparkLay
         pkc, pvc = _dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4)
         cap = k_cache.shape[2]
     B, T = q.shape[0], q.shape[1]
-    _raise(_lib().spark_attn_prefill(po, pq, pk, pv, pg, pkc, pvc, cap, B, T, pp, ctypes.byref(cfg), flags,
-                                     _stream(stream)))
+    _raise(_lib().spark_attn_prefill(po, pq, pk, pv, pg, pkc, pvc, cap, B, T, q_sB, q_sT, kv_sB, kv_sT, pp,
+                                     ctypes.byref(cfg), flags, _stream(stream)))
 
 
 def spark_decode_cp_record_bytes(B: int) -> int:
@@ -256,8 +289,10 @@ def spark_decode_workspace_bytes(B: int, cap: int, cfg: SparkLayerCfg) -> int:
 
 def spark_attn_decode(out, q, gate, k_cache, v_cache, pos, cfg: SparkLayerCfg, workspace: torch.Tensor,
                       flags: int = 0, stream=None) -> None:
-    """Attention of one new token per sequence at pos[b] (its k/v already appended)."""
-    po, pq = _dev(out, "out", ndim=3), _dev(q, "q", ndim=3)
+    """Attention of one new token per sequence at pos[b] (its k/v already appended); q [B, 16, 256] may be
+    a view with any sequence stride."""
+    po = _dev(out, "out", ndim=3)
+    pq, q_sB, _ = _tokens(q, "q", 16, ndim=3)
     pg = _dev(gate, "gate", ndim=2)
     pkc, pvc = _dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4)
     pp = _dev(pos, "pos", torch.int32, 1)
@@ -266,8 +301,40 @@ def spark_attn_decode(out, q, gate, k_cache, v_cache, pos, cfg: SparkLayerCfg, w
     ws_bytes = workspace.numel() * workspace.element_size()
     B = q.shape[0]
     cap = k_cache.shape[2]
-    _raise(_lib().spark_attn_decode(po, pq, pg, pkc, pvc, cap, B, pp, ctypes.byref(cfg), workspace.data_ptr(),
-                                    ws_bytes, flags, _stream(stream)))
+    _raise(_lib().spark_attn_decode(po, pq, q_sB, pg, pkc, pvc, cap, B, pp, ctypes.byref(cfg),
+                                    workspace.data_ptr(), ws_bytes, flags, _stream(stream)))
+
+
+def spark_decode_fused_workspace_bytes(B: int, cap: int, cfg: SparkLayerCfg) -> int:
+    return int(_lib().spark_decode_fused_workspace_bytes(B, cap, ctypes.byref(cfg)))
+
+
+def spark_decode_fused_workspace(B: int, cap: int, cfg: SparkLayerCfg, device="cuda"):
+    """A zero-filled workspace for spark_attn_decode_fused (it must hold zeros before its first use)."""
+    return torch.zeros(spark_decode_fused_workspace_bytes(B, cap, cfg), dtype=torch.uint8, device=device)
+
+
+def spark_attn_decode_fused(out, q, k, v, gate, k_cache, v_cache, pos, cfg: SparkLayerCfg, workspace,
+                            flags: int = 0, stream=None) -> None:
+    """Append the new token (k, v [B, 4, 256] or [B, 1, 4, 256]) and attend q [B, 16, 256] in one launch
+    (see include/spark_attn.h); workspace from spark_decode_fused_workspace."""
+    po = _dev(out, "out", ndim=3)
+    pq, q_sB, _ = _tokens(q, "q", 16, ndim=3)
+    if k.dim() == 4:
+        k, v = k[:, 0], v[:, 0]
+    pk, kv_sB, _ = _tokens(k, "k", 4, ndim=3)
+    pv, v_sB, _ = _tokens(v, "v", 4, ndim=3)
+    if v_sB != kv_sB:
+        raise ValueError("k and v must have the same strides")
+    pg = _dev(gate, "gate", ndim=2)
+    pkc, pvc = _dev(k_cache, "k_cache", ndim=4), _dev(v_cache, "v_cache", ndim=4)
+    pp = _dev(pos, "pos", torch.int32, 1)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _raise(_lib().spark_attn_decode_fused(po, pq, q_sB, pk, pv, kv_sB, pg, pkc, pvc, k_cache.shape[2], q.shape[0],
+                                          pp, ctypes.byref(cfg), workspace.data_ptr(), ws_bytes, flags,
+                                          _stream(stream)))
 
 
 def spark_attn_decode_static(out, q, gate, k_cache, v_cache, pos, cfg: SparkLayerCfg, flags: int = 0,

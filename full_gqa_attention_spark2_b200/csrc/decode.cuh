@@ -35,7 +35,8 @@ constexpr int kDecSmemBytes = 1024 /*align slack*/ + kDecStages * kDecStageBytes
                               kDecMergeBytes + 1024 /*q, barriers, m/l*/;
 
 struct DecodeParams {
-  const __nv_bfloat16* q;     // [B][16][256]
+  const __nv_bfloat16* q;     // [B][16][256], sequence b at element b * q_sB
+  long long q_sB;
   const int* pos;             // [B]
   float* o_part;              // [B][16][splits][256]
   float* ml_part;             // [B][16][splits][2]
@@ -89,10 +90,194 @@ __device__ __forceinline__ float decode_out_scale(float l, __nv_bfloat16 gate_lo
   return (l > 0.f) ? (1.f / l) * (1.f / (1.f + expf(-gl))) : 0.f;
 }
 
+// Byte address of (key, dim) in a tile of four [kNK keys x 128 B] boxes (one per 64 dims) with
+// the 128-byte swizzle.
+template <int kNK = kDecNK>
 __device__ __forceinline__ uint32_t swz_addr(uint32_t tile, int key, int dim) {
-  // byte address of (key, dim) in a tile of four [64 keys x 128 B] boxes, 128 B swizzle
-  return tile + (uint32_t)(dim >> 6) * kDecBoxBytes + (uint32_t)key * 128u +
+  return tile + (uint32_t)(dim >> 6) * (uint32_t)(kNK * 128) + (uint32_t)key * 128u +
          ((uint32_t)(((dim & 63) >> 3) ^ (key & 7)) << 4);
+}
+
+// ----------------------------------------------- consumer steps, shared ----
+// The decode kernels' consumer warps, kW of them, each take 16 keys of every kNK = 16 kW key tile.
+
+// Stage the four query rows of KV group g (qrow: [4][256]) as bf16 q / 16: rotated at position p
+// first when `rope` (bf16 rounding of the rotated value, as the stand-alone RoPE kernel does), then
+// scaled by 1/16 (exact) and rounded.  Thread tid of nthr.
+__device__ __forceinline__ void dec_stage_q(__nv_bfloat16* qs, const __nv_bfloat16* qrow, int p, bool rope, int rot,
+                                            const RopeFreq& freq, int tid, int nthr) {
+  const int half = rot >> 1;
+  for (int e = tid; e < 4 * kHeadDim; e += nthr) {
+    const int d = e & (kHeadDim - 1);
+    float x = __bfloat162float(qrow[e]);
+    if (rope && d < rot) {
+      const int i = d < half ? d : d - half;
+      const float xp = __bfloat162float(qrow[e + (d < half ? half : -half)]);
+      float c, s;
+      rope_angle(p, pow_u8(freq.f[1], i), c, s);
+      x = __bfloat162float(__float2bfloat16_rn(d < half ? x * c - xp * s : x * c + xp * s));
+    }
+    qs[e] = __float2bfloat16_rn(x * 0.0625f);
+  }
+}
+
+// A warp's A fragments of the staged q rows (rows 4..15 of the m16 tile are zero).
+__device__ __forceinline__ void dec_q_fragments(const __nv_bfloat16* qs, int lane, uint32_t (&qa)[16][2]) {
+  const int gq = lane >> 2, cq = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < 16; ++ks) {
+    if (gq < 4) {
+      qa[ks][0] = *reinterpret_cast<const uint32_t*>(qs + gq * kHeadDim + 16 * ks + 2 * cq);
+      qa[ks][1] = *reinterpret_cast<const uint32_t*>(qs + gq * kHeadDim + 16 * ks + 2 * cq + 8);
+    } else {
+      qa[ks][0] = 0u;
+      qa[ks][1] = 0u;
+    }
+  }
+}
+
+// One K/V tile (kt, vt: its K and V halves in shared memory) for this warp's 16 keys: S = Q K^T
+// (mma.m16n8k16, K from the swizzled tile by ldmatrix), the online softmax in the exp2 domain, and
+// O^T += V^T P^T (V^T by ldmatrix.trans, P from S's registers).  The tile's key k is cache row
+// row0 + k; rows < row_end other than `hole` are visible.  Invisible rows may hold anything, NaN
+// included, and a zero probability does not cancel a NaN, so when the tile has any, this warp
+// first clears the V rows of its own keys there; the clearing is ordered before the stage's next
+// TMA load by a proxy fence.
+template <int kNK>
+__device__ __forceinline__ void dec_consume_tile(uint32_t kt, uint32_t vt, const uint32_t (&qa)[16][2],
+                                                 float (&o)[16][4], float& m_run, float& l_part, int row0,
+                                                 int row_end, int hole, int warp, int lane) {
+  const int cq = lane & 3;
+  const int mi = lane >> 3, r8 = lane & 7;             // ldmatrix: matrix index, row
+  const int key_l = warp * 16 + (mi >> 1) * 8 + r8;    // key row this lane addresses
+  const int dim_off = (mi & 1) * 8;
+  const float kLog2e = 1.4426950408889634f;
+  if (row0 + kNK > row_end || (hole >= row0 && hole < row0 + kNK)) {
+    for (int e = lane; e < 16 * 32; e += 32) {
+      const int key = warp * 16 + (e >> 5);
+      const int row = row0 + key;
+      if (row >= row_end || row == hole)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(swz_addr<kNK>(vt, key, (e & 31) * 8)), "r"(0)
+                     : "memory");
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+  }
+  // S = Q K^T for this warp's 16 keys, two accumulation chains per n-tile
+  float sa[2][2][4];
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) sa[a][c][0] = sa[a][c][1] = sa[a][c][2] = sa[a][c][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 16; ++ks) {
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4(swz_addr<kNK>(kt, key_l, 16 * ks + dim_off), b0, b1, b2, b3);
+    mma_bf16_16816(sa[0][ks & 1], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
+    mma_bf16_16816(sa[1][ks & 1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
+  }
+  // scores of row gq at keys (8*nt + 2*cq + j)
+  const int rbase = row0 + warp * 16;
+  float tv[2][2];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int row = rbase + nt * 8 + 2 * cq + j;
+      const float sv = (sa[nt][0][j] + sa[nt][1][j]) * kLog2e;
+      tv[nt][j] = (row < row_end && row != hole) ? sv : -INFINITY;
+      mx = fmaxf(mx, tv[nt][j]);
+    }
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  const float m_new = fmaxf(m_run, mx);
+  const float m_use = m_new == -INFINITY ? 0.f : m_new;
+  const float alpha = fast_exp2(m_run - m_use);
+  float pv[2][2], psum = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      pv[nt][j] = fast_exp2(tv[nt][j] - m_use);
+      psum += pv[nt][j];
+    }
+  l_part = l_part * alpha + psum;
+  m_run = m_new;
+  const float a_lo = __shfl_sync(0xffffffffu, alpha, (8 * cq) & 31);
+  const float a_hi = __shfl_sync(0xffffffffu, alpha, (8 * cq + 4) & 31);
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    o[t][0] *= a_lo;
+    o[t][1] *= a_hi;
+    o[t][2] *= a_lo;
+    o[t][3] *= a_hi;
+  }
+  const uint32_t pb0 = pack_bf16(pv[0][0], pv[0][1]);
+  const uint32_t pb1 = pack_bf16(pv[1][0], pv[1][1]);
+  // O^T += V^T P^T
+#pragma unroll
+  for (int mt = 0; mt < 16; ++mt) {
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4_t(swz_addr<kNK>(vt, key_l, 16 * mt + dim_off), a0, a1, a2, a3);
+    mma_bf16_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
+  }
+}
+
+// Merge of the kW consumer warps' (m, l, o) through shared memory (mrg_o: kW x 4 heads x 256 floats;
+// sm_m, sm_l: kW x 4).  Afterwards thread (warp w, lane) holds, for each query head hh = w, w + kW,
+// .. < 4 of the group, the merged max ms[i], sum ls[i] and numerator acc[i][k] at dims lane + 32 k.
+// `bar`: the consumers' named barrier; the first one also orders the staged q's last reads.
+template <int kW>
+__device__ __forceinline__ void dec_merge_warps(float* mrg_o, float* sm_m, float* sm_l, const float (&o)[16][4],
+                                                float m_run, float l_part, int warp, int lane,
+                                                float (&ms)[4 / kW], float (&ls)[4 / kW],
+                                                float (&acc)[4 / kW][8]) {
+  const int gq = lane >> 2, cq = lane & 3;
+  float l_row = l_part;
+  l_row += __shfl_xor_sync(0xffffffffu, l_row, 1);
+  l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
+  if (cq == 0 && gq < 4) {
+    sm_m[warp * 4 + gq] = m_run;
+    sm_l[warp * 4 + gq] = l_row;
+  }
+  if (cq < 2) {
+    float* w = mrg_o + warp * 4 * kHeadDim;
+#pragma unroll
+    for (int mt = 0; mt < 16; ++mt) {
+      const int d0 = 16 * mt + gq;
+      w[(2 * cq) * kHeadDim + d0] = o[mt][0];
+      w[(2 * cq + 1) * kHeadDim + d0] = o[mt][1];
+      w[(2 * cq) * kHeadDim + d0 + 8] = o[mt][2];
+      w[(2 * cq + 1) * kHeadDim + d0 + 8] = o[mt][3];
+    }
+  }
+  if (kW == 4) asm volatile("bar.sync 1, 128;" ::: "memory");
+  else asm volatile("bar.sync 1, 64;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 4 / kW; ++i) {
+    const int hh = warp + kW * i;
+    float mw[kW], ew[kW];
+    ms[i] = -INFINITY;
+    ls[i] = 0.f;
+#pragma unroll
+    for (int w = 0; w < kW; ++w) {
+      mw[w] = sm_m[w * 4 + hh];
+      ms[i] = fmaxf(ms[i], mw[w]);
+    }
+#pragma unroll
+    for (int w = 0; w < kW; ++w) {
+      ew[w] = (ms[i] == -INFINITY) ? 0.f : fast_exp2(mw[w] - ms[i]);
+      ls[i] += ew[w] * sm_l[w * 4 + hh];
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float a = 0.f;
+#pragma unroll
+      for (int w = 0; w < kW; ++w) a += ew[w] * mrg_o[(w * 4 + hh) * kHeadDim + lane + 32 * k];
+      acc[i][k] = a;
+    }
+  }
 }
 
 template <bool kPaged>
@@ -170,49 +355,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   // -------------------------------------------------------------- consumers
   const int tid = threadIdx.x;                 // 0..127
-  const int gq = lane >> 2, cq = lane & 3;     // mma fragment row group / column pair
-  {
-    // Stage the four query rows of this KV group: rotate (optional), scale by
-    // 1/16 (exact in binary), round to bf16.
-    const __nv_bfloat16* qrow = P.q + ((long long)b * kNq + g * 4) * kHeadDim;
-    const int half = P.rot >> 1;
-    for (int e = tid; e < 4 * kHeadDim; e += 128) {
-      const int d = e & (kHeadDim - 1);
-      float x = __bfloat162float(qrow[e]);
-      if (P.rope && d < P.rot && !bad) {
-        const int i = d < half ? d : d - half;
-        const float xp = __bfloat162float(qrow[e + (d < half ? half : -half)]);
-        float c, s;
-        rope_angle(p, pow_u8(P.freq.f[1], i), c, s);
-        // bf16 rounding of the rotated value, as the stand-alone RoPE kernel does
-        x = __bfloat162float(__float2bfloat16_rn(d < half ? x * c - xp * s : x * c + xp * s));
-      }
-      qs[e] = __float2bfloat16_rn(x * 0.0625f);
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-  }
+  dec_stage_q(qs, P.q + (long long)b * P.q_sB + g * 4 * kHeadDim, p, P.rope && !bad, P.rot, P.freq, tid, 128);
+  asm volatile("bar.sync 1, 128;" ::: "memory");
   uint32_t qa[16][2];
-#pragma unroll
-  for (int ks = 0; ks < 16; ++ks) {
-    if (gq < 4) {
-      qa[ks][0] = *reinterpret_cast<const uint32_t*>(qs + gq * kHeadDim + 16 * ks + 2 * cq);
-      qa[ks][1] = *reinterpret_cast<const uint32_t*>(qs + gq * kHeadDim + 16 * ks + 2 * cq + 8);
-    } else {
-      qa[ks][0] = 0u;
-      qa[ks][1] = 0u;
-    }
-  }
+  dec_q_fragments(qs, lane, qa);
 
   float o[16][4];
 #pragma unroll
   for (int t = 0; t < 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
   float m_run = -INFINITY, l_part = 0.f;
-  const float kLog2e = 1.4426950408889634f;
-
-  // ldmatrix lane addressing: matrix mi = lane / 8, row r = lane % 8
-  const int mi = lane >> 3, r8 = lane & 7;
-  const int key_l = warp * 16 + (mi >> 1) * 8 + r8;     // key row this lane addresses
-  const int dim_off = (mi & 1) * 8;
 
   for (int i = 0; i < n_tiles; ++i) {
     const int s = i % kDecStages;
@@ -220,145 +371,32 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, (i / kDecStages) & 1, abort_flag, P.timeout_ns, 0x12u)))
       break;
     const uint32_t kt = base + s * kDecStageBytes;
-    const uint32_t vt = kt + kDecTileBytes;
-    const int tile_key0 = key_begin + i * kDecNK;
-    if (tile_key0 + kDecNK > key_end) {
-      // Rows past the last key may hold anything, NaN included, and a zero
-      // probability does not cancel a NaN.  Each warp clears the V rows of its
-      // own keys there (its P.V reads no other rows).  This is the split's
-      // last tile, so no later copy lands in this stage.
-      for (int e = lane; e < 16 * 32; e += 32) {
-        const int key = warp * 16 + (e >> 5);
-        if (tile_key0 + key >= key_end)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(swz_addr(vt, key, (e & 31) * 8)), "r"(0)
-                       : "memory");
-      }
-      __syncwarp();
-    }
-
-    // S = Q K^T for this warp's 16 keys, two accumulation chains per n-tile
-    float sa[2][2][4];
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) sa[a][c][0] = sa[a][c][1] = sa[a][c][2] = sa[a][c][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < 16; ++ks) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(swz_addr(kt, key_l, 16 * ks + dim_off), b0, b1, b2, b3);
-      mma_bf16_16816(sa[0][ks & 1], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
-      mma_bf16_16816(sa[1][ks & 1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
-    }
-    // scores of row gq at keys (8*nt + 2*cq + j)
-    const int kbase = key_begin + i * kDecNK + warp * 16;
-    float tv[2][2];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int kidx = kbase + nt * 8 + 2 * cq + j;
-        const float sv = (sa[nt][0][j] + sa[nt][1][j]) * kLog2e;
-        tv[nt][j] = kidx < key_end ? sv : -INFINITY;
-        mx = fmaxf(mx, tv[nt][j]);
-      }
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(m_run, mx);
-    const float m_use = m_new == -INFINITY ? 0.f : m_new;
-    const float alpha = fast_exp2(m_run - m_use);
-    float pv[2][2], psum = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        pv[nt][j] = fast_exp2(tv[nt][j] - m_use);
-        psum += pv[nt][j];
-      }
-    l_part = l_part * alpha + psum;
-    m_run = m_new;
-    const float a_lo = __shfl_sync(0xffffffffu, alpha, (8 * cq) & 31);
-    const float a_hi = __shfl_sync(0xffffffffu, alpha, (8 * cq + 4) & 31);
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      o[t][0] *= a_lo;
-      o[t][1] *= a_hi;
-      o[t][2] *= a_lo;
-      o[t][3] *= a_hi;
-    }
-    const uint32_t pb0 = pack_bf16(pv[0][0], pv[0][1]);
-    const uint32_t pb1 = pack_bf16(pv[1][0], pv[1][1]);
-
-    // O^T += V^T P^T
-#pragma unroll
-    for (int mt = 0; mt < 16; ++mt) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4_t(swz_addr(vt, key_l, 16 * mt + dim_off), a0, a1, a2, a3);
-      mma_bf16_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
-    }
+    dec_consume_tile<kDecNK>(kt, kt + kDecTileBytes, qa, o, m_run, l_part, key_begin + i * kDecNK, key_end, -1, warp,
+                             lane);
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_empty + 8 * s);
   }
 
   // ----------------------------------------------------- merge the 4 warps
   asm volatile("bar.sync 1, 128;" ::: "memory");    // q staging area is free again
-  float l_row = l_part;
-  l_row += __shfl_xor_sync(0xffffffffu, l_row, 1);
-  l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
-  if (cq == 0 && gq < 4) {
-    sm_m[warp * 4 + gq] = m_run;
-    sm_l[warp * 4 + gq] = l_row;
+  float ms[1], ls[1], acc[1][8];
+  dec_merge_warps<kDecConsumerWarps>(mrg_o, sm_m, sm_l, o, m_run, l_part, warp, lane, ms, ls, acc);
+  const int hh = warp;                            // query head within the group
+  const long long row = ((long long)b * kNq + g * 4 + hh) * P.n_splits + split;
+  if (P.n_splits == 1 && !P.shard) {
+    // a single split is the whole answer: normalise, gate and store it here
+    const float scale = decode_out_scale(ls[0], P.gate[(long long)b * kNq + g * 4 + hh]);
+    __nv_bfloat16* dst = P.out + ((long long)b * kNq + g * 4 + hh) * kHeadDim;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) dst[lane + 32 * k] = __float2bfloat16_rn(acc[0][k] * scale);
+    return;
   }
-  if (cq < 2) {
-    float* w = mrg_o + warp * 4 * kHeadDim;
+  float* dst = P.o_part + row * kHeadDim;
 #pragma unroll
-    for (int mt = 0; mt < 16; ++mt) {
-      const int d0 = 16 * mt + gq;
-      w[(2 * cq) * kHeadDim + d0] = o[mt][0];
-      w[(2 * cq + 1) * kHeadDim + d0] = o[mt][1];
-      w[(2 * cq) * kHeadDim + d0 + 8] = o[mt][2];
-      w[(2 * cq + 1) * kHeadDim + d0 + 8] = o[mt][3];
-    }
-  }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  {
-    const int hh = tid >> 5;                      // query head within the group
-    float mw[kDecConsumerWarps], ms = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kDecConsumerWarps; ++w) {
-      mw[w] = sm_m[w * 4 + hh];
-      ms = fmaxf(ms, mw[w]);
-    }
-    float ew[kDecConsumerWarps], ls = 0.f;
-#pragma unroll
-    for (int w = 0; w < kDecConsumerWarps; ++w) {
-      ew[w] = (ms == -INFINITY) ? 0.f : fast_exp2(mw[w] - ms);
-      ls += ew[w] * sm_l[w * 4 + hh];
-    }
-    const long long row = ((long long)b * kNq + g * 4 + hh) * P.n_splits + split;
-    if (P.n_splits == 1 && !P.shard) {
-      // a single split is the whole answer: normalise, gate and store it here
-      const float scale = decode_out_scale(ls, P.gate[(long long)b * kNq + g * 4 + hh]);
-      __nv_bfloat16* dst = P.out + ((long long)b * kNq + g * 4 + hh) * kHeadDim;
-      for (int d = (tid & 31); d < kHeadDim; d += 32) {
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < kDecConsumerWarps; ++w) acc += ew[w] * mrg_o[(w * 4 + hh) * kHeadDim + d];
-        dst[d] = __float2bfloat16_rn(acc * scale);
-      }
-      return;
-    }
-    float* dst = P.o_part + row * kHeadDim;
-    for (int d = (tid & 31); d < kHeadDim; d += 32) {
-      float acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kDecConsumerWarps; ++w) acc += ew[w] * mrg_o[(w * 4 + hh) * kHeadDim + d];
-      dst[d] = acc;
-    }
-    if ((tid & 31) == 0) {
-      P.ml_part[row * 2 + 0] = ms;
-      P.ml_part[row * 2 + 1] = ls;
-    }
+  for (int k = 0; k < 8; ++k) dst[lane + 32 * k] = acc[0][k];
+  if (lane == 0) {
+    P.ml_part[row * 2 + 0] = ms[0];
+    P.ml_part[row * 2 + 1] = ls[0];
   }
 }
 

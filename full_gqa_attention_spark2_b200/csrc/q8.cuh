@@ -62,7 +62,8 @@ __device__ __forceinline__ int q8_pad(int i) { return i + (i >> 5); }
 __global__ void __launch_bounds__(128) kv_append_q8_kernel(
     uint8_t* __restrict__ k_codes, __half* __restrict__ k_scales, uint8_t* __restrict__ v_codes,
     __half* __restrict__ v_scales, int cap, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, int B, int T, int t_first, const int* __restrict__ pos0, int sliding,
+    const __nv_bfloat16* __restrict__ v, int B, int T, long long sB, long long sT, int t_first,
+    const int* __restrict__ pos0, int sliding,
     int rope, const RopeFreq rf, int rot, CachePages pages, const int* __restrict__ cu, int key_off, int shard) {
   __shared__ float xs[2][kNkv * kHeadDim + kNkv * kHeadDim / 32];
   const int b = blockIdx.y;
@@ -78,7 +79,7 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
   }
   const int pos = p0 + t;
   if (shard && (pos - key_off < 0 || pos - key_off >= cap)) return;   // another rank's position
-  const long long src = (sp.tok0 + t) * kNkv * kHeadDim;
+  const long long src = token_offset(cu, b, t, sp.tok0, sB, sT);
   // thread = one 16-byte chunk (8 dims) of K and of V: head tid / 32, dims 8 (tid % 32) ..
   {
     const uint4 kr = reinterpret_cast<const uint4*>(k + src)[tid];
@@ -279,7 +280,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
   {
     // the group's four query rows: rotate (optional), bf16-round, scale by
     // 1/16; then per row a power of two that keeps |q| below 2^15 in fp16
-    const __nv_bfloat16* qrow = P.q + ((long long)b * kNq + g * 4) * kHeadDim;
+    const __nv_bfloat16* qrow = P.q + (long long)b * P.q_sB + g * 4 * kHeadDim;
     const int half = P.rot >> 1;
     float qv[4];
 #pragma unroll

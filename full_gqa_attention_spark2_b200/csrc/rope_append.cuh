@@ -60,9 +60,11 @@ constexpr int kRopeIters = 8;
 // are in flight together (3x faster on full layers than one head at a time).  k's four heads go
 // one at a time: there the separate instantiation keeps fewer registers and more warps resident,
 // which measured faster.
+// Token rows: dense batches put token t of sequence b at element b * sB + t * sT; packed rows
+// (ragged) put row n at n * sT.  Within a token the H heads are contiguous rows of 256.
 template <bool kAllHeads>
 __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x, int B, int T,
-                                                   int H, const int* __restrict__ pos0,
+                                                   int H, long long sB, long long sT, const int* __restrict__ pos0,
                                                    const RopeFreq rf, int rot, const int* __restrict__ cu) {
   __shared__ double freq[128];
   const int half = rot >> 1;
@@ -99,7 +101,7 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
     float c0, s0, c1, s1;
     rope_angle(pos, freq[2 * j], c0, s0);
     rope_angle(pos, freq[2 * j + 1], c1, s1);
-    __nv_bfloat16* row = x + n * H * kHeadDim;
+    __nv_bfloat16* row = x + (cu == nullptr ? (long long)b * sB + (long long)t * sT : n * sT);
     if constexpr (kAllHeads) {
       uint32_t lo[16], hi[16];
 #pragma unroll
@@ -158,13 +160,20 @@ __device__ __forceinline__ TokenSpan token_span(int b, int T, int t_first, int s
   return TokenSpan{(long long)cu[b], T_b, (sliding && T_b > kWindow) ? T_b - kWindow : 0};
 }
 
+// Element offset of token t of sequence b: dense batches b * sB + t * sT, packed rows (ragged)
+// (tok0 + t) * sT, with tok0 the sequence's first packed row.
+__device__ __forceinline__ long long token_offset(const int* cu, int b, int t, long long tok0, long long sB,
+                                                  long long sT) {
+  return cu == nullptr ? (long long)b * sB + (long long)t * sT : (tok0 + t) * sT;
+}
+
 // Append k/v [B][T][4][256] of T new tokens into caches [B][4][cap][256].
 // One block per written token, thread = (head, 16-byte chunk of 8 dims).
 // Sliding layers (ring of 512 rows) only write the last min(T, 512) tokens.
 __global__ void __launch_bounds__(128) kv_append_kernel(
     __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache, int cap,
-    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int B, int T,
-    int t_first, const int* __restrict__ pos0, int sliding, int rope, const RopeFreq rf, int rot,
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int B, int T, long long sB,
+    long long sT, int t_first, const int* __restrict__ pos0, int sliding, int rope, const RopeFreq rf, int rot,
     CachePages pages, const int* __restrict__ cu, int key_off, int shard) {
   const int b = blockIdx.y;
   const int h = threadIdx.x >> 5;
@@ -182,7 +191,7 @@ __global__ void __launch_bounds__(128) kv_append_kernel(
   // full layers: row = position - key_off (0 unless the cache is one rank's shard of positions)
   const int row = sliding ? (pos & (kWindow - 1)) : pos - key_off;
   if (shard && (row < 0 || row >= cap)) return;   // another rank's position
-  const long long src = ((sp.tok0 + t) * kNkv + h) * kHeadDim;
+  const long long src = token_offset(cu, b, t, sp.tok0, sB, sT) + h * kHeadDim;
   const long long crow = cache_row(pages, b, h, cap, row);
   if (crow < 0) {                        // a page index outside the pool
     if (ch == 0) raise_error(kErrPosition, 0x900u | (unsigned)b);

@@ -14,6 +14,7 @@
 
 #include "../../include/spark_attn.h"
 #include "decode.cuh"
+#include "decode_fused.cuh"
 #include "prefill.cuh"
 #include "prefill2.cuh"
 #include "prefill3.cuh"
@@ -87,6 +88,12 @@ int device_ready(int* dev_out) {
     if (a == cudaSuccess)
       a = cudaFuncSetAttribute(spark::decode_partial_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                spark::kDecSmemBytes);
+    if (a == cudaSuccess)
+      a = cudaFuncSetAttribute(spark::decode_fused_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               spark::DfShape<4>::kSmemBytes);
+    if (a == cudaSuccess)
+      a = cudaFuncSetAttribute(spark::decode_fused_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               spark::DfShape<2>::kSmemBytes);
     cudaError_t b = cudaFuncSetAttribute(spark::prefill2_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          spark::kP2SmemBytes);
@@ -197,6 +204,25 @@ const spark::RopeFreq& rope_freq(const spark_layer_cfg* cfg) { return rope_table
 
 // -------------------------------------------------------------- checks -----
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Element strides of a token tensor [B][T][H][256] whose H heads of 256 are contiguous within a
+// token (a view of a wider projection output is allowed).  sB = sT = 0 selects the dense layout.
+// Otherwise: multiples of 8 elements (16-byte rows), a token's heads fit in sT, sequences do not
+// overlap, and both stay below 2^36 elements (tensor-map strides are below 2^40 bytes).
+int token_strides(int B, int T, int H, long long* sB, long long* sT, const char* what) {
+  const long long row = (long long)H * SPARK_HEAD_DIM;
+  if (*sB == 0 && *sT == 0) {
+    *sT = row;
+    *sB = (long long)T * row;
+    return SPARK_OK;
+  }
+  if (*sT < row || (*sT & 7) || *sB < 0 || (*sB & 7) || *sT >= (1LL << 36) || *sB >= (1LL << 36) ||
+      (B > 1 && *sB < (long long)(T - 1) * *sT + row))
+    return fail(SPARK_ERR_INVALID_ARG, "%s: strides sB=%lld sT=%lld do not describe [%d][%d][%d][256] token rows",
+                what, *sB, *sT, B, T, H);
+  if (B == 1) *sB = (long long)T * *sT;      // unused: any value the tensor maps accept
+  return SPARK_OK;
+}
 
 int check_cfg(const spark_layer_cfg* c) {
   if (!c) return fail(SPARK_ERR_INVALID_ARG, "cfg is NULL");
@@ -328,14 +354,17 @@ int check_view(const CacheView& c, const spark_layer_cfg* cfg) {
 // with sequence b at rows cu_seqlens[b] .. cu_seqlens[b+1]-1 and T the longest.
 // key_off / shard: the cache holds positions key_off .. key_off + cap - 1 of a
 // full layer sharded across ranks; tokens outside that range are skipped.
+// sB, sT: element strides of k and v (0, 0: dense; packed rows of a ragged batch are dense).
 int append_impl(const CacheView& c, const void* k, const void* v, int B, int T, const int* pos0,
                 const spark_layer_cfg* cfg, unsigned flags, void* stream, const int* cu_seqlens = nullptr,
-                int key_off = 0, int shard = 0) {
+                int key_off = 0, int shard = 0, long long sB = 0, long long sT = 0) {
   int rc = check_view(c, cfg);
   if (rc) return rc;
   if (!k || !v || !pos0) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
   if (B <= 0 || B > 65535 || T <= 0 || T > SPARK_MAX_POSITION)
     return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d", B, T);
+  if ((rc = token_strides(B, T, SPARK_N_KV_HEADS, &sB, &sT, "k, v"))) return rc;
+  if (cu_seqlens) sT = (long long)SPARK_N_KV_HEADS * SPARK_HEAD_DIM;
   if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if (!aligned16(k) || !aligned16(v)) return fail(SPARK_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   int dev;
@@ -347,12 +376,12 @@ int append_impl(const CacheView& c, const void* k, const void* v, int B, int T, 
   if (c.q8()) {
     spark::kv_append_q8_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
         (uint8_t*)c.k, (__half*)c.ks, (uint8_t*)c.v, (__half*)c.vs, c.cap, (const __nv_bfloat16*)k,
-        (const __nv_bfloat16*)v, B, T, t_first, pos0, sliding, rope, rope_freq(cfg), cfg->rot_dim, pages_of(c),
-        cu_seqlens, key_off, shard);
+        (const __nv_bfloat16*)v, B, T, sB, sT, t_first, pos0, sliding, rope, rope_freq(cfg), cfg->rot_dim,
+        pages_of(c), cu_seqlens, key_off, shard);
   } else {
     spark::kv_append_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(
         (__nv_bfloat16*)c.k, (__nv_bfloat16*)c.v, c.cap, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, B, T,
-        t_first, pos0, sliding, rope, rope_freq(cfg), cfg->rot_dim, pages_of(c), cu_seqlens, key_off, shard);
+        sB, sT, t_first, pos0, sliding, rope, rope_freq(cfg), cfg->rot_dim, pages_of(c), cu_seqlens, key_off, shard);
   }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, c.q8() ? "kv_append_q8_kernel launch" : "kv_append_kernel launch");
@@ -429,11 +458,14 @@ DecodePlan fit_plan(DecodePlan pl, int B, int tiles, size_t max_bytes) {
 // record != nullptr: context parallelism (a full layer's cache is one rank's
 // shard, positions key_off ..): no output, this rank's record is written instead.
 // fit_ws: the workspace is a fixed array of ws_bytes; the plan is fitted to it.
+// q_sB: element stride between sequences of q (0: dense [B][16][256]).
 int decode_impl(void* out, const void* q, const void* gate, const CacheView& c, int B, const int* pos,
                 const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes, unsigned flags, void* stream,
-                int key_off = 0, float* record = nullptr, bool fit_ws = false) {
+                int key_off = 0, float* record = nullptr, bool fit_ws = false, long long q_sB = 0) {
   int rc = check_view(c, cfg);
   if (rc) return rc;
+  long long q_sT = q_sB ? (long long)SPARK_N_Q_HEADS * SPARK_HEAD_DIM : 0;     // one token per sequence
+  if (B > 0 && B <= 65535 && (rc = token_strides(B, 1, SPARK_N_Q_HEADS, &q_sB, &q_sT, "q"))) return rc;
   if (record) {
     out = record;                      // checked below like an output
     gate = record;
@@ -456,6 +488,7 @@ int decode_impl(void* out, const void* q, const void* gate, const CacheView& c, 
 
   spark::DecodeParams P;
   P.q = (const __nv_bfloat16*)q;
+  P.q_sB = q_sB;
   P.pos = pos;
   P.o_part = (float*)workspace;
   P.ml_part = (float*)workspace + (size_t)B * spark::kNq * pl.n_splits * spark::kHeadDim;
@@ -509,6 +542,119 @@ int decode_impl(void* out, const void* q, const void* gate, const CacheView& c, 
       (__nv_bfloat16*)out, (const __nv_bfloat16*)gate, P.o_part, P.ml_part, pl.n_splits);
   e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_combine_kernel launch");
+}
+
+// ------------------------------------------------------- fused decode ----
+// Split plan of spark_attn_decode_fused.  Full layers: the 64-key, one-block-per-SM shape and the
+// plan of spark_attn_decode.  Sliding layers: the 32-key shape, two blocks per SM; the same cost
+// model with twice the block slots and per-block overhead counted in 32-key tiles.
+struct FusedPlan {
+  int warps;           // consumer warps: 4 (64-key tiles) or 2 (32-key tiles)
+  DecodePlan pl;
+};
+
+FusedPlan fused_plan(int B, int cap, int sliding, int sm_count) {
+  if (!sliding) return FusedPlan{4, decode_plan(B, cap, 0, sm_count)};
+  const int tiles = spark::kWindow / 32;
+  const long long units = (long long)B * spark::kNkv;
+  const int slots = 2 * sm_count;
+  DecodePlan best{1, tiles};
+  double best_cost = 1e300;
+  for (int s = 1; s <= tiles; ++s) {
+    const int tps = (tiles + s - 1) / s;
+    const int s_eff = (tiles + tps - 1) / tps;
+    const long long waves = (units * s_eff + slots - 1) / slots;
+    const double cost = (double)waves * (tps + 4.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = DecodePlan{s_eff, tps};
+    }
+  }
+  return FusedPlan{2, best};
+}
+
+// Workspace: the arrival counters first (B * 4 ints, at a fixed place whatever the plan, so one
+// workspace can serve layers of both kinds in turn), then the partials.
+size_t fused_cnt_bytes(int B) { return ((size_t)B * spark::kNkv * sizeof(int) + 255) & ~(size_t)255; }
+
+size_t decode_fused_ws_bytes(int B, int cap, int sliding, int sm_count) {
+  return fused_cnt_bytes(B) + decode_ws_bytes(B, fused_plan(B, cap, sliding, sm_count).pl);
+}
+
+template <int kW>
+cudaError_t launch_fused(const CUtensorMap& km, const CUtensorMap& vm, const spark::DecodeFusedParams& P, int B,
+                         cudaStream_t st) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)P.n_splits, spark::kNkv, (unsigned)B);
+  lc.blockDim = dim3(spark::DfShape<kW>::kThreads);
+  lc.dynamicSmemBytes = spark::DfShape<kW>::kSmemBytes;
+  lc.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, spark::decode_fused_kernel<kW>, km, vm, P);
+}
+
+int decode_fused_impl(void* out, const void* q, long long q_sB, const void* k, const void* v, long long kv_sB,
+                      const void* gate, void* k_cache, void* v_cache, int cap, int B, const int* pos,
+                      const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes, unsigned flags, void* stream) {
+  const CacheView c = dense_view(k_cache, v_cache, nullptr, nullptr, cap);
+  int rc = check_view(c, cfg);
+  if (rc) return rc;
+  if (!out || !q || !k || !v || !gate || !pos || !workspace) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B > 65535) return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d", B);
+  long long q_sT = q_sB ? (long long)SPARK_N_Q_HEADS * SPARK_HEAD_DIM : 0;      // one token per sequence
+  long long kv_sT = kv_sB ? (long long)SPARK_N_KV_HEADS * SPARK_HEAD_DIM : 0;
+  if ((rc = token_strides(B, 1, SPARK_N_Q_HEADS, &q_sB, &q_sT, "q"))) return rc;
+  if ((rc = token_strides(B, 1, SPARK_N_KV_HEADS, &kv_sB, &kv_sT, "k, v"))) return rc;
+  if (flags & ~SPARK_ROPE_FUSED) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(workspace))
+    return fail(SPARK_ERR_INVALID_ARG, "tensors and workspace must be 16-byte aligned");
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  const int sliding = cfg->kind == SPARK_SLIDING;
+  const int sms = g_dev[dev].sm_count;
+  const FusedPlan fp = fused_plan(B, cap, sliding, sms);
+  if (ws_bytes < decode_fused_ws_bytes(B, cap, sliding, sms))
+    return fail(SPARK_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu needed", ws_bytes,
+                decode_fused_ws_bytes(B, cap, sliding, sms));
+  // K and V maps with boxes of the shape's tile (64-dim slabs of 16 * warps keys)
+  CUtensorMap km, vm;
+  {
+    const cuuint64_t dims[3] = {256, (cuuint64_t)cap, (cuuint64_t)B * 4};
+    const cuuint64_t str[2] = {512, (cuuint64_t)cap * 512};
+    const cuuint32_t box[3] = {64, (cuuint32_t)(16 * fp.warps), 1};
+    if ((rc = make_map(&km, k_cache, 3, dims, str, box))) return rc;
+    if ((rc = make_map(&vm, v_cache, 3, dims, str, box))) return rc;
+  }
+  spark::DecodeFusedParams P;
+  P.q = (const __nv_bfloat16*)q;
+  P.k_new = (const __nv_bfloat16*)k;
+  P.v_new = (const __nv_bfloat16*)v;
+  P.q_sB = q_sB;
+  P.kv_sB = kv_sB;
+  P.gate = (const __nv_bfloat16*)gate;
+  P.pos = pos;
+  P.out = (__nv_bfloat16*)out;
+  P.k_cache = (__nv_bfloat16*)k_cache;
+  P.v_cache = (__nv_bfloat16*)v_cache;
+  P.cnt = (int*)workspace;
+  P.o_part = (float*)((char*)workspace + fused_cnt_bytes(B));
+  P.ml_part = P.o_part + (size_t)B * spark::kNq * fp.pl.n_splits * spark::kHeadDim;
+  P.B = B;
+  P.cap = cap;
+  P.sliding = sliding;
+  P.n_splits = fp.pl.n_splits;
+  P.tiles_per_split = fp.pl.tiles_per_split;
+  P.rope = (flags & SPARK_ROPE_FUSED) ? 1 : 0;
+  P.rot = cfg->rot_dim;
+  P.timeout_ns = wait_timeout_ns();
+  P.freq = rope_freq(cfg);
+  const cudaError_t e = fp.warps == 2 ? launch_fused<2>(km, vm, P, B, (cudaStream_t)stream)
+                                      : launch_fused<4>(km, vm, P, B, (cudaStream_t)stream);
+  return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_fused_kernel launch");
 }
 
 // ------------------------------------------------- context parallelism ----
@@ -611,13 +757,14 @@ long long spark_stack_kv_bytes(int B, long long ctx) {
   return total;
 }
 
-int spark_rope_apply(void* x, int B, int T, int H, const int* pos0, const spark_layer_cfg* cfg,
-                     void* stream) {
+int spark_rope_apply(void* x, int B, int T, int H, long long sB, long long sT, const int* pos0,
+                     const spark_layer_cfg* cfg, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (!x || !pos0) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
   if (B <= 0 || T <= 0 || T > SPARK_MAX_POSITION || (H != 16 && H != 4))
     return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d H=%d", B, T, H);
+  if ((rc = token_strides(B, T, H, &sB, &sT, "x"))) return rc;
   if (!aligned16(x)) return fail(SPARK_ERR_INVALID_ARG, "x must be 16-byte aligned");
   int dev;
   if ((rc = device_ready(&dev))) return rc;
@@ -628,20 +775,21 @@ int spark_rope_apply(void* x, int B, int T, int H, const int* pos0, const spark_
   if (grid > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "too many tokens");
   if (H == 16)
     spark::rope_kernel<true><<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>(
-        (__nv_bfloat16*)x, B, T, H, pos0, rope_freq(cfg), cfg->rot_dim, nullptr);
+        (__nv_bfloat16*)x, B, T, H, sB, sT, pos0, rope_freq(cfg), cfg->rot_dim, nullptr);
   else
     spark::rope_kernel<false><<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>(
-        (__nv_bfloat16*)x, B, T, H, pos0, rope_freq(cfg), cfg->rot_dim, nullptr);
+        (__nv_bfloat16*)x, B, T, H, sB, sT, pos0, rope_freq(cfg), cfg->rot_dim, nullptr);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "rope_kernel launch");
 }
 
 int spark_kv_append(void* k_cache, void* v_cache, int cap, const void* k, const void* v, int B,
-                    int T, const int* pos0, const spark_layer_cfg* cfg, unsigned flags,
+                    int T, long long sB, long long sT, const int* pos0, const spark_layer_cfg* cfg, unsigned flags,
                     void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  return append_impl(dense_view(k_cache, v_cache, nullptr, nullptr, cap), k, v, B, T, pos0, cfg, flags, stream);
+  return append_impl(dense_view(k_cache, v_cache, nullptr, nullptr, cap), k, v, B, T, pos0, cfg, flags, stream,
+                     nullptr, 0, 0, sB, sT);
 }
 
 size_t spark_decode_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg) {
@@ -649,14 +797,29 @@ size_t spark_decode_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg) 
   return decode_ws_for(B, dense_view((void*)1, (void*)1, nullptr, nullptr, cap), cfg);
 }
 
-int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_cache,
+int spark_attn_decode(void* out, const void* q, long long q_sB, const void* gate, const void* k_cache,
                       const void* v_cache, int cap, int B, const int* pos,
                       const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
                       unsigned flags, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
   return decode_impl(out, q, gate, dense_view((void*)k_cache, (void*)v_cache, nullptr, nullptr, cap), B, pos, cfg,
-                     workspace, ws_bytes, flags, stream);
+                     workspace, ws_bytes, flags, stream, 0, nullptr, false, q_sB);
+}
+
+size_t spark_decode_fused_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg) {
+  if (check_cfg(cfg) != SPARK_OK || B <= 0 || B > 65535 || cap <= 0) return 0;
+  return decode_fused_ws_bytes(B, cap, cfg->kind == SPARK_SLIDING, current_sm_count());
+}
+
+int spark_attn_decode_fused(void* out, const void* q, long long q_sB, const void* k, const void* v,
+                            long long kv_sB, const void* gate, void* k_cache, void* v_cache, int cap, int B,
+                            const int* pos, const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
+                            unsigned flags, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  return decode_fused_impl(out, q, q_sB, k, v, kv_sB, gate, k_cache, v_cache, cap, B, pos, cfg, workspace,
+                           ws_bytes, flags, stream);
 }
 
 long long spark_kv_cache_q8_bytes(const spark_layer_cfg* cfg, int B, long long cap) {
@@ -717,8 +880,9 @@ int spark_attn_decode_paged(void* out, const void* q, const void* gate, const sp
 }
 
 int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, const void* gate,
-                       const void* k_cache, const void* v_cache, int cap, int B, int T,
-                       const int* pos0, const spark_layer_cfg* cfg, unsigned flags, void* stream) {
+                       const void* k_cache, const void* v_cache, int cap, int B, int T, long long q_sB,
+                       long long q_sT, long long kv_sB, long long kv_sT, const int* pos0, const spark_layer_cfg* cfg,
+                       unsigned flags, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (!out || !q || !k || !v || !gate || !pos0) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
@@ -726,6 +890,8 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
     return fail(SPARK_ERR_INVALID_ARG, "pass both caches or neither");
   if (B <= 0 || B > 65535 || T <= 0 || T > SPARK_MAX_POSITION)
     return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d", B, T);
+  if ((rc = token_strides(B, T, SPARK_N_Q_HEADS, &q_sB, &q_sT, "q"))) return rc;
+  if ((rc = token_strides(B, T, SPARK_N_KV_HEADS, &kv_sB, &kv_sT, "k, v"))) return rc;
   if (flags & ~(SPARK_ROPE_FUSED | SPARK_APPEND_FUSED)) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if ((flags & SPARK_APPEND_FUSED) && !k_cache)
     return fail(SPARK_ERR_INVALID_ARG, "SPARK_APPEND_FUSED needs the caches to append to");
@@ -740,17 +906,19 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   int dev;
   if ((rc = device_ready(&dev))) return rc;
 
-  // Q, chunk K/V: [B][T][H][256] as 4-D (dim, head, token, batch); caches
-  // [B][4][cap][256] as 3-D (dim, row, batch*head).  128-byte swizzled boxes of 64 dims.
+  // Q, chunk K/V: [B][T][H][256] as 4-D (dim, head, token, batch) with the callers' token and
+  // sequence strides; out dense; caches [B][4][cap][256] as 3-D (dim, row, batch*head).
+  // 128-byte swizzled boxes of 64 dims.
   CUtensorMap qm, km, vm, kcm, vcm, om;
   {
     const cuuint64_t dq[4] = {256, 16, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t sq[3] = {512, 512ull * 16, 512ull * 16 * T};
+    const cuuint64_t sq[3] = {512, 2ull * (cuuint64_t)q_sT, 2ull * (cuuint64_t)q_sB};
+    const cuuint64_t so[3] = {512, 512ull * 16, 512ull * 16 * T};
     const cuuint32_t bq[4] = {64, 1, (cuuint32_t)spark::kPfM, 1};
     if ((rc = make_map(&qm, q, 4, dq, sq, bq))) return rc;
-    if ((rc = make_map(&om, out, 4, dq, sq, bq))) return rc;    // the output has q's layout
+    if ((rc = make_map(&om, out, 4, dq, so, bq))) return rc;
     const cuuint64_t dk[4] = {256, 4, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t sk[3] = {512, 512ull * 4, 512ull * 4 * T};
+    const cuuint64_t sk[3] = {512, 2ull * (cuuint64_t)kv_sT, 2ull * (cuuint64_t)kv_sB};
     const cuuint32_t bk[4] = {64, 1, (cuuint32_t)(spark::kPfN / 2), 1};   // each block of the pair: 64 keys
     const cuuint32_t bv[4] = {64, 1, 32, 1};
     if ((rc = make_map(&km, k, 4, dk, sk, bk))) return rc;
@@ -811,7 +979,7 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   // the chunk's k (rotated) and v into the cache, after the attention on the same stream: a sliding
   // ring's rows are overwritten only once the attention has read them as history
   return append_impl(dense_view((void*)k_cache, (void*)v_cache, nullptr, nullptr, cap), k, v, B, T, pos0, cfg, 0,
-                     stream);
+                     stream, nullptr, 0, 0, kv_sB, kv_sT);
 }
 
 int spark_rope_apply_varlen(void* x, int H, const int* cu_seqlens, int max_seqlen, const int* pos0, int B,
@@ -827,11 +995,13 @@ int spark_rope_apply_varlen(void* x, int H, const int* cu_seqlens, int max_seqle
   const int tok_per_block = 128 / (cfg->rot_dim / 4) * spark::kRopeIters;
   dim3 grid((max_seqlen + tok_per_block - 1) / tok_per_block, B);
   if (H == 16)
-    spark::rope_kernel<true><<<grid, 128, 0, (cudaStream_t)stream>>>((__nv_bfloat16*)x, B, max_seqlen, H, pos0,
-                                                                    rope_freq(cfg), cfg->rot_dim, cu_seqlens);
+    spark::rope_kernel<true><<<grid, 128, 0, (cudaStream_t)stream>>>(
+        (__nv_bfloat16*)x, B, max_seqlen, H, 0, (long long)H * SPARK_HEAD_DIM, pos0, rope_freq(cfg), cfg->rot_dim,
+        cu_seqlens);
   else
-    spark::rope_kernel<false><<<grid, 128, 0, (cudaStream_t)stream>>>((__nv_bfloat16*)x, B, max_seqlen, H, pos0,
-                                                                     rope_freq(cfg), cfg->rot_dim, cu_seqlens);
+    spark::rope_kernel<false><<<grid, 128, 0, (cudaStream_t)stream>>>(
+        (__nv_bfloat16*)x, B, max_seqlen, H, 0, (long long)H * SPARK_HEAD_DIM, pos0, rope_freq(cfg), cfg->rot_dim,
+        cu_seqlens);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "rope_kernel launch");
 }

@@ -22,12 +22,23 @@
  * (x_i, x_{i+rot/2}) turns by angle pos * theta^(-2i/rot).
  *
  * Conventions shared by every call:
- *   - All tensors are bf16 (the q8 cache: uint8 codes and fp16 scales),
- *     contiguous, in device memory, allocated and owned by the caller.  The
- *     library allocates and frees nothing.
+ *   - All tensors are bf16 (the q8 cache: uint8 codes and fp16 scales), in
+ *     device memory, allocated and owned by the caller.  The library
+ *     allocates and frees nothing.  Tensors are contiguous except the token
+ *     tensors q, k, v of the calls that take element strides (sB, sT):
+ *     there, token t of sequence b starts at element b * sB + t * sT and its
+ *     heads are contiguous rows of 256, so q, k and v may be views of one
+ *     fused projection output [B][T][16 + 4 + 4][256] ("Spark-X2.6-4B-FP8
+ *     W8A8" page §三: one q_k_v_proj before attention).  Strides 0, 0 select
+ *     the dense layout; otherwise both are multiples of 8 elements, a token's
+ *     heads fit in sT, sequences do not overlap, and both are below 2^36.
  *   - Positions are absolute (0 <= pos < 2^20).  Per-sequence positions live
  *     in caller-owned device int32 arrays, so a captured CUDA graph can replay
- *     with new positions.
+ *     with new positions.  The T tokens a call takes for sequence b sit at
+ *     consecutive positions pos0[b] .. pos0[b] + T - 1: a prompt chunk
+ *     processed after a history of pos0[b] tokens, as the pages measure
+ *     prefill ("Sharp-Spark-X2.5-4B-GGUF" page §三, prompt processing at a
+ *     context depth).
  *   - Every call is asynchronous on `stream` (a cudaStream_t, NULL = legacy
  *     default stream) and runs on the current device, which must be sm_100.
  *   - Host-side argument checks run before any launch; on failure nothing is
@@ -103,28 +114,30 @@ long long spark_kv_cache_bytes(const spark_layer_cfg* cfg, int B, long long cap)
  * page §三: only the 9 full layers grow).  Returns -1 on bad arguments. */
 long long spark_stack_kv_bytes(int B, long long ctx);
 
-/* Rotate x [B][T][H][256] in place; token t of sequence b is at position
- * pos0[b] + t (pos0: device int32 [B]).  H is 16 (queries) or 4 (keys).
- * Dims >= cfg->rot_dim are not touched. */
-int spark_rope_apply(void* x, int B, int T, int H, const int* pos0, const spark_layer_cfg* cfg,
-                     void* stream);
+/* Rotate x [B][T][H][256] (element strides sB, sT) in place; token t of
+ * sequence b is at position pos0[b] + t (pos0: device int32 [B]).  H is 16
+ * (queries) or 4 (keys).  Dims >= cfg->rot_dim are not touched. */
+int spark_rope_apply(void* x, int B, int T, int H, long long sB, long long sT, const int* pos0,
+                     const spark_layer_cfg* cfg, void* stream);
 
 /* Append T new tokens per sequence to a layer's K/V cache.  k, v
- * [B][T][4][256]; token t of sequence b is at position pos0[b] + t.
+ * [B][T][4][256], both with element strides sB, sT; token t of sequence b is
+ * at position pos0[b] + t.
  * Full layer: row = position, requires pos0[b] + T <= cap.
  * Sliding layer: cap must be 512; row = position mod 512; only the last
  * min(T, 512) tokens are written (older ones would be overwritten anyway).
  * With SPARK_ROPE_FUSED, k is raw and is rotated on its way into the cache
  * (the k buffer itself is not modified); v is copied bit for bit. */
 int spark_kv_append(void* k_cache, void* v_cache, int cap, const void* k, const void* v, int B,
-                    int T, const int* pos0, const spark_layer_cfg* cfg, unsigned flags,
-                    void* stream);
+                    int T, long long sB, long long sT, const int* pos0, const spark_layer_cfg* cfg,
+                    unsigned flags, void* stream);
 
 /* Attention of a chunk of T queries per sequence (prefill).
  *   q [B][T][16][256] (rotated, or raw with SPARK_ROPE_FUSED: the kernel then
  *   rotates each Q tile in shared memory after loading it; q itself is not
- *   modified), k [B][T][4][256] rotated, v [B][T][4][256], gate [B][T][16];
- *   out [B][T][16][256].
+ *   modified; element strides q_sB, q_sT), k [B][T][4][256] rotated and
+ *   v [B][T][4][256] (element strides kv_sB, kv_sT), gate [B][T][16];
+ *   out [B][T][16][256] (dense).
  *   Token t of sequence b is at position pos0[b] + t (pos0: device int32 [B]).
  *   The chunk's own keys come from k/v.  Earlier keys (the history,
  *   positions < pos0[b]) come from the cache: full layers read rows
@@ -141,8 +154,9 @@ int spark_kv_append(void* k_cache, void* v_cache, int cap, const void* k, const 
  * therefore best attended without caches and appended by spark_kv_append.
  * Device requirements: sm_100a, about 225 KB of shared memory per block. */
 int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, const void* gate,
-                       const void* k_cache, const void* v_cache, int cap, int B, int T,
-                       const int* pos0, const spark_layer_cfg* cfg, unsigned flags, void* stream);
+                       const void* k_cache, const void* v_cache, int cap, int B, int T, long long q_sB,
+                       long long q_sT, long long kv_sB, long long kv_sT, const int* pos0,
+                       const spark_layer_cfg* cfg, unsigned flags, void* stream);
 
 /* Workspace bytes spark_attn_decode needs for B sequences and cache capacity
  * cap (split-KV partials: per sequence, query head and split, 256 + 2 fp32).
@@ -150,8 +164,9 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
 size_t spark_decode_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg);
 
 /* Attention of one new token per sequence (decode, append-then-attend).
- *   q [B][16][256] (rotated, or raw with SPARK_ROPE_FUSED), gate [B][16];
- *   out [B][16][256].  The new token of sequence b is at position pos[b]
+ *   q [B][16][256] (rotated, or raw with SPARK_ROPE_FUSED; sequence b at
+ *   element b * q_sB, 0: dense), gate [B][16]; out [B][16][256].  The new
+ *   token of sequence b is at position pos[b]
  *   (device int32 [B]) and its k/v must already be in the cache.
  *   Full layer: attends to cache rows 0..pos[b] (pos[b] < cap).
  *   Sliding layer (cap 512): attends to ring rows 0..min(pos[b], 511), which
@@ -161,10 +176,43 @@ size_t spark_decode_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg);
  *   that share a workspace must not overlap on the device.  When the split
  *   plan has one split per (sequence, KV head), as for sliding layers at
  *   B >= 37, one kernel writes `out` directly and the workspace is unused. */
-int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_cache,
+int spark_attn_decode(void* out, const void* q, long long q_sB, const void* gate, const void* k_cache,
                       const void* v_cache, int cap, int B, const int* pos,
                       const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
                       unsigned flags, void* stream);
+
+/* One decode layer in one launch: the append of the new token and the
+ * attention of spark_attn_decode, fused (the two calls spark_kv_append +
+ * spark_attn_decode give the same result up to fp32 rounding order).
+ *   q [B][16][256] and k, v [B][4][256] (sequence b at elements b * q_sB and
+ *   b * kv_sB, 0: dense): the new token of each sequence at
+ *   position pos[b] (raw with SPARK_ROPE_FUSED: q and k are rotated at
+ *   pos[b] here; k is written into the cache rotated and rounded to bf16,
+ *   exactly as spark_kv_append writes it; v bit for bit).  gate [B][16];
+ *   out [B][16][256].  k_cache, v_cache [B][4][cap][256] as for
+ *   spark_kv_append / spark_attn_decode: the call writes row pos[b] (full,
+ *   pos[b] < cap) or pos[b] mod 512 (sliding, cap 512) and attends to
+ *   positions 0..pos[b] (full) or max(0, pos[b] - 511)..pos[b] (sliding), the
+ *   new token's key and value taken from k and v.  Cache rows past the last
+ *   cached position may hold anything.
+ *   workspace: caller-owned device memory of at least
+ *   spark_decode_fused_workspace_bytes(B, cap, cfg) bytes, 16-byte aligned,
+ *   which must hold zeros before its first use (cudaMemsetAsync once after
+ *   allocating it).  Its last B * 4 ints count, per (sequence, KV head), the
+ *   blocks that have finished their share; every call that completes leaves
+ *   them at zero again, so one workspace serves any number of calls and
+ *   layers in turn.  After a call that spark_check() reported as failed
+ *   (a wait that ran out), zero it again.  Calls that share a workspace must
+ *   not overlap on the device.
+ * The kernel is launched with programmatic stream serialisation: its blocks
+ * may be scheduled while the previous kernel of the stream is still running,
+ * but they read and write memory only after that kernel has completed. */
+size_t spark_decode_fused_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg);
+
+int spark_attn_decode_fused(void* out, const void* q, long long q_sB, const void* k, const void* v,
+                            long long kv_sB, const void* gate, void* k_cache, void* v_cache, int cap, int B,
+                            const int* pos, const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
+                            unsigned flags, void* stream);
 
 /* Size of the fixed scratch array spark_attn_decode_static uses. */
 #define SPARK_STATIC_SCRATCH_BYTES (16u << 20)
@@ -174,7 +222,8 @@ int spark_attn_decode(void* out, const void* q, const void* gate, const void* k_
  * front and forbid allocation later, some only lend the library their inputs
  * and outputs, and code recording a CUDA graph cannot record cudaMalloc.  This
  * call computes exactly what spark_attn_decode computes, with the same
- * arguments minus the workspace: the split-KV partials go to a fixed
+ * arguments minus q's stride (q is dense) and the workspace: the split-KV
+ * partials go to a fixed
  * SPARK_STATIC_SCRATCH_BYTES array in the library's own device memory, which
  * every GPU that loads the library holds until the process exits.  It calls no
  * allocating routine.

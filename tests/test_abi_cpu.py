@@ -91,10 +91,49 @@ def test_host_argument_checks_run_before_the_device(lib):
     assert L.spark_decode_cp_record_bytes(3) == 3 * 16 * 257 * 4
     assert L.spark_decode_cp_record_bytes(0) == 0
     # prefill: SPARK_APPEND_FUSED needs the caches; unknown flags are refused
-    args = (fake, fake, fake, fake, fake, None, None, 0, 1, 128, fake, ctypes.byref(full))
+    args = (fake, fake, fake, fake, fake, None, None, 0, 1, 128, 0, 0, 0, 0, fake, ctypes.byref(full))
     assert L.spark_attn_prefill(*args, sa.SPARK_APPEND_FUSED, None) == -1
     assert L.spark_attn_prefill(*args, 0x80, None) == -1
     assert "SPARK_APPEND_FUSED" in sa.spark_last_error() or "flags" in sa.spark_last_error()
+
+
+def test_token_strides_are_checked_on_the_host(lib):
+    """Element strides of the token tensors: 0, 0 is the dense layout; a view of a fused projection
+    output [B, T, 24, 256] is accepted; rows that are not 16-byte multiples, heads that do not fit a
+    token, or sequences that overlap are refused before any device call."""
+    import full_gqa_attention_spark2_b200 as sa
+    L = sa._lib()
+    full = ctypes.byref(sa.spark_layer_cfg_for_kind(sa.SPARK_FULL))
+    fake = ctypes.c_void_p(1 << 20)
+    B, T = 2, 100
+    bad_q = [(T * 4096, 4100), (T * 4096, 2048), (99 * 4096, 4096), (T * 4096 + 4, 4096)]
+    for sB, sT in bad_q:
+        assert L.spark_rope_apply(fake, B, T, 16, sB, sT, fake, full, None) == -1, (sB, sT)
+        assert "strides" in sa.spark_last_error()
+        assert L.spark_attn_prefill(fake, fake, fake, fake, fake, None, None, 0, B, T, sB, sT, 0, 0, fake, full, 0,
+                                    None) == -1, (sB, sT)
+    for sB, sT in [(T * 1024, 1028), (T * 1024, 512), (50 * 1024, 1024)]:
+        assert L.spark_kv_append(fake, fake, 4096, fake, fake, B, T, sB, sT, fake, full, 0, None) == -1, (sB, sT)
+        assert L.spark_attn_prefill(fake, fake, fake, fake, fake, None, None, 0, B, T, 0, 0, sB, sT, fake, full, 0,
+                                    None) == -1, (sB, sT)
+    # decode: q's sequence stride must hold a token's 16 heads and keep 16-byte rows
+    for q_sB in (4000, 4100):
+        assert L.spark_attn_decode(fake, fake, q_sB, fake, fake, fake, 64, B, fake, full, fake, 1 << 30, 0,
+                                   None) == -1, q_sB
+        assert L.spark_attn_decode_fused(fake, fake, q_sB, fake, fake, 0, fake, fake, fake, 64, B, fake, full, fake,
+                                         1 << 30, 0, None) == -1, q_sB
+    assert L.spark_attn_decode_fused(fake, fake, 0, fake, fake, 1000, fake, fake, fake, 64, B, fake, full, fake,
+                                     1 << 30, 0, None) == -1
+    # views of one [B, T, 24, 256] projection output pass the host checks (and fail later, at the device)
+    sB, sT = T * 24 * 256, 24 * 256
+    assert L.spark_rope_apply(fake, B, T, 16, sB, sT, fake, full, None) not in (0, -1)
+    assert L.spark_kv_append(fake, fake, 4096, fake, fake, B, T, sB, sT, fake, full, 0, None) not in (0, -1)
+    assert L.spark_attn_prefill(fake, fake, fake, fake, fake, None, None, 0, B, T, sB, sT, sB, sT, fake, full, 0,
+                                None) not in (0, -1)
+    assert L.spark_attn_decode(fake, fake, 24 * 256, fake, fake, fake, 64, B, fake, full, fake, 1 << 30, 0,
+                               None) not in (0, -1)
+    assert L.spark_attn_decode_fused(fake, fake, 24 * 256, fake, fake, 24 * 256, fake, fake, fake, 64, B, fake, full,
+                                     fake, 1 << 30, 0, None) not in (0, -1)
 
 
 def test_static_decode_plan_fits_and_covers_every_tile(lib):
