@@ -1029,6 +1029,16 @@ def run_profile_case(torch, sa, synth, which: str):
         ws = torch.empty(sa.spark_decode_workspace_bytes(B, p + 1, cfg), dtype=torch.uint8, device=dev)
         for _ in range(3):
             sa.spark_attn_decode(out, q.view(B, HQ, D), g.view(B, HQ), kc, vc, pos, cfg, ws, flags=sa.SPARK_ROPE_FUSED)
+    elif which in ("decode_fused_full", "decode_fused_sliding"):
+        # one layer of the fused decode: full, B=16 at 32768 (2.1 GB of KV); sliding, B=128 (268 MB > L2)
+        full = which == "decode_fused_full"
+        B, p = (16, DECODE_CTX) if full else (128, DECODE_CTX)
+        L = decode_layers(torch, sa, synth, dev, B, p, (3,) if full else (0,))[0]
+        pos = torch.full((B,), p, dtype=torch.int32, device=dev)
+        wsf = torch.zeros(sa.spark_decode_fused_workspace_bytes(B, L["cap"], L["cfg"]), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            sa.spark_attn_decode_fused(L["out"], L["q"], L["kn"], L["vn"], L["g"], L["kc"], L["vc"], pos, L["cfg"], wsf,
+                                       flags=sa.SPARK_ROPE_FUSED)
     elif which == "prefill_ragged_full":
         # run_prefill_ragged at its smallest: the second prefill2_kernel launch is the full layer's
         import types
@@ -1059,7 +1069,7 @@ def main():
     ap.add_argument("--cp-decode", action="store_true",
                     help="also run context-parallel decode (B=1 at 2^20, full-layer caches split over the ranks)")
     ap.add_argument("--profile", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_q8_full",
-                                          "prefill_ragged_full"],
+                                          "prefill_ragged_full", "decode_fused_full", "decode_fused_sliding"],
                     default=None,
                     help="run a small case of one kernel for ncu and exit")
     args = ap.parse_args()

@@ -49,6 +49,9 @@ __device__ __forceinline__ void pf_unit_of(const PrefillParams& P, int u, PfUnit
   x.b = id >> 2;
 }
 
+// The sequence of unit u.
+__device__ __forceinline__ int pf_batch_of(const PrefillParams& P, int u) { return ((u >> 1) / P.n_qt) >> 2; }
+
 constexpr int kUq = 8;          // unit queue entries
 constexpr int kUqReaders = 14;  // per entry: MMA thread, 2 Q warps, 4 softmax warps (even block);
                                 // producer, 2 Q warps, 4 softmax warps (odd block)
@@ -85,17 +88,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   const uint32_t bar_uq_full = misc + 184;          // [kUq] unit queue entry written (both)
   const uint32_t bar_uq_empty = misc + 248;         // [kUq] entry read by every role (even block's)
   const uint32_t bar_clc = misc + 312;              // cancellation answer landed (even block's)
-  volatile int* uq = reinterpret_cast<volatile int*>(gmisc + 320);   // [kUq] unit ids (-1: none left)
-  const uint32_t clc_resp = misc + 352;             // 16-byte cancellation answer
+  const uint32_t clc_resp = misc + 320;             // 16-byte cancellation answer
+  // [kUq] entries of (unit id, -1: none left; the first position of its sequence)
+  volatile int* uq = reinterpret_cast<volatile int*>(gmisc + 384);
 
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Unit u and its schedule: returns its tile count (0: a bad position, which is flagged).
-  auto unit_schedule = [&](int u, PfUnit& x, PfSchedule& S) -> int {
+  // Unit u (its sequence's first position pos0, read once by the scheduler) and its schedule:
+  // returns its tile count (0: a bad position, which is flagged).
+  auto unit_schedule = [&](int u, int pos0, PfUnit& x, PfSchedule& S) -> int {
     pf_unit_of(P, u, x);
-    const int pos0 = P.pos0[x.b];
     const bool bad = pos0 < 0 || pos0 > kMaxPos - P.T || (P.has_cache && !P.sliding && pos0 > P.cap);
     S = pf_schedule(P, x.qt, bad ? 0 : pos0, bad ? 0 : P.T);
     if (bad) {
@@ -106,9 +110,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   };
   // The k-th unit id of this cluster from the queue (every lane of a warp, or one thread), and
   // the hand-back of its entry (one thread per reader).
-  auto uq_get = [&](int k, int& u, unsigned where) -> bool {
+  auto uq_get = [&](int k, int& u, int& pos0, unsigned where) -> bool {
     if (!mbar_wait_cluster(bar_uq_full + 8 * (k % kUq), (k / kUq) & 1, abort_flag, P.timeout_ns, where)) return false;
-    u = uq[k % kUq];
+    u = uq[2 * (k % kUq)];
+    pos0 = uq[2 * (k % kUq) + 1];
     return true;
   };
   auto uq_release = [&](int k) {
@@ -161,29 +166,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       }
       const int key_half = 64 * (int)rank;       // this block's keys of a K tile
       const int dim_half = 128 * (int)rank;      // this block's dims of a V tile
-      int li = 0, qu = 0;
+      int li = 0;
       bool ok = true;
-      // even block: the scheduler.  Entry k of both blocks' queues gets unit k's id.
-      auto publish = [&](int k, int u) -> bool {
+      // even block: the scheduler.  Entry k of both blocks' queues gets unit k's id and its
+      // sequence's first position.
+      auto publish = [&](int k, int u, int pos0) -> bool {
         const int e = k % kUq;
         if (k >= kUq &&
             !mbar_wait_cluster(bar_uq_empty + 8 * e, ((k / kUq) - 1) & 1, abort_flag, P.timeout_ns, 0x8Du))
           return false;
-        uq[e] = u;
+        uq[2 * e] = u;
+        uq[2 * e + 1] = pos0;
         mbar_arrive(bar_uq_full + 8 * e);
-        asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(mapa_shared(smem_u32((const void*)(uq + e)), 1)), "r"(u)
-                     : "memory");
+        const uint32_t peer = mapa_shared(smem_u32((const void*)(uq + 2 * e)), 1);
+        asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(peer), "r"(u), "r"(pos0) : "memory");
         mbar_arrive_remote_cluster(mapa_shared(bar_uq_full + 8 * e, 1));
         return true;
       };
       int clc_asked = 0, clc_got = 0;        // cancellation requests issued / answered
       bool clc_more = true;                  // no request has come back empty yet
       int u_next = (int)(blockIdx.x >> 1);   // this cluster's own unit first
-      if (leader) ok = publish(0, u_next);
+      int pos0_next = P.pos0[pf_batch_of(P, u_next)];
+      if (leader) ok = publish(0, u_next, pos0_next);
       for (int k = 0; ok; ++k) {
-        int u = u_next;
+        int u = u_next, pos0 = pos0_next;
         if (!leader) {
-          ok = uq_get(k, u, 0x8Eu);
+          ok = uq_get(k, u, pos0, 0x8Eu);
           if (!ok) break;
           uq_release(k);
         }
@@ -200,26 +208,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         }
         PfUnit x;
         PfSchedule S;
-        const int n = unit_schedule(u, x, S);
-        const int h = x.kvh * 4 + x.hp * 2 + (int)rank;
-        bool q_issued = false;
+        const int n = unit_schedule(u, pos0, x, S);
         for (int step = 0; step <= n && ok; ++step) {
           for (int part = 0; part < 2 && ok; ++part) {
             const bool is_k = (part == 0);
             const int j = is_k ? step : step - 1;
             if (j < 0 || j >= n) continue;
-            if (!q_issued && !(is_k && j == 0)) {
-              // after the unit's first K tile: its Q, once the previous unit's S MMAs have read
-              // this block's Q buffer
-              if (qu > 0 && !mbar_wait(bar_q_free, (qu - 1) & 1, abort_flag, P.timeout_ns, 0x80u)) {
-                ok = false;
-                break;
-              }
-              mbar_arrive_expect_tx(bar_q, kPfQBytes);
-              for (int d = 0; d < 4; ++d) tma_load_4d(q_s + d * 16384, &qmap, bar_q, d * 64, h, x.qt * kPfM, x.b);
-              ++qu;
-              q_issued = true;
-            }
             const PfTile t = pf_tile(S, P, j);
             const int s = li % kP2Slots;
             if (li >= kP2Slots &&
@@ -252,6 +246,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         }
         if (leader && ok) {
           u_next = -1;
+          pos0_next = 0;
           if (clc_more) {
             ok = mbar_wait(bar_clc, clc_got & 1, abort_flag, P.timeout_ns, 0x8Fu);
             if (!ok) break;
@@ -271,18 +266,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             if (valid) u_next = (int)(cx >> 1);
             else clc_more = false;
           }
-          ok = publish(k + 1, u_next);
+          if (u_next >= 0) pos0_next = P.pos0[pf_batch_of(P, u_next)];
+          ok = publish(k + 1, u_next, pos0_next);
         }
       }
       // an unanswered cancellation request must land before the block leaves
       if (leader && clc_asked > clc_got) mbar_drain(bar_clc, clc_got & 1, 200000000ull);
-      // never leave with copies in flight: this block's last Q, and (even block) every slot's bytes
-      const bool q_landed = qu == 0 || mbar_drain(bar_q, (qu - 1) & 1, 200000000ull);
+      // never leave with copies in flight: (even block) every slot's bytes
       if (leader) {
-        if (q_landed) {
-          for (int i = max(0, li - kP2Slots); i < li; ++i)
-            if (!mbar_drain(bar_slot_full + 8 * (i % kP2Slots), (i / kP2Slots) & 1, 200000000ull)) break;
-        }
+        for (int i = max(0, li - kP2Slots); i < li; ++i)
+          if (!mbar_drain(bar_slot_full + 8 * (i % kP2Slots), (i / kP2Slots) & 1, 200000000ull)) break;
       } else if (!ok) {
         __nanosleep(200000);   // aborted: let this block's last copies land before the pair leaves
       }
@@ -331,13 +324,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         return true;
       };
       for (int k = 0; ok; ++k) {
-        int u;
-        if (!uq_get(k, u, 0x90u)) break;
+        int u, pos0;
+        if (!uq_get(k, u, pos0, 0x90u)) break;
         uq_release(k);
         if (u < 0) break;
         PfUnit x;
         PfSchedule S;
-        const int n = unit_schedule(u, x, S);
+        const int n = unit_schedule(u, pos0, x, S);
         if (n == 0) continue;
         li_end = li + 2 * n;
         ok = mbar_wait_cluster(bar_q_ready, qu & 1, abort_flag, P.timeout_ns, 0x85u);
@@ -361,12 +354,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     }
     __syncwarp();
   } else if (warp < 4) {
-    // ---------------------------------- Q warps (both): each unit's Q landed, rotated (RoPE at
-    // load, the whole tile: these warps are otherwise idle, so the rotation of the next unit's
-    // Q overlaps the current unit's work), handed to the MMA thread; then (thread 64) the TMA
-    // store of the previous unit's staged output, after which its two slots go back to the
-    // producer.  In time, unit k+1's Q lands before unit k's output is staged.
-    int qu = 0, li = 0;
+    // ---------------------------------- Q warps (both): each unit's Q loaded (thread 64, as soon as
+    // the previous unit's S MMAs have read the Q buffer, so the producer never waits for that),
+    // rotated (RoPE at load, the whole tile: these warps are otherwise idle, so the rotation of
+    // the next unit's Q overlaps the current unit's work), handed to the MMA thread; then (thread
+    // 64) the TMA store of the previous unit's staged output, after which its two slots go back to
+    // the producer.  In time, unit k+1's Q lands before unit k's output is staged.
+    int qu = 0, li = 0, q_issued = 0;
     bool ok = true;
     PfUnit px{0, 0, 0, 0};      // the unit whose output is to be stored
     int p_end = -1;             // its slot counter past its last tile (-1: none)
@@ -391,8 +385,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       return __all_sync(0xffffffffu, good);
     };
     for (int k = 0; ok; ++k) {
-      int u;
-      if (!__all_sync(0xffffffffu, uq_get(k, u, 0x91u))) {
+      int u, pos0;
+      if (!__all_sync(0xffffffffu, uq_get(k, u, pos0, 0x91u))) {
         ok = false;
         break;
       }
@@ -401,9 +395,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       if (u < 0) break;
       PfUnit x;
       PfSchedule S;
-      const int n = unit_schedule(u, x, S);
+      const int n = unit_schedule(u, pos0, x, S);
       if (n == 0) continue;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_q, qu & 1, abort_flag, P.timeout_ns, 0x87u))) {
+      if (threadIdx.x == 64) {
+        // this block's Q tile, once the previous unit's S MMAs have read the buffer
+        if (qu > 0 && !mbar_wait(bar_q_free, (qu - 1) & 1, abort_flag, P.timeout_ns, 0x80u)) {
+          ok = false;
+        } else {
+          const int h = x.kvh * 4 + x.hp * 2 + (int)rank;
+          mbar_arrive_expect_tx(bar_q, kPfQBytes);
+          for (int d = 0; d < 4; ++d) tma_load_4d(q_s + d * 16384, &qmap, bar_q, d * 64, h, x.qt * kPfM, x.b);
+          ++q_issued;
+        }
+      }
+      if (!__all_sync(0xffffffffu, ok) ||
+          !__all_sync(0xffffffffu, mbar_wait(bar_q, qu & 1, abort_flag, P.timeout_ns, 0x87u))) {
         ok = false;
         break;
       }
@@ -426,7 +432,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       ++qu;                     // the last unit's phase of bar_o_staged is qu - 1
       store_prev();
     }
-    if (threadIdx.x == 64) bulk_wait_group0();      // never leave with a store in flight
+    if (threadIdx.x == 64) {
+      bulk_wait_group0();       // never leave with a store in flight,
+      // nor with a Q load in flight (only after an abort: otherwise every issued Q was waited for)
+      if (!ok && q_issued > 0) mbar_drain(bar_q, (q_issued - 1) & 1, 200000000ull);
+    }
   } else {
     // ------------------------------------------------- softmax warps (both)
     const int r = threadIdx.x - 128;
@@ -437,8 +447,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     int jg = 0, qu = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      int u;
-      if (!__all_sync(0xffffffffu, uq_get(k, u, 0x91u))) {
+      int u, pos0;
+      if (!__all_sync(0xffffffffu, uq_get(k, u, pos0, 0x91u))) {
         ok = false;
         break;
       }
@@ -447,7 +457,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       if (u < 0) break;
       PfUnit x;
       PfSchedule S;
-      const int n = unit_schedule(u, x, S);
+      const int n = unit_schedule(u, pos0, x, S);
       if (n == 0) continue;
       const int h = x.kvh * 4 + x.hp * 2 + (int)rank;
       const int qp = S.qp0 + r;
