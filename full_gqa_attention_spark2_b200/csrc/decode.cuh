@@ -101,21 +101,32 @@ __device__ __forceinline__ uint32_t swz_addr(uint32_t tile, int key, int dim) {
 // ----------------------------------------------- consumer steps, shared ----
 // The decode kernels' consumer warps, kW of them, each take 16 keys of every kNK = 16 kW key tile.
 
-// Stage the four query rows of KV group g (qrow: [4][256]) as bf16 q / 16: rotated at position p
-// first when `rope` (bf16 rounding of the rotated value, as the stand-alone RoPE kernel does), then
-// scaled by 1/16 (exact) and rounded.  Thread tid of nthr.
-__device__ __forceinline__ void dec_stage_q(__nv_bfloat16* qs, const __nv_bfloat16* qrow, int p, bool rope, int rot,
-                                            const RopeFreq& freq, int tid, int nthr) {
+// The rotation of position p: (cos, sin) of p f_i for the rot/2 frequencies, one angle per
+// thread (an fp64 reduction and sincosf each, as the RoPE and append kernels compute them), into
+// tab[rot/2] in shared memory.  A block's q rows and new key all turn by these rot/2 angles.
+__device__ __forceinline__ void dec_rope_table(float2* tab, int p, int rot, const RopeFreq& freq, int tid,
+                                               int nthr) {
+  for (int i = tid; i < (rot >> 1); i += nthr) {
+    float c, s;
+    rope_angle(p, freq.f[i], c, s);
+    tab[i] = make_float2(c, s);
+  }
+}
+
+// Stage the four query rows of KV group g (qrow: [4][256]) as bf16 q / 16: rotated first when
+// `rope` by the angles of tab (bf16 rounding of the rotated value, as the stand-alone RoPE kernel
+// does), then scaled by 1/16 (exact) and rounded.  Thread tid of nthr; tab is complete.
+__device__ __forceinline__ void dec_stage_q(__nv_bfloat16* qs, const __nv_bfloat16* qrow, const float2* tab,
+                                            bool rope, int rot, int tid, int nthr) {
   const int half = rot >> 1;
   for (int e = tid; e < 4 * kHeadDim; e += nthr) {
     const int d = e & (kHeadDim - 1);
     float x = __bfloat162float(qrow[e]);
     if (rope && d < rot) {
-      const int i = d < half ? d : d - half;
+      const float2 cs = tab[d < half ? d : d - half];
       const float xp = __bfloat162float(qrow[e + (d < half ? half : -half)]);
-      float c, s;
-      rope_angle(p, pow_u8(freq.f[1], i), c, s);
-      x = __bfloat162float(__float2bfloat16_rn(d < half ? x * c - xp * s : x * c + xp * s));
+      x = __bfloat162float(
+          __float2bfloat16_rn(d < half ? rope_lo(x, xp, cs.x, cs.y) : rope_hi(xp, x, cs.x, cs.y)));
     }
     qs[e] = __float2bfloat16_rn(x * 0.0625f);
   }
@@ -355,7 +366,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   // -------------------------------------------------------------- consumers
   const int tid = threadIdx.x;                 // 0..127
-  dec_stage_q(qs, P.q + (long long)b * P.q_sB + g * 4 * kHeadDim, p, P.rope && !bad, P.rot, P.freq, tid, 128);
+  float2* rtab = reinterpret_cast<float2*>(mrg_o + 4 * kHeadDim);       // after qs, before the loop only
+  if (P.rope && !bad) {
+    dec_rope_table(rtab, p, P.rot, P.freq, tid, 128);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  }
+  dec_stage_q(qs, P.q + (long long)b * P.q_sB + g * 4 * kHeadDim, rtab, P.rope && !bad, P.rot, tid, 128);
   asm volatile("bar.sync 1, 128;" ::: "memory");
   uint32_t qa[16][2];
   dec_q_fragments(qs, lane, qa);
@@ -409,9 +425,11 @@ __global__ void __launch_bounds__(64) decode_combine_kernel(__nv_bfloat16* __res
   const int h = blockIdx.x, b = blockIdx.y;
   const long long row0 = ((long long)b * kNq + h) * n_splits;
   float ms = -INFINITY;
+#pragma unroll 4
   for (int s = 0; s < n_splits; ++s) ms = fmaxf(ms, ml_part[(row0 + s) * 2]);
   float ls = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
   for (int s = 0; s < n_splits; ++s) {
     const float m = ml_part[(row0 + s) * 2];
     const float e = (m == -INFINITY) ? 0.f : fast_exp2(m - ms);
@@ -442,9 +460,11 @@ __global__ void __launch_bounds__(64) decode_cp_reduce_kernel(float* __restrict_
   const int h = blockIdx.x, b = blockIdx.y;
   const long long row0 = ((long long)b * kNq + h) * n_splits;
   float ms = -INFINITY;
+#pragma unroll 4
   for (int s = 0; s < n_splits; ++s) ms = fmaxf(ms, ml_part[(row0 + s) * 2]);
   float ls = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
   for (int s = 0; s < n_splits; ++s) {
     const float m = ml_part[(row0 + s) * 2];
     const float e = (m == -INFINITY) ? 0.f : fast_exp2(m - ms);

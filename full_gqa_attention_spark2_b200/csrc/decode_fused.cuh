@@ -156,7 +156,14 @@ __global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
 
   // -------------------------------------------------------------- consumers
   const int tid = threadIdx.x;
-  dec_stage_q(qs, P.q + (long long)b * P.q_sB + g * 4 * kHeadDim, p, P.rope && !bad, P.rot, P.freq, tid, kNC);
+  // the rotation of position p, for q and the new key (the merge area is free until the merge)
+  float2* rtab = reinterpret_cast<float2*>(mrg_o);
+  if (P.rope && !bad) {
+    dec_rope_table(rtab, p, P.rot, P.freq, tid, kNC);
+    if (kW == 4) asm volatile("bar.sync 1, 128;" ::: "memory");
+    else asm volatile("bar.sync 1, 64;" ::: "memory");
+  }
+  dec_stage_q(qs, P.q + (long long)b * P.q_sB + g * 4 * kHeadDim, rtab, P.rope && !bad, P.rot, tid, kNC);
   if (last_split && !bad) {
     // the new token of (b, g): k rotated as the append kernel rotates it, v as it is; staged for its
     // score below and written into its cache row
@@ -185,12 +192,10 @@ __global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i0 = c * 8 + 2 * e;
-          float c0, s0, c1, s1;
-          rope_angle(p, P.freq.f[i0], c0, s0);
-          rope_angle(p, P.freq.f[i0 + 1], c1, s1);
+          const float2 a0 = rtab[i0], a1 = rtab[i0 + 1];   // the append kernel's angles, bit for bit
           const float l0 = bf16_lo(l[e]), l1 = bf16_hi(l[e]), h0 = bf16_lo(hv[e]), h1 = bf16_hi(hv[e]);
-          l[e] = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
-          hv[e] = pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);
+          l[e] = pack_bf16(rope_lo(l0, h0, a0.x, a0.y), rope_lo(l1, h1, a1.x, a1.y));
+          hv[e] = pack_bf16(rope_hi(l0, h0, a0.x, a0.y), rope_hi(l1, h1, a1.x, a1.y));
         }
         reinterpret_cast<uint4*>(kn_s)[c] = lo;
         reinterpret_cast<uint4*>(kn_s)[pc] = hi;
@@ -294,8 +299,10 @@ __global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
     const long long bh = (long long)b * kNq + g * 4 + hh;
     const long long r0 = bh * P.n_splits;
     float mm = -INFINITY;
+#pragma unroll 4
     for (int s = 0; s < P.n_splits; ++s) mm = fmaxf(mm, __ldcg(P.ml_part + (r0 + s) * 2));
     float L = 0.f, A[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
     for (int s = 0; s < P.n_splits; ++s) {
       const float m = __ldcg(P.ml_part + (r0 + s) * 2);
       const float e = (m == -INFINITY) ? 0.f : fast_exp2(m - mm);

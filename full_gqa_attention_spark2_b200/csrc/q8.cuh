@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
         float c, s;
         rope_angle(pos, rf.f[i], c, s);
         const float xp = xs[0][q8_pad(8 * tid + e + (lo ? half : -half))];
-        r[e] = __bfloat162float(__float2bfloat16_rn(lo ? x * c - xp * s : x * c + xp * s));
+        r[e] = __bfloat162float(__float2bfloat16_rn(lo ? rope_lo(x, xp, c, s) : rope_hi(xp, x, c, s)));
       }
     }
     __syncthreads();
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
         const float xp = __bfloat162float(qrow[e + (d < half ? half : -half)]);
         float c, s;
         rope_angle(p, pow_u8(P.freq.f[1], i), c, s);
-        x = __bfloat162float(__float2bfloat16_rn(d < half ? x * c - xp * s : x * c + xp * s));
+        x = __bfloat162float(__float2bfloat16_rn(d < half ? rope_lo(x, xp, c, s) : rope_hi(xp, x, c, s)));
       }
       qv[k8] = x * 0.0625f;
       atomicMax(&row_amax[e >> 8], __float_as_uint(fabsf(qv[k8])));

@@ -38,6 +38,17 @@ __device__ __forceinline__ double pow_u8(double r, int n) {
   return y;
 }
 
+// A pair (lo, hi) = (x_i, x_{i+rot/2}) turned by the angle whose cosine and sine are c, s:
+// lo' = lo c - hi s, hi' = hi c + lo s.  The rounding is pinned (the second product rounded,
+// then one fused multiply-add), so every kernel that rotates the same value at the same
+// position writes the same bits whatever the compiler would contract.
+__device__ __forceinline__ float rope_lo(float lo, float hi, float c, float s) {
+  return __fmaf_rn(lo, c, -__fmul_rn(hi, s));
+}
+__device__ __forceinline__ float rope_hi(float lo, float hi, float c, float s) {
+  return __fmaf_rn(hi, c, __fmul_rn(lo, s));
+}
+
 // cos/sin of pos * f for an integer position, via an fp64 reduction mod 2*pi.
 __device__ __forceinline__ void rope_angle(int pos, double f, float& c, float& s) {
   const double kTwoPi = 6.283185307179586476925286766559;
@@ -112,9 +123,10 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
 #pragma unroll
       for (int h = 0; h < 16; ++h) {
         const float l0 = bf16_lo(lo[h]), l1 = bf16_hi(lo[h]), h0 = bf16_lo(hi[h]), h1 = bf16_hi(hi[h]);
-        *reinterpret_cast<uint32_t*>(row + h * kHeadDim + 2 * j) = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
+        *reinterpret_cast<uint32_t*>(row + h * kHeadDim + 2 * j) =
+            pack_bf16(rope_lo(l0, h0, c0, s0), rope_lo(l1, h1, c1, s1));
         *reinterpret_cast<uint32_t*>(row + h * kHeadDim + half + 2 * j) =
-            pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);
+            pack_bf16(rope_hi(l0, h0, c0, s0), rope_hi(l1, h1, c1, s1));
       }
     } else {
       for (int h = 0; h < H; ++h) {
@@ -122,8 +134,8 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
         uint32_t* hi_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + half + 2 * j);
         uint32_t lo = *lo_p, hi = *hi_p;
         float l0 = bf16_lo(lo), l1 = bf16_hi(lo), h0 = bf16_lo(hi), h1 = bf16_hi(hi);
-        *lo_p = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
-        *hi_p = pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);
+        *lo_p = pack_bf16(rope_lo(l0, h0, c0, s0), rope_lo(l1, h1, c1, s1));
+        *hi_p = pack_bf16(rope_hi(l0, h0, c0, s0), rope_hi(l1, h1, c1, s1));
       }
     }
   }
@@ -221,8 +233,8 @@ __global__ void __launch_bounds__(128) kv_append_kernel(
     rope_angle(pos, rf.f[i0], c0, s0);
     rope_angle(pos, rf.f[i0 + 1], c1, s1);
     float l0 = bf16_lo(l[e]), l1 = bf16_hi(l[e]), h0 = bf16_lo(hh[e]), h1 = bf16_hi(hh[e]);
-    l[e] = pack_bf16(l0 * c0 - h0 * s0, l1 * c1 - h1 * s1);
-    hh[e] = pack_bf16(h0 * c0 + l0 * s0, h1 * c1 + l1 * s1);
+    l[e] = pack_bf16(rope_lo(l0, h0, c0, s0), rope_lo(l1, h1, c1, s1));
+    hh[e] = pack_bf16(rope_hi(l0, h0, c0, s0), rope_hi(l1, h1, c1, s1));
   }
   kd[ch] = lo;
   kd[pc] = hi;
