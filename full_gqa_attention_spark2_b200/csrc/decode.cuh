@@ -263,8 +263,7 @@ __device__ __forceinline__ void dec_merge_warps(float* mrg_o, float* sm_m, float
       w[(2 * cq + 1) * kHeadDim + d0 + 8] = o[mt][3];
     }
   }
-  if (kW == 4) asm volatile("bar.sync 1, 128;" ::: "memory");
-  else asm volatile("bar.sync 1, 64;" ::: "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kW) : "memory");
 #pragma unroll
   for (int i = 0; i < 4 / kW; ++i) {
     const int hh = warp + kW * i;

@@ -4,9 +4,15 @@
 // Work.  A block is (split s, KV head g, sequence b), as in
 // decode_partial_kernel: the four query heads of the group against tiles
 // [s * tiles_per_split, (s + 1) * tiles_per_split) of that head's cache rows,
-// streamed by a producer warp through three TMA stages.  Two shapes:
-//   kW = 4 consumer warps, 64-key tiles (192 KB of stages: one block per SM),
-//   kW = 2 consumer warps, 32-key tiles (96 KB: two blocks per SM).
+// streamed through three TMA stages.  The consumers are kG groups of kW warps;
+// group j takes tiles j, j + kG, .. (each warp 16 keys of a 16 kW key tile),
+// so kG tiles are worked on at once.  Two shapes:
+//   kW = 4, kG = 1: 64-key tiles (192 KB of stages: one block per SM) and a
+//     producer warp that streams them;
+//   kW = 2, kG = 2: 32-key tiles (96 KB: two blocks per SM) and no producer
+//     warp: the group that frees a stage issues the load of the tile three
+//     ahead into it.  Two blocks of four warps keep two warps per scheduler,
+//     so a thread keeps its 255 registers (a fifth warp would cap it at 168).
 // Sliding layers use the second: at B=64 their 256 units of 512 keys then run
 // as one wave of 256 blocks on 148 SMs instead of 1.7 waves of one block per
 // SM.  The hardware deals the blocks to the SMs as they free up, which keeps
@@ -43,16 +49,20 @@
 
 namespace spark {
 
-template <int kW>
+template <int kW, int kG>
 struct DfShape {
   static constexpr int kNK = 16 * kW;                      // keys per tile
-  static constexpr int kThreads = (kW + 1) * 32;           // + the producer warp
+  static constexpr int kNW = kW * kG;                      // consumer warps
+  static constexpr bool kProducer = kG == 1;               // a producer warp (else the groups issue)
+  static constexpr int kThreads = (kNW + (kProducer ? 1 : 0)) * 32;
   static constexpr int kBoxBytes = kNK * 128;              // one 64-dim box of the tile
   static constexpr int kTileBytes = 4 * kBoxBytes;         // K (or V) of one tile
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kMergeBytes = kW * 4 * kHeadDim * 4;
-  static constexpr int kMiscBytes = 4096;                  // q rows, new k and v, barriers, m/l, flags
-  static constexpr int kSmemBytes = 1024 /*align slack*/ + kDecStages * kStageBytes + kMergeBytes + kMiscBytes;
+  static constexpr int kMiscBytes = 5120;                  // q rows, new k/v, RoPE angles, barriers, m/l, flags
+  static constexpr int kSmemBytes = 1024 /*align slack*/ + kDecStages * kStageBytes + kMiscBytes;
+  // the warps' merge reuses the stages once every tile has been consumed
+  static_assert(kNW * 4 * kHeadDim * 4 <= kDecStages * kStageBytes, "merge area");
+  static_assert(kNW <= 4, "one query head per consumer warp in the merge");
 };
 
 struct DecodeFusedParams {
@@ -73,29 +83,39 @@ struct DecodeFusedParams {
   RopeFreq freq;
 };
 
-template <int kW>
-__global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
+// Named barrier of the consumer warps (barrier 1, n threads).
+template <int kN>
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kN) : "memory");
+}
+
+template <int kW, int kG>
+__global__ void __launch_bounds__(DfShape<kW, kG>::kThreads, kW == 2 ? 2 : 1)
     decode_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                         const DecodeFusedParams P) {
-  using S = DfShape<kW>;
+  using S = DfShape<kW, kG>;
   constexpr int kNK = S::kNK;
-  constexpr int kNC = 32 * kW;                 // consumer threads
+  constexpr int kNW = S::kNW;
+  constexpr int kNC = 32 * kNW;                // consumer threads
   extern __shared__ uint8_t dsmem[];
   const uint32_t raw = smem_u32(dsmem);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = dsmem + (base - raw);
-  // layout: [stages x (K tile | V tile)] | merge area | q rows, new k/v, barriers, abort, m, l, flag
-  float* mrg_o = reinterpret_cast<float*>(gbase + kDecStages * S::kStageBytes);
-  uint8_t* misc = gbase + kDecStages * S::kStageBytes + S::kMergeBytes;
+  // layout: [stages x (K tile | V tile)] (the merge area once every tile is consumed) |
+  //         q rows, new k/v, RoPE angles, barriers, abort, m, l, flag
+  float* mrg_o = reinterpret_cast<float*>(gbase);
+  uint8_t* misc = gbase + kDecStages * S::kStageBytes;
   __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(misc);            // [4][256], q / 16
   __nv_bfloat16* kn_s = reinterpret_cast<__nv_bfloat16*>(misc + 2048);   // [256], the new key (rotated)
   __nv_bfloat16* vn_s = reinterpret_cast<__nv_bfloat16*>(misc + 2560);   // [256], the new value
-  const uint32_t bar_full = smem_u32(misc + 3072);
+  float2* rtab = reinterpret_cast<float2*>(misc + 3072);                 // [128] angles of position p
+  const uint32_t bar_full = smem_u32(misc + 4096);
   const uint32_t bar_empty = bar_full + 8 * kDecStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 3072 + 16 * kDecStages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4096 + 16 * kDecStages);
   volatile int* last_flag = abort_flag + 1;
-  float* sm_m = reinterpret_cast<float*>(misc + 3072 + 16 * kDecStages + 16);
-  float* sm_l = sm_m + 4 * kW;
+  int* max_issued = const_cast<int*>(abort_flag) + 2;                  // last tile loaded (no producer)
+  float* sm_m = reinterpret_cast<float*>(misc + 4096 + 16 * kDecStages + 16);
+  float* sm_l = sm_m + 4 * kNW;
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -103,12 +123,13 @@ __global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, kW);
+      mbar_init(bar_empty + 8 * s, kW);      // the warps of the group that owns the tile
     }
     *abort_flag = 0;
+    *max_issued = -1;
     fence_mbar_init();
   }
-  if (threadIdx.x == kNC) {
+  if (threadIdx.x == (S::kProducer ? kNC : 0)) {
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&vmap);
   }
@@ -128,7 +149,26 @@ __global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
   const bool last_split = split == P.n_splits - 1;      // adds and writes the new token
   if (bad && last_split && g == 0 && threadIdx.x == 0) raise_error(kErrPosition, 0x340u | (unsigned)b);
 
-  if (warp == kW) {
+  // tile i of this block into stage i % 3 (one thread)
+  auto load_tile = [&](int i) {
+    const int s = i % kDecStages;
+    const uint32_t full = bar_full + 8 * s;
+    mbar_arrive_expect_tx(full, S::kStageBytes);
+    const uint32_t kt = base + s * S::kStageBytes;
+#pragma unroll
+    for (int d = 0; d < 4; ++d) {
+      tma_load_3d(kt + d * S::kBoxBytes, &kmap, full, d * 64, (t_lo + i) * kNK, b * kNkv + g);
+      tma_load_3d(kt + S::kTileBytes + d * S::kBoxBytes, &vmap, full, d * 64, (t_lo + i) * kNK, b * kNkv + g);
+    }
+  };
+  if constexpr (!S::kProducer) {
+    if (threadIdx.x == 0 && n_tiles > 0) {
+      for (int i = 0; i < min(n_tiles, kDecStages); ++i) load_tile(i);
+      atomicMax(max_issued, min(n_tiles, kDecStages) - 1);
+    }
+  }
+
+  if (S::kProducer && warp == kNW) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_tiles > 0) {
       int issued = 0;
@@ -137,14 +177,7 @@ __global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
         if (i >= kDecStages &&
             !mbar_wait(bar_empty + 8 * s, ((i / kDecStages) - 1) & 1, abort_flag, P.timeout_ns, 0x20u))
           break;
-        const uint32_t full = bar_full + 8 * s;
-        mbar_arrive_expect_tx(full, S::kStageBytes);
-        const uint32_t kt = base + s * S::kStageBytes;
-#pragma unroll
-        for (int d = 0; d < 4; ++d) {
-          tma_load_3d(kt + d * S::kBoxBytes, &kmap, full, d * 64, (t_lo + i) * kNK, b * kNkv + g);
-          tma_load_3d(kt + S::kTileBytes + d * S::kBoxBytes, &vmap, full, d * 64, (t_lo + i) * kNK, b * kNkv + g);
-        }
+        load_tile(i);
         issued = i + 1;
       }
       // never leave with copies in flight
@@ -156,12 +189,10 @@ __global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
 
   // -------------------------------------------------------------- consumers
   const int tid = threadIdx.x;
-  // the rotation of position p, for q and the new key (the merge area is free until the merge)
-  float2* rtab = reinterpret_cast<float2*>(mrg_o);
+  // the rotation of position p, for q and the new key
   if (P.rope && !bad) {
     dec_rope_table(rtab, p, P.rot, P.freq, tid, kNC);
-    if (kW == 4) asm volatile("bar.sync 1, 128;" ::: "memory");
-    else asm volatile("bar.sync 1, 64;" ::: "memory");
+    consumers_sync<kNC>();
   }
   dec_stage_q(qs, P.q + (long long)b * P.q_sB + g * 4 * kHeadDim, rtab, P.rope && !bad, P.rot, tid, kNC);
   if (last_split && !bad) {
@@ -204,8 +235,7 @@ __global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
       }
     }
   }
-  if (kW == 4) asm volatile("bar.sync 1, 128;" ::: "memory");
-  else asm volatile("bar.sync 1, 64;" ::: "memory");
+  consumers_sync<kNC>();
   uint32_t qa[16][2];
   dec_q_fragments(qs, lane, qa);
 
@@ -214,18 +244,40 @@ __global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
   for (int t = 0; t < 16; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
   float m_run = -INFINITY, l_part = 0.f;
   bool ok = true;
-  for (int i = 0; i < n_tiles; ++i) {
+  const int grp = warp / kW, wl = warp % kW;    // tile group, warp within it
+  for (int i = grp; i < n_tiles; i += kG) {
     const int s = i % kDecStages;
+    // Without a producer, a stage serves the two groups in turn, so this group can reach tile i while
+    // the stage's previous tile (the other group's) is still in flight; the full barrier's parity
+    // would then name that earlier phase.  Waiting first until the other group has released the
+    // stage (its empty phase cannot run ahead: the next one needs this group) makes the full wait
+    // name this tile's phase.
+    if (!S::kProducer && i >= kDecStages &&
+        !__all_sync(0xffffffffu, mbar_wait(bar_empty + 8 * s, ((i / kDecStages) - 1) & 1, abort_flag,
+                                           P.timeout_ns, 0x24u))) {
+      ok = false;
+      break;
+    }
     if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, (i / kDecStages) & 1, abort_flag, P.timeout_ns,
                                            0x22u))) {
       ok = false;           // the other warps see the abort flag at their next wait
       break;
     }
     const uint32_t kt = base + s * S::kStageBytes;
-    dec_consume_tile<kNK>(kt, kt + S::kTileBytes, qa, o, m_run, l_part, (t_lo + i) * kNK, row_end, hole, warp,
+    dec_consume_tile<kNK>(kt, kt + S::kTileBytes, qa, o, m_run, l_part, (t_lo + i) * kNK, row_end, hole, wl,
                           lane);
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+    if (!S::kProducer && wl == 0 && lane == 0 && i + kDecStages < n_tiles) {
+      // the group's warps are done with the stage: load the tile three ahead into it
+      if (mbar_wait(bar_empty + 8 * s, (i / kDecStages) & 1, abort_flag, P.timeout_ns, 0x23u)) {
+        load_tile(i + kDecStages);
+        atomicMax(max_issued, i + kDecStages);
+      } else {
+        ok = false;
+      }
+    }
+    if (!S::kProducer && !__all_sync(0xffffffffu, ok)) break;
   }
   {
     // every consumer thread reaches this barrier; a wait that ran out in any warp ends the block here
@@ -238,15 +290,23 @@ __global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
         : "=r"(all_ok)
         : "r"((uint32_t)ok), "n"(kNC)
         : "memory");
-    if (!all_ok) return;
+    if (!all_ok) {
+      if (!S::kProducer && tid == 0) {
+        // never leave with copies in flight: only the last three loads can be outstanding
+        const int mi = *max_issued;
+        for (int j = max(0, mi - (kDecStages - 1)); j <= mi; ++j)
+          mbar_drain(bar_full + 8 * (j % kDecStages), (j / kDecStages) & 1, 200000000ull);
+      }
+      return;
+    }
   }
 
   // -------------------------------------------- merge the consumer warps
-  float ms[4 / kW], ls[4 / kW], acc[4 / kW][8];
-  dec_merge_warps<kW>(mrg_o, sm_m, sm_l, o, m_run, l_part, warp, lane, ms, ls, acc);
+  float ms[4 / kNW], ls[4 / kNW], acc[4 / kNW][8];
+  dec_merge_warps<kNW>(mrg_o, sm_m, sm_l, o, m_run, l_part, warp, lane, ms, ls, acc);
 #pragma unroll
-  for (int i = 0; i < 4 / kW; ++i) {
-    const int hh = warp + kW * i;
+  for (int i = 0; i < 4 / kNW; ++i) {
+    const int hh = warp + kNW * i;
     if (last_split && !bad) {
       // the new token: its score from the same bf16 q / 16 and rotated bf16 key, summed in fp32
       float sdot = 0.f;
@@ -285,17 +345,15 @@ __global__ void __launch_bounds__(DfShape<kW>::kThreads, kW == 2 ? 2 : 1)
 
   // ------------------------- arrival; the unit's last block merges the splits
   __threadfence();
-  if (kW == 4) asm volatile("bar.sync 1, 128;" ::: "memory");
-  else asm volatile("bar.sync 1, 64;" ::: "memory");
+  consumers_sync<kNC>();
   const int unit = b * kNkv + g;
   if (tid == 0) *last_flag = atomicAdd(P.cnt + unit, 1) == P.n_splits - 1;
-  if (kW == 4) asm volatile("bar.sync 1, 128;" ::: "memory");
-  else asm volatile("bar.sync 1, 64;" ::: "memory");
+  consumers_sync<kNC>();
   if (!*last_flag) return;
   __threadfence();
 #pragma unroll
-  for (int i = 0; i < 4 / kW; ++i) {
-    const int hh = warp + kW * i;
+  for (int i = 0; i < 4 / kNW; ++i) {
+    const int hh = warp + kNW * i;
     const long long bh = (long long)b * kNq + g * 4 + hh;
     const long long r0 = bh * P.n_splits;
     float mm = -INFINITY;

@@ -47,7 +47,7 @@ constexpr int kQ8CodeBox = kQ8NK * 128;                     // 8 KB: one 128-dim
 constexpr int kQ8ScaleTile = kQ8NK * 8 * 2;                 // 1 KB: scales of 64 keys
 constexpr int kQ8StageBytes = 2 * kQ8CodeTile + 2 * kQ8ScaleTile;
 constexpr int kQ8QBytes = 4 * kHeadDim * 2;                 // staged q, fp16
-constexpr int kQ8MiscBytes = 512;
+constexpr int kQ8MiscBytes = 1536;   // barriers, flags, m/l; from byte 512 the RoPE angle table
 constexpr int kQ8SmemBytes = 1024 /*align slack*/ + kQ8Stages * kQ8StageBytes + kQ8QBytes + kQ8MiscBytes;
 static_assert(kQ8MergeBytes <= kQ8Stages * kQ8StageBytes, "the merge area reuses the stages");
 static_assert(kQ8StageBytes % 1024 == 0, "128-byte swizzled boxes need 1024-byte alignment");
@@ -282,6 +282,11 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
     // 1/16; then per row a power of two that keeps |q| below 2^15 in fp16
     const __nv_bfloat16* qrow = P.q + (long long)b * P.q_sB + g * 4 * kHeadDim;
     const int half = P.rot >> 1;
+    float2* rtab = reinterpret_cast<float2*>(misc + 512);    // one angle per RoPE frequency
+    if (P.rope && !bad) {
+      dec_rope_table(rtab, p, P.rot, P.freq, tid, 256);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+    }
     float qv[4];
 #pragma unroll
     for (int k8 = 0; k8 < 4; ++k8) {
@@ -289,11 +294,10 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
       const int d = e & (kHeadDim - 1);
       float x = __bfloat162float(qrow[e]);
       if (P.rope && d < P.rot && !bad) {
-        const int i = d < half ? d : d - half;
+        const float2 cs = rtab[d < half ? d : d - half];
         const float xp = __bfloat162float(qrow[e + (d < half ? half : -half)]);
-        float c, s;
-        rope_angle(p, pow_u8(P.freq.f[1], i), c, s);
-        x = __bfloat162float(__float2bfloat16_rn(d < half ? rope_lo(x, xp, c, s) : rope_hi(xp, x, c, s)));
+        x = __bfloat162float(
+            __float2bfloat16_rn(d < half ? rope_lo(x, xp, cs.x, cs.y) : rope_hi(xp, x, cs.x, cs.y)));
       }
       qv[k8] = x * 0.0625f;
       atomicMax(&row_amax[e >> 8], __float_as_uint(fabsf(qv[k8])));

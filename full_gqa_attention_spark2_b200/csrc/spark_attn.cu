@@ -89,11 +89,11 @@ int device_ready(int* dev_out) {
       a = cudaFuncSetAttribute(spark::decode_partial_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                spark::kDecSmemBytes);
     if (a == cudaSuccess)
-      a = cudaFuncSetAttribute(spark::decode_fused_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               spark::DfShape<4>::kSmemBytes);
+      a = cudaFuncSetAttribute(spark::decode_fused_kernel<4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               spark::DfShape<4, 1>::kSmemBytes);
     if (a == cudaSuccess)
-      a = cudaFuncSetAttribute(spark::decode_fused_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               spark::DfShape<2>::kSmemBytes);
+      a = cudaFuncSetAttribute(spark::decode_fused_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               spark::DfShape<2, 2>::kSmemBytes);
     cudaError_t b = cudaFuncSetAttribute(spark::prefill2_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          spark::kP2SmemBytes);
@@ -581,20 +581,20 @@ size_t decode_fused_ws_bytes(int B, int cap, int sliding, int sm_count) {
   return fused_cnt_bytes(B) + decode_ws_bytes(B, fused_plan(B, cap, sliding, sm_count).pl);
 }
 
-template <int kW>
+template <int kW, int kG>
 cudaError_t launch_fused(const CUtensorMap& km, const CUtensorMap& vm, const spark::DecodeFusedParams& P, int B,
                          cudaStream_t st) {
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3((unsigned)P.n_splits, spark::kNkv, (unsigned)B);
-  lc.blockDim = dim3(spark::DfShape<kW>::kThreads);
-  lc.dynamicSmemBytes = spark::DfShape<kW>::kSmemBytes;
+  lc.blockDim = dim3(spark::DfShape<kW, kG>::kThreads);
+  lc.dynamicSmemBytes = spark::DfShape<kW, kG>::kSmemBytes;
   lc.stream = st;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = at;
   lc.numAttrs = 1;
-  return cudaLaunchKernelEx(&lc, spark::decode_fused_kernel<kW>, km, vm, P);
+  return cudaLaunchKernelEx(&lc, spark::decode_fused_kernel<kW, kG>, km, vm, P);
 }
 
 int decode_fused_impl(void* out, const void* q, long long q_sB, const void* k, const void* v, long long kv_sB,
@@ -652,8 +652,8 @@ int decode_fused_impl(void* out, const void* q, long long q_sB, const void* k, c
   P.rot = cfg->rot_dim;
   P.timeout_ns = wait_timeout_ns();
   P.freq = rope_freq(cfg);
-  const cudaError_t e = fp.warps == 2 ? launch_fused<2>(km, vm, P, B, (cudaStream_t)stream)
-                                      : launch_fused<4>(km, vm, P, B, (cudaStream_t)stream);
+  const cudaError_t e = fp.warps == 2 ? launch_fused<2, 2>(km, vm, P, B, (cudaStream_t)stream)
+                                      : launch_fused<4, 1>(km, vm, P, B, (cudaStream_t)stream);
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "decode_fused_kernel launch");
 }
 
