@@ -346,7 +346,12 @@ def run_prefill(torch, sa, synth, dist, args, peaks, world):
         "per_layer_kind": {
             name: {"kernel_us": ms * 1e3, "tok_s": B * T / (ms * 1e-3),
                    "tflops": f / (ms * 1e-3) / 1e12, "algorithmic_flops": f,
-                   "tile_flops": prefill_tile_flops(B, T, kind)}
+                   "tile_flops": prefill_tile_flops(B, T, kind),
+                   "roofline": {"bound": "tensor", "kernel": f"prefill3_kernel ({name} layer)",
+                                "achieved": f / (ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                                "frac": f / (ms * 1e-3) / 1e12 / peak,
+                                "peak_source": f"bf16_tflops burst, {peaks['source']}",
+                                "traffic": ncu_traffic(f"prefill3_kernel_{name}")}}
             for name, kind, ms, f in (("sliding", SLIDING, slide_ms, f_slide), ("full", FULL, kern_ms, f_full))},
         "stack36_derived": {"ms": 27 * slide_ms + 9 * kern_ms,
                             "tok_s": B * T / ((27 * slide_ms + 9 * kern_ms) * 1e-3),
@@ -461,14 +466,17 @@ def graph_of(torch, fn):
 
 
 def event_ms(torch, fn, reps: int = 10) -> float:
-    """Mean device time of fn() over reps back-to-back calls on the current stream (CUDA events)."""
-    fn()
+    """Mean device time of fn() over reps back-to-back calls captured in one CUDA graph (CUDA events
+    around its replay): the calls' own host-side cost does not leave the device idle between them."""
+    g = graph_of(torch, lambda: [fn() for _ in range(reps)])
+    g.replay()
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(reps):
-        fn()
+    g.replay()
     e1.record()
     torch.cuda.synchronize()
+    del g
     return e0.elapsed_time(e1) / reps
 
 
@@ -496,7 +504,7 @@ def run_decode(torch, sa, synth, dist, args, peaks, world):
         sa.spark_check()
         del graph
     ms_step = res["fused"]
-    # one layer of each kind alone, eager, for the rooflines
+    # one layer of each kind alone (ten calls in one CUDA graph) for the rooflines
     per_kind = {}
     for name, L in (("sliding", layers[0]), ("full", layers[3])):
         k_ms = event_ms(torch, lambda: sa.spark_attn_decode_fused(
