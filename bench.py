@@ -801,19 +801,54 @@ def run_long_prefill(torch, sa, synth, dist, args, peaks, world):
                                       flags=sa.SPARK_ROPE_FUSED)
                 sa.spark_kv_append(w["kc"], w["vc"], k, w["v"][:, sl], pos[c], w["cfg"])
 
+    # the same chunks over 8-bit caches: a chunk with history reads it through spark_attn_prefill_q8
+    # (the history dequantised into a workspace, then the bf16 prefill) and appends itself quantised
+    for kind in (SLIDING, FULL):
+        w = L[kind]
+        cap = w["kc"].shape[2]
+        w["kq"] = torch.empty(1, HKV, cap, D, dtype=torch.uint8, device=dev)
+        w["vq"] = torch.empty_like(w["kq"])
+        w["ks"] = torch.empty(1, HKV, cap, D // 32, dtype=torch.float16, device=dev)
+        w["vs"] = torch.empty_like(w["ks"])
+        w["ws"] = torch.empty(sa.spark_prefill_q8_workspace_bytes(1, cap, w["cfg"]), dtype=torch.uint8, device=dev)
+
+    def step_q8(i=0):
+        for kind in (SLIDING, FULL):
+            w = L[kind]
+            for c in range(T // C):
+                sl = slice(c * C, (c + 1) * C)
+                q, k, v, g = w["q"][:, sl], w["k"][:, sl], w["v"][:, sl], w["g"][:, sl]
+                sa.spark_rope_apply(k, pos[c], w["cfg"])
+                if c == 0:
+                    sa.spark_attn_prefill(w["out"][:, sl], q, k, v, g, None, None, pos[c], w["cfg"],
+                                          flags=sa.SPARK_ROPE_FUSED)
+                    sa.spark_kv_append_q8(w["kq"], w["ks"], w["vq"], w["vs"], k, v, pos[c], w["cfg"])
+                else:
+                    sa.spark_attn_prefill_q8(w["out"][:, sl], q, k, v, g, w["kq"], w["ks"], w["vq"], w["vs"], pos[c],
+                                             w["cfg"], w["ws"], flags=sa.SPARK_ROPE_FUSED | sa.SPARK_APPEND_FUSED)
+
     for _ in range(max(1, min(args.warmup, 3))):
         step()
     sa.spark_check()
     steps = max(2, min(args.steps, 5))
     ms = timed_region(torch, dist, step, steps) / steps
     sa.spark_check()
+    for _ in range(max(1, min(args.warmup, 3))):
+        step_q8()
+    sa.spark_check()
+    ms_q8 = timed_region(torch, dist, step_q8, steps) / steps
+    sa.spark_check()
     f_full = sum(prefill_flops(1, C, c * C, FULL, True) for c in range(T // C))
     f_slide = sum(prefill_flops(1, C, c * C, SLIDING, True) for c in range(T // C))
     del L
     torch.cuda.empty_cache()
+    n_ch = T // C
     return {"workload": "long_prefill_b1_t131072_chunks8192_sliding+full", "value": T * world / (ms * 1e-3),
             "unit": "tok/s", "ms_per_step": ms, "tflops": (f_full + f_slide) * world / (ms * 1e-3) / 1e12,
-            "gpu_launches_per_step": 2 * (T // C) * 3}
+            "gpu_launches_per_step": 2 * n_ch * 3,
+            "q8_cache": {"value": T * world / (ms_q8 * 1e-3), "unit": "tok/s", "ms_per_step": ms_q8,
+                         "gpu_launches_per_step": 2 * (3 + (n_ch - 1) * 4),
+                         "note": "history in 8-bit q8_0 caches, dequantised per chunk into a bf16 workspace"}}
 
 
 def run_long_decode(torch, sa, synth, dist, args, peaks, world):

@@ -87,6 +87,9 @@ def _lib():
         "spark_decode_q8_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
         "spark_attn_decode_q8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _P, cfgp, _P, ctypes.c_size_t,
                                       ctypes.c_uint, _P]),
+        "spark_prefill_q8_workspace_bytes": (ctypes.c_size_t, [_I, _I, cfgp]),
+        "spark_attn_prefill_q8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _LL, _LL, _LL, _LL, _P, cfgp,
+                                       _P, ctypes.c_size_t, ctypes.c_uint, _P]),
         "spark_kv_append_paged": (_I, [ctypes.POINTER(SparkPagedKV), _P, _P, _I, _I, _P, cfgp, ctypes.c_uint, _P]),
         "spark_decode_paged_workspace_bytes": (ctypes.c_size_t, [_I, ctypes.POINTER(SparkPagedKV), cfgp]),
         "spark_attn_decode_paged": (_I, [_P, _P, _P, ctypes.POINTER(SparkPagedKV), _I, _P, cfgp, _P,
@@ -121,7 +124,8 @@ def exported_symbols():
             "spark_decode_workspace_bytes", "spark_attn_decode", "spark_attn_decode_static", "spark_decode_static_plan",
             "spark_decode_fused_workspace_bytes", "spark_attn_decode_fused",
             "spark_kv_cache_q8_bytes", "spark_kv_append_q8", "spark_decode_q8_workspace_bytes",
-            "spark_attn_decode_q8", "spark_kv_append_paged", "spark_decode_paged_workspace_bytes",
+            "spark_attn_decode_q8", "spark_prefill_q8_workspace_bytes", "spark_attn_prefill_q8",
+            "spark_kv_append_paged", "spark_decode_paged_workspace_bytes",
             "spark_attn_decode_paged", "spark_rope_apply_varlen", "spark_kv_append_varlen",
             "spark_attn_prefill_varlen", "spark_decode_cp_record_bytes", "spark_kv_append_cp",
             "spark_attn_decode_cp_partial", "spark_attn_decode_cp_merge", "spark_selftest_wait_timeout",
@@ -402,6 +406,33 @@ def spark_attn_decode_q8(out, q, gate, k_codes, k_scales, v_codes, v_scales, pos
     _raise(_lib().spark_attn_decode_q8(po, pq, pg, pkc, pks, pvc, pvs, k_codes.shape[2], q.shape[0], pp,
                                        ctypes.byref(cfg), workspace.data_ptr(), ws_bytes, flags,
                                        _stream(stream)))
+
+
+def spark_prefill_q8_workspace_bytes(B: int, cap: int, cfg: SparkLayerCfg) -> int:
+    return int(_lib().spark_prefill_q8_workspace_bytes(B, cap, ctypes.byref(cfg)))
+
+
+def spark_attn_prefill_q8(out, q, k, v, gate, k_codes, k_scales, v_codes, v_scales, pos0, cfg: SparkLayerCfg,
+                          workspace: torch.Tensor, flags: int = 0, stream=None) -> None:
+    """spark_attn_prefill with the history in 8-bit caches (codes + scales per K and V); workspace: a
+    contiguous CUDA tensor of at least spark_prefill_q8_workspace_bytes(B, cap, cfg) bytes."""
+    po = _dev(out, "out", ndim=4)
+    pq, q_sB, q_sT = _tokens(q, "q", 16)
+    pk, kv_sB, kv_sT = _tokens(k, "k", 4)
+    pv, vB, vT = _tokens(v, "v", 4)
+    if (vB, vT) != (kv_sB, kv_sT) or k.shape != v.shape or tuple(q.shape[:2]) != tuple(k.shape[:2]):
+        raise ValueError("k and v must have the same shape and strides, and q the same [B, T]")
+    pg = _dev(gate, "gate", ndim=3)
+    pp = _dev(pos0, "pos0", torch.int32, 1)
+    pkc, pks = _q8_pair(k_codes, k_scales, "k")
+    pvc, pvs = _q8_pair(v_codes, v_scales, "v")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    B, T = q.shape[0], q.shape[1]
+    _raise(_lib().spark_attn_prefill_q8(po, pq, pk, pv, pg, pkc, pks, pvc, pvs, k_codes.shape[2], B, T, q_sB, q_sT,
+                                        kv_sB, kv_sT, pp, ctypes.byref(cfg), workspace.data_ptr(), ws_bytes, flags,
+                                        _stream(stream)))
 
 
 def paged_kv(k_pool, v_pool, block_table, k_scales=None, v_scales=None) -> SparkPagedKV:

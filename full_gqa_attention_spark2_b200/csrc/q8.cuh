@@ -515,4 +515,37 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
   }
 }
 
+// The history a prefill chunk reads from an 8-bit cache, as bf16 rows in the bf16 cache's layout
+// ([B][4][cap][256]): rows [0, min(pos0[b], cap)) of sequence b (a full layer's positions; a
+// sliding ring's rows, cap 512, which then hold every history position the chunk can see).  Rows
+// past them, and every row of a sequence with a bad position, are left as they are (the prefill
+// never reads them; it flags a bad position itself).  Each value is code * scale, exact in fp32
+// (an 8-bit code times an 11-bit significand), then rounded once to bf16.  One warp per (row,
+// tensor): lane i takes codes 8i .. 8i+7 of block i/4 (256 bytes read, 512 written per warp).
+// Grid (ceil(cap / 4), 4 KV heads, B), 256 threads: warp w takes row 4 blockIdx.x + w/2, K (even
+// w) or V (odd w).
+__global__ void __launch_bounds__(256) q8_history_kernel(const uint8_t* __restrict__ k_codes,
+                                                         const __half* __restrict__ k_scales,
+                                                         const uint8_t* __restrict__ v_codes,
+                                                         const __half* __restrict__ v_scales, int cap,
+                                                         const int* __restrict__ pos0, __nv_bfloat16* __restrict__ k_out,
+                                                         __nv_bfloat16* __restrict__ v_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 4 + (warp >> 1);
+  const int b = blockIdx.z;
+  const int p = pos0[b];
+  if (p < 0 || row >= min(p, cap)) return;
+  const bool is_v = warp & 1;
+  const long long r = ((long long)b * kNkv + blockIdx.y) * cap + row;
+  const uint2 c8 = *reinterpret_cast<const uint2*>((is_v ? v_codes : k_codes) + r * kHeadDim + lane * 8);
+  const float d = __half2float((is_v ? v_scales : k_scales)[r * (kHeadDim / 32) + (lane >> 2)]);
+  auto val = [&](uint32_t w, int i) { return (float)((int)((w >> (8 * i)) & 0xFFu) - 128) * d; };
+  uint4 o;
+  o.x = pack_bf16(val(c8.x, 0), val(c8.x, 1));
+  o.y = pack_bf16(val(c8.x, 2), val(c8.x, 3));
+  o.z = pack_bf16(val(c8.y, 0), val(c8.y, 1));
+  o.w = pack_bf16(val(c8.y, 2), val(c8.y, 3));
+  *reinterpret_cast<uint4*>((is_v ? v_out : k_out) + r * kHeadDim + lane * 8) = o;
+}
+
 }  // namespace spark

@@ -982,6 +982,48 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
                      stream, nullptr, 0, 0, kv_sB, kv_sT);
 }
 
+size_t spark_prefill_q8_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg) {
+  if (check_cfg(cfg) != SPARK_OK || B <= 0 || B > 65535 || cap <= 0 || cap > SPARK_MAX_POSITION) return 0;
+  if (cfg->kind == SPARK_SLIDING && cap != SPARK_WINDOW) return 0;
+  return 2ull * B * SPARK_N_KV_HEADS * (size_t)cap * SPARK_HEAD_DIM * 2;
+}
+
+int spark_attn_prefill_q8(void* out, const void* q, const void* k, const void* v, const void* gate,
+                          const void* k_codes, const void* k_scales, const void* v_codes, const void* v_scales,
+                          int cap, int B, int T, long long q_sB, long long q_sT, long long kv_sB, long long kv_sT,
+                          const int* pos0, const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
+                          unsigned flags, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!k_codes || !k_scales || !v_codes || !v_scales || !workspace || !pos0)
+    return fail(SPARK_ERR_INVALID_ARG, "null pointer");
+  if (flags & ~(SPARK_ROPE_FUSED | SPARK_APPEND_FUSED)) return fail(SPARK_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (B <= 0 || B > 65535 || T <= 0 || T > SPARK_MAX_POSITION)
+    return fail(SPARK_ERR_INVALID_ARG, "bad shape B=%d T=%d", B, T);
+  const size_t need = spark_prefill_q8_workspace_bytes(B, cap, cfg);
+  if (need == 0) return fail(SPARK_ERR_INVALID_ARG, "bad cap %d for this layer", cap);
+  if (ws_bytes < need) return fail(SPARK_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+  if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(k_scales) || !aligned16(v_scales) ||
+      !aligned16(workspace))
+    return fail(SPARK_ERR_INVALID_ARG, "codes, scales and workspace must be 16-byte aligned");
+  int dev;
+  if ((rc = device_ready(&dev))) return rc;
+  __nv_bfloat16* hk = (__nv_bfloat16*)workspace;
+  __nv_bfloat16* hv = hk + need / 4;
+  spark::q8_history_kernel<<<dim3((unsigned)((cap + 3) / 4), SPARK_N_KV_HEADS, (unsigned)B), 256, 0,
+                             (cudaStream_t)stream>>>((const uint8_t*)k_codes, (const __half*)k_scales,
+                                                     (const uint8_t*)v_codes, (const __half*)v_scales, cap, pos0,
+                                                     hk, hv);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "q8_history_kernel launch");
+  rc = spark_attn_prefill(out, q, k, v, gate, hk, hv, cap, B, T, q_sB, q_sT, kv_sB, kv_sT, pos0, cfg,
+                          flags & ~SPARK_APPEND_FUSED, stream);
+  if (rc || !(flags & SPARK_APPEND_FUSED)) return rc;
+  // the chunk's k (rotated) and v, quantised into the 8-bit cache after the attention
+  return append_impl(dense_view((void*)k_codes, (void*)v_codes, (void*)k_scales, (void*)v_scales, cap), k, v, B, T,
+                     pos0, cfg, 0, stream, nullptr, 0, 0, kv_sB, kv_sT);
+}
+
 int spark_rope_apply_varlen(void* x, int H, const int* cu_seqlens, int max_seqlen, const int* pos0, int B,
                             const spark_layer_cfg* cfg, void* stream) {
   int rc = check_cfg(cfg);

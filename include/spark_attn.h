@@ -289,6 +289,32 @@ int spark_attn_decode_q8(void* out, const void* q, const void* gate, const void*
                          int B, const int* pos, const spark_layer_cfg* cfg, void* workspace,
                          size_t ws_bytes, unsigned flags, void* stream);
 
+/* Workspace bytes spark_attn_prefill_q8 needs: the history as bf16, K and V
+ * [B][4][cap][256] each (cap = 512 on sliding layers).  0 on bad arguments. */
+size_t spark_prefill_q8_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg);
+
+/* spark_attn_prefill over a q8 cache history ("Sharp-Spark-X2.5-4B-GGUF" page
+ * §四 runs the model with the K/V cache as q8_0, and §三 measures prefill at
+ * 131072 tokens of context over it).  Same arguments, positions, visibility,
+ * rotation and output as spark_attn_prefill, with the history's caches given
+ * as codes + scales (the q8_0 layout above, cap rows) and a workspace.  The
+ * history keys and values are code * scale rounded to bf16; the chunk's own
+ * keys and values are the bf16 k/v passed in, as in spark_attn_prefill.
+ * The call first writes the history rows each sequence reads (full layers:
+ * rows [0, pos0[b]); sliding layers: the 512-row ring) into the workspace as
+ * bf16, then runs the bf16 prefill over it, both on `stream`.
+ *   workspace: caller-owned device memory of at least
+ *   spark_prefill_q8_workspace_bytes(B, cap, cfg) bytes, 16-byte aligned,
+ *   scratch only (its contents are undefined after the call, also after an
+ *   argument error); calls sharing it must not overlap on the device.
+ * With SPARK_APPEND_FUSED the chunk's k (as passed: rotated) and v are then
+ * quantised into the 8-bit cache, as spark_kv_append_q8 would. */
+int spark_attn_prefill_q8(void* out, const void* q, const void* k, const void* v, const void* gate,
+                          const void* k_codes, const void* k_scales, const void* v_codes, const void* v_scales,
+                          int cap, int B, int T, long long q_sB, long long q_sT, long long kv_sB, long long kv_sT,
+                          const int* pos0, const spark_layer_cfg* cfg, void* workspace, size_t ws_bytes,
+                          unsigned flags, void* stream);
+
 /* ---- Paged KV caches (the serving form; "Spark-X2.6-4B-Base" hybrid-attention
  * page §配套效率设计 serves the model through vLLM with prefix caching, whose
  * KV lives in fixed-size pages).  One layer's K and V live in pools of pages;
@@ -354,7 +380,8 @@ int spark_kv_append_varlen(const spark_paged_kv* kv, const void* k, const void* 
  * itself and to its history in the paged pool `history` (NULL: no history),
  * which must hold positions [0, pos0[b]) for full layers and the ring of the
  * last 512 for sliding layers (bf16 pools only; an 8-bit pool is
- * SPARK_ERR_UNSUPPORTED here).  History tiles stay page-aligned, so the rows
+ * SPARK_ERR_UNSUPPORTED here: a dense 8-bit history goes through
+ * spark_attn_prefill_q8).  History tiles stay page-aligned, so the rows
  * of a sequence's last history page past pos0[b] must hold finite values (a
  * zero-initialised pool, or rows an earlier append wrote). */
 int spark_attn_prefill_varlen(void* out, const void* q, const void* k, const void* v, const void* gate,

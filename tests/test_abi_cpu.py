@@ -19,6 +19,14 @@ def _declared():
     return sorted(set(names))
 
 
+def _no_gpu():
+    """The calls below pass placeholder pointers that only host-side checks may see: with a GPU
+    present, a call that passes its checks would launch a kernel on them, so those tests skip."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("placeholder pointers: host-side checks are tested only where no GPU is present")
+
+
 @pytest.fixture(scope="module")
 def lib():
     import __graft_entry__
@@ -71,6 +79,7 @@ def test_calls_fail_loudly_without_a_device(lib):
 def test_host_argument_checks_run_before_the_device(lib):
     """Host-side validation of the C entry points returns its status before any device call, so it
     is checked here without a GPU (fake, never dereferenced pointers)."""
+    _no_gpu()
     import full_gqa_attention_spark2_b200 as sa
     L = sa._lib()
     full = sa.spark_layer_cfg_for_kind(sa.SPARK_FULL)
@@ -95,12 +104,27 @@ def test_host_argument_checks_run_before_the_device(lib):
     assert L.spark_attn_prefill(*args, sa.SPARK_APPEND_FUSED, None) == -1
     assert L.spark_attn_prefill(*args, 0x80, None) == -1
     assert "SPARK_APPEND_FUSED" in sa.spark_last_error() or "flags" in sa.spark_last_error()
+    # prefill over an 8-bit history: workspace size, flags, pointers and cap before the device
+    ws_need = 2 * 4 * 1000 * 256 * 2
+    assert L.spark_prefill_q8_workspace_bytes(1, 1000, ctypes.byref(full)) == ws_need
+    assert L.spark_prefill_q8_workspace_bytes(2, 512, ctypes.byref(sliding)) == 2 * 2 * 4 * 512 * 256 * 2
+    assert L.spark_prefill_q8_workspace_bytes(1, 600, ctypes.byref(sliding)) == 0
+    assert L.spark_prefill_q8_workspace_bytes(0, 512, ctypes.byref(sliding)) == 0
+    q8 = (fake, fake, fake, fake, fake, fake, fake, fake, fake)
+    tail = (1, 128, 0, 0, 0, 0, fake, ctypes.byref(full), fake)
+    assert L.spark_attn_prefill_q8(*q8, 1000, *tail, ws_need - 16, 0, None) == -1
+    assert "workspace" in sa.spark_last_error()
+    assert L.spark_attn_prefill_q8(*q8, 1000, *tail, ws_need, 0x80, None) == -1
+    assert L.spark_attn_prefill_q8(*q8[:5], None, *q8[6:], 1000, *tail, ws_need, 0, None) == -1
+    assert L.spark_attn_prefill_q8(*q8, 600, 1, 128, 0, 0, 0, 0, fake, ctypes.byref(sliding), fake, 1 << 30, 0,
+                                   None) == -1
 
 
 def test_token_strides_are_checked_on_the_host(lib):
     """Element strides of the token tensors: 0, 0 is the dense layout; a view of a fused projection
     output [B, T, 24, 256] is accepted; rows that are not 16-byte multiples, heads that do not fit a
     token, or sequences that overlap are refused before any device call."""
+    _no_gpu()
     import full_gqa_attention_spark2_b200 as sa
     L = sa._lib()
     full = ctypes.byref(sa.spark_layer_cfg_for_kind(sa.SPARK_FULL))

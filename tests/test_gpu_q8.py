@@ -233,3 +233,96 @@ def test_decode_q8_large_values():
     assert_close(got / 512.0, ref / 512.0, "q8 decode full, large V")
     got, ref = _decode_q8_case(O.SLIDING, 2, [700, 700], sigma_q=float(1 << 22))
     assert_close(got, ref, "q8 decode sliding, huge q")
+
+
+# ----------------------------------------------------------------- prefill ----
+
+def _prefill_q8_case(kind, T, pos0_list, seed=43, layer=0, cap_extra=9, flags=None, sigma_v=1.0):
+    """A chunk of T tokens per sequence over an 8-bit history.  The history (keys taken as rotated)
+    is quantised on the host by the oracle's quantiser and uploaded, so the comparison covers the
+    prefill alone; cache rows that hold no history position, and the whole workspace, start as
+    garbage (codes 255, NaN scales, NaN bf16).  Returns (out, reference, device tensors)."""
+    sliding = kind == O.SLIDING
+    B = len(pos0_list)
+    cap = 512 if sliding else max(pos0_list) + T + cap_extra
+    cfg = sa.spark_layer_cfg_for_kind(kind)
+    codes = {n: np.full((B, 4, cap, 256), 255, np.uint8) for n in "kv"}
+    scales = {n: np.full((B, 4, cap, 8), np.nan, np.float16) for n in "kv"}
+    hist = {}
+    for b, p0 in enumerate(pos0_list):
+        hp = np.arange(max(0, p0 - 512) if sliding else 0, p0)
+        rows = hp % 512 if sliding else hp
+        for n, role, sig in (("k", synth.ROLE_K, 1.0), ("v", synth.ROLE_V, sigma_v)):
+            x = np.stack([f64(synth.head_slice(seed, tid(layer, role), b, g, 4, 256, hp, sig)) for g in range(4)], 1)
+            c, s = O.quantize_q8(x.astype(np.float32))                 # [n, 4, 256], [n, 4, 8]
+            codes[n][b, :, rows] = c                               # (advanced index first: [n, 4, 256])
+            scales[n][b, :, rows] = s
+            hist[b, n] = O.dequantize_q8(c, s)
+        hist[b, "pos"] = hp
+    pos = np.array([[p + t for t in range(T)] for p in pos0_list])
+    qb = synth.token_tensor(seed, tid(layer, synth.ROLE_Q), B, 16, 256, pos)
+    kb = synth.token_tensor(seed, tid(layer, synth.ROLE_K), B, 4, 256, pos)
+    vb = synth.token_tensor(seed, tid(layer, synth.ROLE_V), B, 4, 256, pos, sigma_v)
+    gb = synth.token_tensor(seed, tid(layer, synth.ROLE_GATE), B, 16, 1, pos)
+    p0 = _pos_tensor(pos0_list)
+    q, k, v, g = to_dev(qb), to_dev(kb), to_dev(vb), to_dev(gb)
+    sa.spark_rope_apply(k, p0, cfg)
+    dev = {n + "c": torch.from_numpy(codes[n]).cuda() for n in "kv"}
+    dev.update({n + "s": torch.from_numpy(scales[n]).cuda() for n in "kv"})
+    ws = torch.full((sa.spark_prefill_q8_workspace_bytes(B, cap, cfg),), 255, dtype=torch.uint8, device="cuda")
+    out = torch.full((B, T, 16, 256), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sa.spark_attn_prefill_q8(out, q, k, v, g, dev["kc"], dev["ks"], dev["vc"], dev["vs"], p0, cfg, ws,
+                             flags=sa.SPARK_ROPE_FUSED if flags is None else flags)
+    sa.spark_check()
+    refs = [O.layer_prefill(f64(qb[b]), f64(kb[b]), f64(vb[b]), f64(gb[b]), pos[b], kind,
+                            hist.get((b, "k")), hist.get((b, "v")), hist[b, "pos"]) for b in range(B)]
+    return dev_to_f64(out), np.stack(refs), dict(q=q, k=k, v=v, g=g, p0=p0, cfg=cfg, ws=ws, cap=cap, **dev)
+
+
+@pytest.mark.parametrize("kind,T,pos0_list", [(O.SLIDING, 300, [0, 700, 1500]), (O.SLIDING, 129, [511, 512, 513]),
+                                              (O.SLIDING, 1, [4097]), (O.FULL, 200, [0, 333, 1000]),
+                                              (O.FULL, 129, [128, 1]), (O.FULL, 128, [4097])])
+def test_prefill_q8_history(kind, T, pos0_list):
+    """Every element against the oracle's attention over its own dequantised history, per-sequence
+    positions, window edges and ring wraps, NaN in the workspace and garbage past the history."""
+    got, ref, _ = _prefill_q8_case(kind, T, pos0_list)
+    assert_close(got, ref, f"q8-history prefill {KIND_NAME[kind]} T={T} pos0={pos0_list}")
+
+
+def test_prefill_q8_history_large_values():
+    """V of scale 256 through fp16 scales and bf16 history rows."""
+    got, ref, _ = _prefill_q8_case(O.FULL, 160, [900, 77], sigma_v=256.0)
+    assert_close(got / 256.0, ref / 256.0, "q8-history prefill full, large V")
+
+
+@pytest.mark.parametrize("kind,T,pos0_list", [(O.SLIDING, 300, [700, 0]), (O.FULL, 200, [333, 0])])
+def test_prefill_q8_append_fused(kind, T, pos0_list):
+    """SPARK_APPEND_FUSED: the same output, and the 8-bit cache afterwards bit-identical to
+    spark_kv_append_q8 of the chunk after the call (a sliding ring's history rows are overwritten
+    only after the attention has read them)."""
+    got, _, d = _prefill_q8_case(kind, T, pos0_list)
+    kc, ks, vc, vs = (d[n].clone() for n in ("kc", "ks", "vc", "vs"))
+    out2 = torch.empty(len(pos0_list), T, 16, 256, dtype=torch.bfloat16, device="cuda")
+    sa.spark_attn_prefill_q8(out2, d["q"], d["k"], d["v"], d["g"], kc, ks, vc, vs, d["p0"], d["cfg"], d["ws"],
+                             flags=sa.SPARK_ROPE_FUSED | sa.SPARK_APPEND_FUSED)
+    sa.spark_kv_append_q8(d["kc"], d["ks"], d["vc"], d["vs"], d["k"], d["v"], d["p0"], d["cfg"])
+    sa.spark_check()
+    assert np.array_equal(dev_to_f64(out2), got)
+    assert torch.equal(kc, d["kc"]) and torch.equal(vc, d["vc"])
+    assert torch.equal(ks.view(torch.int16), d["ks"].view(torch.int16))
+    assert torch.equal(vs.view(torch.int16), d["vs"].view(torch.int16))
+
+
+def test_prefill_q8_host_checks():
+    cfg = sa.spark_layer_cfg_for_kind(O.SLIDING)
+    full = sa.spark_layer_cfg_for_kind(O.FULL)
+    assert sa.spark_prefill_q8_workspace_bytes(2, 512, cfg) == 2 * 2 * 4 * 512 * 256 * 2
+    assert sa.spark_prefill_q8_workspace_bytes(2, 600, cfg) == 0
+    assert sa.spark_prefill_q8_workspace_bytes(1, 1000, full) == 2 * 4 * 1000 * 256 * 2
+    _, _, d = _prefill_q8_case(O.FULL, 64, [100])
+    out = torch.empty(1, 64, 16, 256, dtype=torch.bfloat16, device="cuda")
+    args = (out, d["q"], d["k"], d["v"], d["g"], d["kc"], d["ks"], d["vc"], d["vs"], d["p0"], d["cfg"])
+    with pytest.raises(sa.SparkError):
+        sa.spark_attn_prefill_q8(*args, d["ws"][:-16])              # workspace too small
+    with pytest.raises(sa.SparkError):
+        sa.spark_attn_prefill_q8(*args, d["ws"], flags=0x80)
