@@ -4,6 +4,8 @@
   launch configuration bench.py times: all 4 x 8192 x 16 x 256 outputs of both layers.
 - Decode B=64 with 32768 cached tokens (seed 3), layers 0 (sliding) and 3 (full), one step through
   the fused call bench.py times: all 64 x 16 x 256 outputs of both layers.
+- Long-context decode, B=16 at 131072 and B=1 at 2^20 (seed 5), the same two layers and call: all
+  outputs.
 
 The oracle's inputs are the seeded generator's values.  The device generator filled the tensors;
 they are read back before any library call touches them (and, for the decode caches, only at rows
@@ -123,5 +125,54 @@ def test_decode_b64_ctx32768_every_sequence():
                 vals = np.concatenate([vh[g], vn_all[b, g][None]])
                 ref = O.attention_group(qr[None, hs], keys, vals, g_all[b][None, hs], np.array([p]), kpos, kind)[0]
                 assert_close(got[b, hs], ref, f"decode B=64 p={p} layer={layer} b={b} group={g}")
+    del layers, wsf
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,p", [(16, 131071), (1, (1 << 20) - 1)])
+def test_long_decode_every_output(B, p):
+    """Long-context decode with the new token at the end of the context (131072 at B=16, 2^20 at
+    B=1; seed 5), one step of a sliding and a full layer through the fused call bench.py times:
+    all B x 16 x 256 outputs of both layers, one (sequence, KV head) at a time."""
+    dev = torch.device("cuda")
+    seed = 5
+    layers = bench.decode_layers(torch, sa, synth, dev, B, p, (0, 3), seed=seed)
+    pos = torch.full((B,), p, dtype=torch.int32, device=dev)
+    wsf = torch.zeros(max(sa.spark_decode_fused_workspace_bytes(B, L["cap"], L["cfg"]) for L in layers),
+                      dtype=torch.uint8, device=dev)
+    bench.decode_fused_step(sa, layers, pos, wsf)
+    sa.spark_check()
+    for L in layers:
+        kind, layer = L["kind"], L["layer"]
+        sliding = kind == O.SLIDING
+        hist = np.arange(max(0, p - (O.WINDOW - 1)) if sliding else 0, p)
+        rows = hist % O.WINDOW if sliding else hist                # cache rows the step did not write
+        got = _host_f64(L["out"])
+        pnew = np.full((B, 1), p)
+        q_all = f64(synth.token_tensor(seed, tid(layer, synth.ROLE_Q), B, 16, 256, pnew))[:, 0]
+        g_all = f64(synth.token_tensor(seed, tid(layer, synth.ROLE_GATE), B, 16, 1, pnew))[:, 0]
+        kn_all = f64(synth.token_tensor(seed, tid(layer, synth.ROLE_K), B, 4, 256, pnew))[:, 0]
+        vn_all = f64(synth.token_tensor(seed, tid(layer, synth.ROLE_V), B, 4, 256, pnew))[:, 0]
+        sample = np.array([0, len(hist) // 3, len(hist) // 2, len(hist) - 1])
+        for b, g in ((0, 0), (B - 1, 3)):
+            host = synth.head_slice(seed, tid(layer, synth.ROLE_K), b, g, 4, 256, hist[sample])
+            assert np.array_equal(_bits(L["kc"][b, g][torch.as_tensor(rows[sample], device=dev)]), host)
+        kpos = np.concatenate([hist, [p]])
+        rows_d = None if not sliding else torch.as_tensor(rows, device=dev)
+        for b in range(B):
+            qr = O.rope(q_all[b][None], np.array([p]), kind)[0]
+            knr = O.rope(kn_all[b][None], np.array([p]), kind)[0]
+            for g in range(4):
+                if sliding:
+                    kh, vh = _host_f64(L["kc"][b, g][rows_d]), _host_f64(L["vc"][b, g][rows_d])
+                else:
+                    kh, vh = _host_f64(L["kc"][b, g, :p]), _host_f64(L["vc"][b, g, :p])
+                hs = slice(4 * g, 4 * g + 4)
+                keys = np.concatenate([kh, knr[g][None]])
+                vals = np.concatenate([vh, vn_all[b, g][None]])
+                del kh, vh
+                ref = O.attention_group(qr[None, hs], keys, vals, g_all[b][None, hs], np.array([p]), kpos, kind)[0]
+                assert_close(got[b, hs], ref, f"long decode B={B} p={p} layer={layer} b={b} group={g}")
+                del keys, vals
     del layers, wsf
     torch.cuda.empty_cache()
