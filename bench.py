@@ -19,6 +19,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -110,11 +111,17 @@ def hbm_roofline(kernel: str, achieved_gbs: float, peaks, traffic=None):
 
 
 def kernel_source_sha():
+    """Hash of the CUDA sources' code (comments and blank space removed), which keys the ncu traffic
+    figures in profiles/traffic.json: they hold until the code changes."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "full_gqa_attention_spark2_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(f.encode())
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -518,8 +518,8 @@ __global__ void __launch_bounds__(kQ8Threads, 1)
 // The history a prefill chunk reads from an 8-bit cache, as bf16 rows in the bf16 cache's layout
 // ([B][4][cap][256]): rows [0, min(pos0[b], cap)) of sequence b (a full layer's positions; a
 // sliding ring's rows, cap 512, which then hold every history position the chunk can see).  Rows
-// past them, and every row of a sequence with a bad position, are left as they are (the prefill
-// never reads them; it flags a bad position itself).  Each value is code * scale, exact in fp32
+// past them, and every row of a sequence with a negative position, are left as they are (the
+// prefill never reads them; it flags a bad position itself).  Each value is code * scale, exact in fp32
 // (an 8-bit code times an 11-bit significand), then rounded once to bf16.  One warp per (row,
 // tensor): lane i takes codes 8i .. 8i+7 of block i/4 (256 bytes read, 512 written per warp).
 // Grid (ceil(cap / 4), 4 KV heads, B), 256 threads: warp w takes row 4 blockIdx.x + w/2, K (even
