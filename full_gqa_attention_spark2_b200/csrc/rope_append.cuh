@@ -59,24 +59,19 @@ __device__ __forceinline__ void rope_angle(int pos, double f, float& c, float& s
   sincosf((float)r, &s, &c);
 }
 
-// x [B][T][H][256] (dense, cu == nullptr) or packed [total][H][256] with
-// sequence b at rows cu[b] .. cu[b+1]-1 (ragged), in place.  One thread per
-// (token, two consecutive pairs); a block walks kRopeIters groups of tokens,
-// so that its frequency table serves many tokens.  Dense: a 1-D grid over the
-// B*T tokens.  Ragged: grid.y = sequence, grid.x over its tokens (T = the
-// longest).
+// 16-head tensors (q): x [B][T][16][256] (dense, cu == nullptr) or packed [total][16][256] with
+// sequence b at rows cu[b] .. cu[b+1]-1 (ragged), in place.  One thread per (token, two
+// consecutive pairs), all sixteen heads' pairs loaded before any is stored, so sixteen loads are
+// in flight together (3x faster on full layers than one head at a time; faster than the run kernel
+// below, whose angle reuse matters less where sixteen heads share each angle).  A block walks
+// kRopeIters groups of tokens, so that its frequency table serves many tokens.  Dense: a 1-D grid
+// over the B*T tokens.  Ragged: grid.y = sequence, grid.x over its tokens (T = the longest).
 constexpr int kRopeIters = 8;
 
-// kAllHeads (q, 16 heads): all heads' pairs are loaded before any is stored, so sixteen loads
-// are in flight together (3x faster on full layers than one head at a time).  k's four heads go
-// one at a time: there the separate instantiation keeps fewer registers and more warps resident,
-// which measured faster.
-// Token rows: dense batches put token t of sequence b at element b * sB + t * sT; packed rows
-// (ragged) put row n at n * sT.  Within a token the H heads are contiguous rows of 256.
-template <bool kAllHeads>
-__global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x, int B, int T,
-                                                   int H, long long sB, long long sT, const int* __restrict__ pos0,
-                                                   const RopeFreq rf, int rot, const int* __restrict__ cu) {
+// Token rows as for rope_kernel below.
+__global__ void __launch_bounds__(128) rope16_kernel(__nv_bfloat16* __restrict__ x, int B, int T,
+                                                     long long sB, long long sT, const int* __restrict__ pos0,
+                                                     const RopeFreq rf, int rot, const int* __restrict__ cu) {
   __shared__ double freq[128];
   const int half = rot >> 1;
   for (int i = threadIdx.x; i < half; i += blockDim.x) freq[i] = rf.f[i];
@@ -113,7 +108,7 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
     rope_angle(pos, freq[2 * j], c0, s0);
     rope_angle(pos, freq[2 * j + 1], c1, s1);
     __nv_bfloat16* row = x + (cu == nullptr ? (long long)b * sB + (long long)t * sT : n * sT);
-    if constexpr (kAllHeads) {
+    {
       uint32_t lo[16], hi[16];
 #pragma unroll
       for (int h = 0; h < 16; ++h) {
@@ -128,15 +123,88 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
         *reinterpret_cast<uint32_t*>(row + h * kHeadDim + half + 2 * j) =
             pack_bf16(rope_hi(l0, h0, c0, s0), rope_hi(l1, h1, c1, s1));
       }
-    } else {
-      for (int h = 0; h < H; ++h) {
-        uint32_t* lo_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + 2 * j);
-        uint32_t* hi_p = reinterpret_cast<uint32_t*>(row + h * kHeadDim + half + 2 * j);
-        uint32_t lo = *lo_p, hi = *hi_p;
-        float l0 = bf16_lo(lo), l1 = bf16_hi(lo), h0 = bf16_lo(hi), h1 = bf16_hi(hi);
-        *lo_p = pack_bf16(rope_lo(l0, h0, c0, s0), rope_lo(l1, h1, c1, s1));
-        *hi_p = pack_bf16(rope_hi(l0, h0, c0, s0), rope_hi(l1, h1, c1, s1));
+    }
+  }
+}
+
+// One 32-bit word of a low chunk and its partner in the high chunk: two pairs rotated by the angles
+// (c0, s0) and (c1, s1), each product rounded before the FMA that adds it (as in the append).
+__device__ __forceinline__ void rope_word(uint32_t& l, uint32_t& u, float c0, float s0, float c1, float s1) {
+  const float a0 = bf16_lo(l), a1 = bf16_hi(l), b0 = bf16_lo(u), b1 = bf16_hi(u);
+  l = pack_bf16(rope_lo(a0, b0, c0, s0), rope_lo(a1, b1, c1, s1));
+  u = pack_bf16(rope_hi(a0, b0, c0, s0), rope_hi(a1, b1, c1, s1));
+}
+
+// 4-head tensors (k): x [B][T][4][256] (dense, cu == nullptr) or packed [total][4][256] with
+// sequence b at rows cu[b] .. cu[b+1]-1 (ragged), in place (H: a multiple of 4).  A thread takes one chunk of eight pairs (dims 8 c .. 8 c + 7 and
+// their partners rot/2 later) in every head of kRopeRun consecutive tokens of one sequence: 16-byte
+// accesses, four heads' loads in flight together.  Its first token's angles are exact (fp64
+// product and reduction); each later token's advance by one position's rotation, so one angle
+// serves H * kRopeRun rotations.  Dense: a 1-D grid over every sequence's runs of tokens.  Ragged:
+// grid.y = sequence, grid.x over its runs (T = the longest).
+// Token rows: dense batches put token t of sequence b at element b * sB + t * sT; packed rows
+// (ragged) put row n at n * sT.  Within a token the H heads are contiguous rows of 256.
+constexpr int kRopeRun = 4;
+
+__global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x, int B, int T, int H, long long sB,
+                                                   long long sT, const int* __restrict__ pos0, const RopeFreq rf,
+                                                   int rot, const int* __restrict__ cu) {
+  const int half = rot >> 1;
+  const int n_ch = half >> 3;                      // chunks per head: 16 (sliding) or 4 (full)
+  const int ch = threadIdx.x % n_ch;
+  const long long run = (long long)blockIdx.x * (blockDim.x / n_ch) + threadIdx.x / n_ch;
+  int b, t0, T_b;
+  if (cu == nullptr) {
+    const int runs_per_seq = (T + kRopeRun - 1) / kRopeRun;
+    if (run >= (long long)B * runs_per_seq) return;
+    b = (int)(run / runs_per_seq);
+    t0 = (int)(run % runs_per_seq) * kRopeRun;
+    T_b = T;
+  } else {
+    b = blockIdx.y;
+    T_b = cu[b + 1] - cu[b];
+    if (run * kRopeRun >= T_b) return;
+    t0 = (int)run * kRopeRun;
+  }
+  const int p0 = pos0[b];
+  if (p0 < 0 || p0 > kMaxPos - T_b) {
+    if (t0 == 0 && ch == 0) raise_error(kErrPosition, 0x100u | (unsigned)b);
+    return;
+  }
+  float c[8], s[8], cs[8], ss[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const double f = rf.f[8 * ch + e];
+    rope_angle(p0 + t0, f, c[e], s[e]);
+    sincosf((float)f, &ss[e], &cs[e]);             // one position: 0 < f <= 1 needs no reduction
+  }
+  for (int i = 0; i < kRopeRun; ++i) {
+    const int t = t0 + i;
+    if (t >= T_b) break;
+    __nv_bfloat16* row = x + (cu == nullptr ? (long long)b * sB + (long long)t * sT : ((long long)cu[b] + t) * sT);
+    for (int h0 = 0; h0 < H; h0 += 4) {
+      uint4 lo[4], hi[4];
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) {
+        lo[hh] = *reinterpret_cast<const uint4*>(row + (h0 + hh) * kHeadDim + 8 * ch);
+        hi[hh] = *reinterpret_cast<const uint4*>(row + (h0 + hh) * kHeadDim + half + 8 * ch);
       }
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) {
+        rope_word(lo[hh].x, hi[hh].x, c[0], s[0], c[1], s[1]);
+        rope_word(lo[hh].y, hi[hh].y, c[2], s[2], c[3], s[3]);
+        rope_word(lo[hh].z, hi[hh].z, c[4], s[4], c[5], s[5]);
+        rope_word(lo[hh].w, hi[hh].w, c[6], s[6], c[7], s[7]);
+        *reinterpret_cast<uint4*>(row + (h0 + hh) * kHeadDim + 8 * ch) = lo[hh];
+        *reinterpret_cast<uint4*>(row + (h0 + hh) * kHeadDim + half + 8 * ch) = hi[hh];
+      }
+    }
+    // the next position: (c + i s)(cs + i ss)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float cn = c[e] * cs[e] - s[e] * ss[e];
+      s[e] = s[e] * cs[e] + c[e] * ss[e];
+      c[e] = cn;
     }
   }
 }

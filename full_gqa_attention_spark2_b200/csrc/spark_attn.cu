@@ -768,17 +768,22 @@ int spark_rope_apply(void* x, int B, int T, int H, long long sB, long long sT, c
   if (!aligned16(x)) return fail(SPARK_ERR_INVALID_ARG, "x must be 16-byte aligned");
   int dev;
   if ((rc = device_ready(&dev))) return rc;
-  const int per_tok = cfg->rot_dim / 4;
-  const int tok_per_block = 128 / per_tok * spark::kRopeIters;
-  const long long n = (long long)B * T;
-  const long long grid = (n + tok_per_block - 1) / tok_per_block;
-  if (grid > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "too many tokens");
-  if (H == 16)
-    spark::rope_kernel<true><<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>(
-        (__nv_bfloat16*)x, B, T, H, sB, sT, pos0, rope_freq(cfg), cfg->rot_dim, nullptr);
-  else
-    spark::rope_kernel<false><<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>(
-        (__nv_bfloat16*)x, B, T, H, sB, sT, pos0, rope_freq(cfg), cfg->rot_dim, nullptr);
+  if (H == 16) {
+    // a thread per (token, two pairs), kRopeIters tokens per thread
+    const int tok_per_block = 128 / (cfg->rot_dim / 4) * spark::kRopeIters;
+    const long long grid = ((long long)B * T + tok_per_block - 1) / tok_per_block;
+    if (grid > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "too many tokens");
+    spark::rope16_kernel<<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>((__nv_bfloat16*)x, B, T, sB, sT, pos0,
+                                                                           rope_freq(cfg), cfg->rot_dim, nullptr);
+  } else {
+    // a thread per (eight-pair chunk, run of kRopeRun tokens); 128 / chunks runs per block
+    const int runs_per_block = 128 / (cfg->rot_dim / 16);
+    const long long runs = (long long)B * ((T + spark::kRopeRun - 1) / spark::kRopeRun);
+    const long long grid = (runs + runs_per_block - 1) / runs_per_block;
+    if (grid > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "too many tokens");
+    spark::rope_kernel<<<(unsigned)grid, 128, 0, (cudaStream_t)stream>>>((__nv_bfloat16*)x, B, T, H, sB, sT, pos0,
+                                                                         rope_freq(cfg), cfg->rot_dim, nullptr);
+  }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "rope_kernel launch");
 }
@@ -1034,16 +1039,20 @@ int spark_rope_apply_varlen(void* x, int H, const int* cu_seqlens, int max_seqle
   if (!aligned16(x)) return fail(SPARK_ERR_INVALID_ARG, "x must be 16-byte aligned");
   int dev;
   if ((rc = device_ready(&dev))) return rc;
-  const int tok_per_block = 128 / (cfg->rot_dim / 4) * spark::kRopeIters;
-  dim3 grid((max_seqlen + tok_per_block - 1) / tok_per_block, B);
-  if (H == 16)
-    spark::rope_kernel<true><<<grid, 128, 0, (cudaStream_t)stream>>>(
-        (__nv_bfloat16*)x, B, max_seqlen, H, 0, (long long)H * SPARK_HEAD_DIM, pos0, rope_freq(cfg), cfg->rot_dim,
-        cu_seqlens);
-  else
-    spark::rope_kernel<false><<<grid, 128, 0, (cudaStream_t)stream>>>(
-        (__nv_bfloat16*)x, B, max_seqlen, H, 0, (long long)H * SPARK_HEAD_DIM, pos0, rope_freq(cfg), cfg->rot_dim,
-        cu_seqlens);
+  if (H == 16) {
+    const int tok_per_block = 128 / (cfg->rot_dim / 4) * spark::kRopeIters;
+    dim3 grid((max_seqlen + tok_per_block - 1) / tok_per_block, B);
+    spark::rope16_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>((__nv_bfloat16*)x, B, max_seqlen, 0,
+                                                                 (long long)H * SPARK_HEAD_DIM, pos0, rope_freq(cfg),
+                                                                 cfg->rot_dim, cu_seqlens);
+  } else {
+    const int runs_per_block = 128 / (cfg->rot_dim / 16);
+    const int runs = (max_seqlen + spark::kRopeRun - 1) / spark::kRopeRun;
+    dim3 grid((runs + runs_per_block - 1) / runs_per_block, B);
+    spark::rope_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>((__nv_bfloat16*)x, B, max_seqlen, H, 0,
+                                                               (long long)H * SPARK_HEAD_DIM, pos0, rope_freq(cfg),
+                                                               cfg->rot_dim, cu_seqlens);
+  }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SPARK_OK : cuda_fail(e, "rope_kernel launch");
 }
