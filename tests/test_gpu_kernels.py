@@ -377,3 +377,43 @@ def test_prefill_ignores_nan_past_the_history(kind, T, pos0_list):
     got, ref = _prefill_case(kind, len(pos0_list), T, pos0_list, poison=True, cap_extra=200)
     assert np.isfinite(got).all()
     assert_close(got, ref, f"prefill {KIND_NAME[kind]} T={T} pos0={pos0_list}, NaN past the history")
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_prefill_step_in_a_cuda_graph(kind):
+    """The prefill step (RoPE on k, the prefill with q rotated at load, the append) captured in a CUDA
+    graph and replayed gives the eager step's output and cache bit for bit (the persistent kernel's
+    cluster launch control and tensor maps inside a graph)."""
+    B, T, seed, layer = 1, 1024, 0, 0
+    cfg = _cfg(kind)
+    pos = np.broadcast_to(np.arange(T), (B, T))
+    qb = synth.token_tensor(seed, tid(layer, synth.ROLE_Q), B, 16, 256, pos)
+    kb = synth.token_tensor(seed, tid(layer, synth.ROLE_K), B, 4, 256, pos)
+    vb = synth.token_tensor(seed, tid(layer, synth.ROLE_V), B, 4, 256, pos)
+    gb = synth.token_tensor(seed, tid(layer, synth.ROLE_GATE), B, 16, 1, pos)
+    p0 = _pos_tensor([0])
+    cap = 512 if kind == O.SLIDING else T
+    runs = []
+    for graph in (False, True):
+        q, k, v, g = to_dev(qb), to_dev(kb), to_dev(vb), to_dev(gb)
+        kc = torch.zeros(B, 4, cap, 256, dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        out = torch.empty(B, T, 16, 256, dtype=torch.bfloat16, device="cuda")
+
+        def step():
+            sa.spark_rope_apply(k, p0, cfg)
+            sa.spark_attn_prefill(out, q, k, v, g, None, None, p0, cfg, flags=sa.SPARK_ROPE_FUSED)
+            sa.spark_kv_append(kc, vc, k, v, p0, cfg)
+        if graph:
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=s):
+                step()
+            gr.replay()
+        else:
+            step()
+        sa.spark_check()
+        runs.append((out.view(torch.int16).clone(), kc.view(torch.int16).clone(), vc.view(torch.int16).clone()))
+    for a, b in zip(*runs):
+        assert torch.equal(a, b)
