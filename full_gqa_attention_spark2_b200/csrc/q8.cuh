@@ -72,7 +72,8 @@ __global__ void __launch_bounds__(128) kv_append_q8_kernel(
   const int t = sp.t_first + blockIdx.x;
   if (t >= sp.T) return;
   const int p0 = pos0[b];
-  const bool bad = p0 < 0 || p0 > kMaxPos - sp.T || (!sliding && !shard && p0 + sp.T > cap);
+  const bool bad = p0 < 0 || p0 > kMaxPos - sp.T || (!sliding && !shard && p0 + sp.T > cap) ||
+                   (cu != nullptr && sp.T > T);    // ragged: longer than max_seqlen, the launch's T
   if (bad) {
     if (blockIdx.x == 0 && tid == 0) raise_error(kErrPosition, 0x400u | (unsigned)b);
     return;

@@ -95,6 +95,10 @@ __global__ void __launch_bounds__(128) rope16_kernel(__nv_bfloat16* __restrict__
       b = blockIdx.y;
       t = (int)slot;
       T_b = cu[b + 1] - cu[b];
+      if (T_b < 0 || T_b > T) {                  // a sequence longer than max_seqlen: not rotated
+        if (t == 0 && j == 0) raise_error(kErrPosition, 0x100u | (unsigned)b);
+        return;
+      }
       if (t >= T_b) return;
       n = (long long)cu[b] + t;
     }
@@ -163,6 +167,10 @@ __global__ void __launch_bounds__(128) rope_kernel(__nv_bfloat16* __restrict__ x
   } else {
     b = blockIdx.y;
     T_b = cu[b + 1] - cu[b];
+    if (T_b < 0 || T_b > T) {                    // a sequence longer than max_seqlen: not rotated
+      if (run == 0 && ch == 0) raise_error(kErrPosition, 0x100u | (unsigned)b);
+      return;
+    }
     if (run * kRopeRun >= T_b) return;
     t0 = (int)run * kRopeRun;
   }
@@ -262,7 +270,9 @@ __global__ void __launch_bounds__(128) kv_append_kernel(
   const int t = sp.t_first + blockIdx.x;
   if (t >= sp.T) return;
   const int p0 = pos0[b];
-  const bool bad = p0 < 0 || p0 > kMaxPos - sp.T || (!sliding && !shard && p0 + sp.T > cap);
+  // (ragged: a sequence longer than max_seqlen, the launch's T, is not written either)
+  const bool bad = p0 < 0 || p0 > kMaxPos - sp.T || (!sliding && !shard && p0 + sp.T > cap) ||
+                   (cu != nullptr && sp.T > T);
   if (bad) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(kErrPosition, 0x200u | (unsigned)b);
     return;

@@ -193,3 +193,68 @@ def test_prefill_varlen_rejects_q8_history():
     with pytest.raises(sa.SparkError) as e:
         sa.spark_attn_prefill_varlen(q.clone(), q, k, k, g, _i32([0, 10]), 10, _i32([5]), kv, cfg)
     assert e.value.status == -2
+
+
+@pytest.mark.parametrize("kind", [O.SLIDING, O.FULL])
+def test_varlen_sequence_longer_than_max_seqlen_is_flagged(kind):
+    """A ragged sequence longer than max_seqlen is a device-side argument error (SPARK_ERR_DEVICE_ARG)
+    in RoPE (4 and 16 heads), the append (bf16 and 8-bit pools) and the prefill: that sequence is left
+    as it was (its rows unrotated, no cache row, no output row), the others are processed."""
+    cfg = sa.spark_layer_cfg_for_kind(kind)
+    lens, pos0, max_seqlen = [5, 40, 7], [3, 0, 900], 20
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    long_rows = slice(int(cu[1]), int(cu[2]))
+    for H in (16, 4):
+        bits, parts = _packed(5, 0, synth.ROLE_Q, lens, pos0, H, 256)
+        x = to_dev(bits)
+        before = x.clone()
+        sa.spark_rope_apply_varlen(x, _i32(cu), max_seqlen, _i32(pos0), cfg)
+        with pytest.raises(sa.SparkError) as e:
+            sa.spark_check()
+        assert e.value.status == -5
+        assert torch.equal(x[long_rows].view(torch.int16), before[long_rows].view(torch.int16))
+        got = dev_to_f64(x)
+        for b in (0, 2):
+            ref = O.rope(f64(parts[b]), pos0[b] + np.arange(lens[b]), kind)
+            assert_close(got[cu[b]:cu[b + 1]], ref, f"rope varlen H={H} b={b} beside a too-long sequence")
+    P = 64
+    max_pages = 512 // P if kind == O.SLIDING else 1024 // P
+    n_pages = 3 * max_pages
+    table = torch.arange(n_pages, dtype=torch.int32, device="cuda").view(3, max_pages)
+    kb, kparts = _packed(7, 3, synth.ROLE_K, lens, pos0, 4, 256)
+    vb, _ = _packed(7, 3, synth.ROLE_V, lens, pos0, 4, 256)
+    for q8 in (False, True):
+        dt = torch.uint8 if q8 else torch.bfloat16
+        kp = torch.zeros(n_pages, 4, P, 256, dtype=dt, device="cuda")
+        vp = torch.zeros_like(kp)
+        ks = vs = None
+        if q8:
+            ks = torch.zeros(n_pages, 4, P, 8, dtype=torch.float16, device="cuda")
+            vs = torch.zeros_like(ks)
+        kv = sa.paged_kv(kp, vp, table, ks, vs)
+        sa.spark_kv_append_varlen(kv, to_dev(kb), to_dev(vb), _i32(cu), max_seqlen, _i32(pos0), cfg)
+        with pytest.raises(sa.SparkError) as e:
+            sa.spark_check()
+        assert e.value.status == -5
+        assert not kp[max_pages:2 * max_pages].any()          # sequence 1's pages: nothing written
+        row = O.cache_slot(pos0[0], kind)                      # sequence 0's first token was written
+        if q8:
+            codes, _ = O.quantize_q8(f64(kparts[0][0]).astype(np.float32))
+            assert np.array_equal(kp[row // P, :, row % P].cpu().numpy(), codes)
+        else:
+            got = kp[row // P, :, row % P].view(torch.int16).cpu().numpy().view(np.uint16)
+            assert np.array_equal(got, kparts[0][0])
+    # the prefill (no history): the too-long sequence's output rows are not written
+    total = int(cu[-1])
+    qb, _ = _packed(9, 0, synth.ROLE_Q, lens, pos0, 16, 256)
+    gb, _ = _packed(9, 0, synth.ROLE_GATE, lens, pos0, 16, 1)
+    out = torch.full((total, 16, 256), float("nan"), dtype=torch.bfloat16, device="cuda")
+    k = to_dev(kb)
+    sa.spark_rope_apply_varlen(k, _i32(cu), max(lens), _i32(pos0), cfg)
+    sa.spark_attn_prefill_varlen(out, to_dev(qb), k, to_dev(vb), to_dev(gb), _i32(cu), max_seqlen, _i32(pos0), None,
+                                 cfg)
+    with pytest.raises(sa.SparkError) as e:
+        sa.spark_check()
+    assert e.value.status == -5
+    assert torch.isnan(out[long_rows].float()).all()
+    assert torch.isfinite(out[:int(cu[1])].float()).all() and torch.isfinite(out[int(cu[2]):].float()).all()
