@@ -884,10 +884,19 @@ int spark_attn_decode_paged(void* out, const void* q, const void* gate, const sp
   return decode_impl(out, q, gate, c, B, pos, cfg, workspace, ws_bytes, flags, stream);
 }
 
-int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, const void* gate,
-                       const void* k_cache, const void* v_cache, int cap, int B, int T, long long q_sB,
-                       long long q_sT, long long kv_sB, long long kv_sT, const int* pos0, const spark_layer_cfg* cfg,
-                       unsigned flags, void* stream) {
+// Everything a prefill needs before it launches: the arguments checked, the tensor maps encoded and
+// the kernel parameters filled.  Nothing is launched until every check has passed.
+struct PrefillPlan {
+  CUtensorMap qm, km, vm, kcm, vcm, om;
+  spark::PrefillParams P;
+  long long blocks;
+  bool has_cache, sliding;
+  long long kv_sB, kv_sT;        // k, v element strides, dense ones filled in
+};
+
+int prefill_prepare(PrefillPlan& L, void* out, const void* q, const void* k, const void* v, const void* gate,
+                    const void* k_cache, const void* v_cache, int cap, int B, int T, long long q_sB, long long q_sT,
+                    long long kv_sB, long long kv_sT, const int* pos0, const spark_layer_cfg* cfg, unsigned flags) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (!out || !q || !k || !v || !gate || !pos0) return fail(SPARK_ERR_INVALID_ARG, "null pointer");
@@ -914,33 +923,32 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   // Q, chunk K/V: [B][T][H][256] as 4-D (dim, head, token, batch) with the callers' token and
   // sequence strides; out dense; caches [B][4][cap][256] as 3-D (dim, row, batch*head).
   // 128-byte swizzled boxes of 64 dims.
-  CUtensorMap qm, km, vm, kcm, vcm, om;
   {
     const cuuint64_t dq[4] = {256, 16, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t sq[3] = {512, 2ull * (cuuint64_t)q_sT, 2ull * (cuuint64_t)q_sB};
     const cuuint64_t so[3] = {512, 512ull * 16, 512ull * 16 * T};
     const cuuint32_t bq[4] = {64, 1, (cuuint32_t)spark::kPfM, 1};
-    if ((rc = make_map(&qm, q, 4, dq, sq, bq))) return rc;
-    if ((rc = make_map(&om, out, 4, dq, so, bq))) return rc;
+    if ((rc = make_map(&L.qm, q, 4, dq, sq, bq))) return rc;
+    if ((rc = make_map(&L.om, out, 4, dq, so, bq))) return rc;
     const cuuint64_t dk[4] = {256, 4, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t sk[3] = {512, 2ull * (cuuint64_t)kv_sT, 2ull * (cuuint64_t)kv_sB};
     const cuuint32_t bk[4] = {64, 1, (cuuint32_t)(spark::kPfN / 2), 1};   // each block of the pair: 64 keys
     const cuuint32_t bv[4] = {64, 1, 32, 1};
-    if ((rc = make_map(&km, k, 4, dk, sk, bk))) return rc;
-    if ((rc = make_map(&vm, v, 4, dk, sk, bv))) return rc;
+    if ((rc = make_map(&L.km, k, 4, dk, sk, bk))) return rc;
+    if ((rc = make_map(&L.vm, v, 4, dk, sk, bv))) return rc;
     if (k_cache) {
       const cuuint64_t dc[3] = {256, (cuuint64_t)cap, (cuuint64_t)B * 4};
       const cuuint64_t sc[2] = {512, (cuuint64_t)cap * 512};
       const cuuint32_t bkc[3] = {64, (cuuint32_t)(spark::kPfN / 2), 1};
       const cuuint32_t bvc[3] = {64, 32, 1};
-      if ((rc = make_map(&kcm, k_cache, 3, dc, sc, bkc))) return rc;
-      if ((rc = make_map(&vcm, v_cache, 3, dc, sc, bvc))) return rc;
+      if ((rc = make_map(&L.kcm, k_cache, 3, dc, sc, bkc))) return rc;
+      if ((rc = make_map(&L.vcm, v_cache, 3, dc, sc, bvc))) return rc;
     } else {
-      kcm = km;
-      vcm = vm;
+      L.kcm = L.km;
+      L.vcm = L.vm;
     }
   }
-  spark::PrefillParams P;
+  spark::PrefillParams& P = L.P;
   P.out = (__nv_bfloat16*)out;
   P.gate = (const __nv_bfloat16*)gate;
   P.pos0 = pos0;
@@ -958,33 +966,53 @@ int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, c
   P.cu_seqlens = nullptr;
   P.block_table = nullptr;
   P.max_pages = P.page_shift = P.n_pages = 0;
-  const long long blocks = (long long)B * spark::kNq * P.n_qt;
-  if (blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");
+  L.blocks = (long long)B * spark::kNq * P.n_qt;
+  if (L.blocks > 0x7FFFFFFFLL) return fail(SPARK_ERR_INVALID_ARG, "grid too large");
+  L.has_cache = k_cache != nullptr;
+  L.sliding = sliding != 0;
+  L.kv_sB = kv_sB;
+  L.kv_sT = kv_sT;
+  return SPARK_OK;
+}
+
+int prefill_launch(const PrefillPlan& L, void* stream) {
   cudaError_t e;
-  if (!k_cache || sliding) {
+  if (!L.has_cache || L.sliding) {
     // the persistent kernel: one cluster per unit (two query heads x one 128-query tile); resident
     // clusters take the units of clusters that have not started (cluster launch control).  Full
     // layers with a history (units of hundreds of KV tiles) measured 5-8 % faster in prefill2.
-    if (k_cache)
-      spark::prefill3_kernel<true><<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes,
-                                     (cudaStream_t)stream>>>(qm, km, vm, kcm, vcm, om, P);
+    if (L.has_cache)
+      spark::prefill3_kernel<true><<<(unsigned)L.blocks, spark::kPfThreads, spark::kP2SmemBytes,
+                                     (cudaStream_t)stream>>>(L.qm, L.km, L.vm, L.kcm, L.vcm, L.om, L.P);
     else
-      spark::prefill3_kernel<false><<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes,
-                                      (cudaStream_t)stream>>>(qm, km, vm, kcm, vcm, om, P);
+      spark::prefill3_kernel<false><<<(unsigned)L.blocks, spark::kPfThreads, spark::kP2SmemBytes,
+                                      (cudaStream_t)stream>>>(L.qm, L.km, L.vm, L.kcm, L.vcm, L.om, L.P);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prefill3_kernel launch");
   } else {
     // clusters of two blocks (an SM pair): two query heads of a KV group, same query tile
-    spark::prefill2_kernel<false><<<(unsigned)blocks, spark::kPfThreads, spark::kP2SmemBytes,
-                                    (cudaStream_t)stream>>>(qm, km, vm, kcm, vcm, om, P);
+    spark::prefill2_kernel<false><<<(unsigned)L.blocks, spark::kPfThreads, spark::kP2SmemBytes,
+                                    (cudaStream_t)stream>>>(L.qm, L.km, L.vm, L.kcm, L.vcm, L.om, L.P);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prefill2_kernel launch");
   }
+  return SPARK_OK;
+}
+
+int spark_attn_prefill(void* out, const void* q, const void* k, const void* v, const void* gate,
+                       const void* k_cache, const void* v_cache, int cap, int B, int T, long long q_sB,
+                       long long q_sT, long long kv_sB, long long kv_sT, const int* pos0, const spark_layer_cfg* cfg,
+                       unsigned flags, void* stream) {
+  PrefillPlan L;
+  int rc = prefill_prepare(L, out, q, k, v, gate, k_cache, v_cache, cap, B, T, q_sB, q_sT, kv_sB, kv_sT, pos0, cfg,
+                           flags);
+  if (rc) return rc;
+  if ((rc = prefill_launch(L, stream))) return rc;
   if (!(flags & SPARK_APPEND_FUSED)) return SPARK_OK;
   // the chunk's k (rotated) and v into the cache, after the attention on the same stream: a sliding
   // ring's rows are overwritten only once the attention has read them as history
   return append_impl(dense_view((void*)k_cache, (void*)v_cache, nullptr, nullptr, cap), k, v, B, T, pos0, cfg, 0,
-                     stream, nullptr, 0, 0, kv_sB, kv_sT);
+                     stream, nullptr, 0, 0, L.kv_sB, L.kv_sT);
 }
 
 size_t spark_prefill_q8_workspace_bytes(int B, int cap, const spark_layer_cfg* cfg) {
@@ -1011,22 +1039,24 @@ int spark_attn_prefill_q8(void* out, const void* q, const void* k, const void* v
   if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(k_scales) || !aligned16(v_scales) ||
       !aligned16(workspace))
     return fail(SPARK_ERR_INVALID_ARG, "codes, scales and workspace must be 16-byte aligned");
-  int dev;
-  if ((rc = device_ready(&dev))) return rc;
+  const CacheView q8c = dense_view((void*)k_codes, (void*)v_codes, (void*)k_scales, (void*)v_scales, cap);
+  if ((rc = check_view(q8c, cfg))) return rc;
   __nv_bfloat16* hk = (__nv_bfloat16*)workspace;
   __nv_bfloat16* hv = hk + need / 4;
+  // the bf16 prefill over the workspace, checked and set up before anything is launched
+  PrefillPlan L;
+  if ((rc = prefill_prepare(L, out, q, k, v, gate, hk, hv, cap, B, T, q_sB, q_sT, kv_sB, kv_sT, pos0, cfg,
+                            flags & ~SPARK_APPEND_FUSED)))
+    return rc;
   spark::q8_history_kernel<<<dim3((unsigned)((cap + 3) / 4), SPARK_N_KV_HEADS, (unsigned)B), 256, 0,
                              (cudaStream_t)stream>>>((const uint8_t*)k_codes, (const __half*)k_scales,
                                                      (const uint8_t*)v_codes, (const __half*)v_scales, cap, pos0,
                                                      hk, hv);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "q8_history_kernel launch");
-  rc = spark_attn_prefill(out, q, k, v, gate, hk, hv, cap, B, T, q_sB, q_sT, kv_sB, kv_sT, pos0, cfg,
-                          flags & ~SPARK_APPEND_FUSED, stream);
-  if (rc || !(flags & SPARK_APPEND_FUSED)) return rc;
+  if ((rc = prefill_launch(L, stream)) || !(flags & SPARK_APPEND_FUSED)) return rc;
   // the chunk's k (rotated) and v, quantised into the 8-bit cache after the attention
-  return append_impl(dense_view((void*)k_codes, (void*)v_codes, (void*)k_scales, (void*)v_scales, cap), k, v, B, T,
-                     pos0, cfg, 0, stream, nullptr, 0, 0, kv_sB, kv_sT);
+  return append_impl(q8c, k, v, B, T, pos0, cfg, 0, stream, nullptr, 0, 0, L.kv_sB, L.kv_sT);
 }
 
 int spark_rope_apply_varlen(void* x, int H, const int* cu_seqlens, int max_seqlen, const int* pos0, int B,

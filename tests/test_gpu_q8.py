@@ -326,3 +326,13 @@ def test_prefill_q8_host_checks():
         sa.spark_attn_prefill_q8(*args, d["ws"][:-16])              # workspace too small
     with pytest.raises(sa.SparkError):
         sa.spark_attn_prefill_q8(*args, d["ws"], flags=0x80)
+    # an argument error of the prefill part (q's token stride not a multiple of 8 elements) is found
+    # before anything is launched: the workspace is left as it was
+    ws = d["ws"]
+    ws.fill_(7)
+    q_bad = torch.zeros(1, 64, 16 * 256 + 4, dtype=torch.bfloat16, device="cuda")[..., :16 * 256].view(1, 64, 16, 256)
+    with pytest.raises(sa.SparkError) as e:
+        sa.spark_attn_prefill_q8(out, q_bad, *args[2:], ws)
+    assert e.value.status == -1
+    torch.cuda.synchronize()
+    assert bool((ws == 7).all())
